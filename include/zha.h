@@ -1,0 +1,254 @@
+/*
+ * zha.h -- C ABI of libzha, the sm_100a (B200) decode path of Zyphra
+ * Hierarchical Attention (ZHA): a tree of key summaries over the KV cache of
+ * one GQA attention layer, top-p routing down that tree, and exact attention
+ * over the routed tokens.
+ *
+ * Method (page "Zyphra AI Introduces Zyphra Hierarchical Attention (ZHA)",
+ * MarkTechPost article):
+ *   - section "Building the tree": keys are cut into contiguous chunks of c;
+ *     each chunk is summarised against R learned reference queries as tangent
+ *     planes of the chunk's log attention mass; summaries are grouped and
+ *     summarised again, level by level; a node's estimate is the max over its
+ *     planes.
+ *   - section "How does top-p routing pick tokens": a decode query scores the
+ *     top-level nodes, keeps the smallest set that holds a fraction p of the
+ *     estimated mass, expands only their children, and repeats down to the
+ *     raw KV; token 0 is always kept as the attention sink.
+ *   - explainer widget, step 5: exact attention over the selected raw KV, the
+ *     sink and the current chunk; the full KV cache stays stored.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *     allocates no device memory; scratch lives in a caller-provided
+ *     workspace of zha_workspace_bytes() bytes, the tree in a caller-provided
+ *     buffer of zha_tree_bytes() bytes. Pointers must be 16-byte aligned.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = legacy default stream) and never synchronises.
+ *   - Argument errors are returned synchronously and nothing is enqueued.
+ *     Errors the GPU detects (a length beyond max_len, a leaf index out of
+ *     range, a capacity overflow) are written to the caller's int32 word
+ *     `dev_status` (first error wins; the caller zeroes it and reads it after
+ *     a sync); kernels never trap.
+ *   - Layouts (row-major, innermost last), dtype = cfg->dtype for
+ *     K, V, q, refs, out, k_new, v_new:
+ *       K, V   [batch][n_kv_heads][max_len][head_dim]
+ *       q      [batch][n_q_heads][head_dim]
+ *       refs   [n_kv_heads][n_refs][head_dim]
+ *       out    [batch][n_q_heads][head_dim]
+ *       lens   [batch] int32: tokens currently in each sequence's cache
+ *     Query head h uses KV head h / G, G = n_q_heads / n_kv_heads.
+ *   - Supported: head_dim in {64, 128}; chunk a power of two in [2, 256];
+ *     1 <= levels <= ZHA_MAX_LEVELS; 1 <= n_refs <= 32; G <= 16;
+ *     dtype BF16 or F32. Anything else returns ZHA_ERR_UNSUPPORTED.
+ */
+#ifndef ZHA_H
+#define ZHA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ZHA_API __attribute__((visibility("default")))
+#else
+#define ZHA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum zha_status {
+    ZHA_OK = 0,
+    ZHA_ERR_INVALID_ARG = 1,
+    ZHA_ERR_UNSUPPORTED = 2,
+    ZHA_ERR_CAPACITY = 3,
+    ZHA_ERR_CUDA = 4,
+    ZHA_ERR_TIMEOUT = 5
+} zha_status;
+
+enum { ZHA_BF16 = 0, ZHA_F32 = 1 };
+
+/* cfg->flags */
+enum {
+    /* current chunk = only the incomplete tail [c*floor(N/c), N) instead of the
+     * chunk holding the newest token [c*floor((N-1)/c), N) */
+    ZHA_FLAG_TAIL_ONLY = 1
+};
+
+#define ZHA_MAX_LEVELS 8
+
+typedef struct zha_config {
+    int32_t batch;       /* B */
+    int32_t n_q_heads;   /* Hq */
+    int32_t n_kv_heads;  /* Hkv; one tree per (sequence, KV head) */
+    int32_t head_dim;    /* d */
+    int32_t chunk;       /* c: keys per leaf, children per parent */
+    int32_t levels;      /* L: levels of the tree (1 = leaves only) */
+    int32_t n_refs;      /* R: reference queries per KV head */
+    int32_t dtype;       /* ZHA_BF16 or ZHA_F32 */
+    int64_t max_len;     /* token capacity of K/V per sequence */
+    float scale;         /* s; <= 0 selects 1/sqrt(head_dim) */
+    int32_t flags;       /* ZHA_FLAG_* */
+    int32_t attn_splits; /* split-K CTAs per (sequence, KV head); 0 = auto */
+    int32_t reserved[3];
+} zha_config;
+
+/*
+ * Routed selection of every (sequence, KV head) group: the union over the
+ * group's G query heads of the kept leaf chunks, ascending, with one bit per
+ * query head saying which heads keep each chunk. All device pointers.
+ *   leaf_idx  [batch][n_kv_heads][cap1] int32   (cap1 = max_len / chunk)
+ *   head_mask [batch][n_kv_heads][cap1] uint32  bit j: query head g*G+j
+ *   count     [batch][n_kv_heads]       int32   entries in use
+ *   level_kept [batch][n_q_heads][levels] int32 optional (NULL = not written):
+ *             nodes kept by each query head at each level (index l-1)
+ */
+typedef struct zha_selection {
+    int32_t *leaf_idx;
+    uint32_t *head_mask;
+    int32_t *count;
+    int32_t *level_kept;
+} zha_selection;
+
+/* Byte offsets, inside the workspace, of the per-level routing state of the
+ * last zha_route / zha_decode call (valid until the workspace is reused):
+ *   cand_idx  [batch][n_kv_heads][cap_l] int32    candidate node indices, ascending
+ *   cand_mask [batch][n_kv_heads][cap_l] uint32   heads for which it is a candidate
+ *   scores    [batch][n_kv_heads][G][cap_l] float estimate max_r(s q.mu_r + b_r)
+ *   kept_mask [batch][n_kv_heads][cap_l] uint32   heads that kept it
+ *   count     [batch][n_kv_heads] int32           candidates in use
+ * cap_l = nodes at level l for max_len tokens. */
+typedef struct zha_level_view {
+    int64_t cap;
+    size_t cand_idx, cand_mask, scores, kept_mask, count;
+} zha_level_view;
+
+/* Message for a status code (static string). */
+ZHA_API const char *zha_status_string(zha_status s);
+
+/* ZHA_OK if the configuration is supported; otherwise why not. */
+ZHA_API zha_status zha_check_config(const zha_config *cfg);
+
+/* Nodes at `level` (1 = leaf chunks) for n tokens: n_1 = floor(n / c)
+ * (only complete chunks enter the tree), n_l = ceil(n_{l-1} / c). */
+ZHA_API int64_t zha_level_nodes(const zha_config *cfg, int64_t n_tokens, int32_t level);
+
+/* Bytes of the tree buffer for cfg->max_len tokens per sequence, and the
+ * byte offsets of level l's arrays inside it:
+ *   mu   [batch][n_kv_heads][cap_l][n_refs][head_dim]  dtype (summary keys)
+ *   bias [batch][n_kv_heads][cap_l][n_refs]            float (plane offsets)
+ * A node's plane r evaluates to s*q.mu_r + bias_r. */
+ZHA_API size_t zha_tree_bytes(const zha_config *cfg);
+ZHA_API zha_status zha_tree_level_offsets(const zha_config *cfg, int32_t level, size_t *mu_off,
+                                  size_t *bias_off);
+
+/* Bytes of scratch every call below may use (routing state + split-K partials). */
+ZHA_API size_t zha_workspace_bytes(const zha_config *cfg);
+ZHA_API zha_status zha_workspace_level_view(const zha_config *cfg, int32_t level, zha_level_view *v);
+
+/*
+ * zha_tree_build -- summarise the first lens[b] tokens of every sequence
+ * from scratch (section "Building the tree").
+ * Leaf j, reference r, keys k_t of chunk j:  l_t = s r.k_t,
+ * F = log sum_t e^{l_t}, w_t = e^{l_t - F}, mu_r = sum_t w_t k_t,
+ * bias_r = F - s r.mu_r. A parent applies the same rule to its existing
+ * children, child i entering as the point mu_{i,r} with log-weight
+ * bias_{i,r}; the rightmost node of a level may have fewer than c children.
+ * mu is rounded to dtype once computed; parents read the rounded children.
+ */
+ZHA_API zha_status zha_tree_build(const zha_config *cfg, void *tree, const void *K, const void *refs,
+                          const int32_t *lens, int32_t *dev_status, void *stream);
+
+/*
+ * zha_tree_append -- the caller has written n_new more tokens into K and
+ * lens[b] already counts them: bring the tree from lens[b]-n_new to lens[b]
+ * tokens (the chunks that completed, then every ancestor from the first
+ * changed node to the right end of each level). Bit-identical to
+ * zha_tree_build at the new lengths. Tree depth is fixed by cfg->levels.
+ */
+ZHA_API zha_status zha_tree_append(const zha_config *cfg, void *tree, const void *K, const void *refs,
+                           const int32_t *lens, int32_t n_new, int32_t *dev_status, void *stream);
+
+/*
+ * zha_route -- top-p routing of every query head (section "How does top-p
+ * routing pick tokens"). Per query head, level L down to 1: the candidates'
+ * estimates E = max_r(s q.mu_r + bias_r) are turned into masses e^{E-max};
+ * with the candidates ordered by (E descending, node index ascending) the
+ * shortest prefix whose running mass reaches p times the total is kept; the
+ * existing children of kept nodes are the next level's candidates. Level L's
+ * candidates are all its nodes. p_levels[l-1] (host array, L entries) is the
+ * fraction at level l; a value >= 1 keeps every candidate; values <= 0 or
+ * NaN are ZHA_ERR_INVALID_ARG. Result in *sel (see zha_selection).
+ */
+ZHA_API zha_status zha_route(const zha_config *cfg, const void *tree, const void *q, const int32_t *lens,
+                     const float *p_levels, const zha_selection *sel, void *workspace,
+                     int32_t *dev_status, void *stream);
+
+/*
+ * zha_sparse_attn -- exact softmax attention of every query head over its
+ * token set {0} U {tokens of the leaf chunks of *sel whose head bit is set}
+ * U current chunk, with the current chunk [c*floor((N-1)/c), N)
+ * (ZHA_FLAG_TAIL_ONLY: [c*floor(N/c), N)), N = lens[b]:
+ *   out_h = sum_t softmax_t(s q_h.k_t) v_t   (fp32 accumulation).
+ * Leaf indices at or beyond floor(N/c) set ZHA_ERR_INVALID_ARG in dev_status
+ * and are skipped. `sel` may come from zha_route or from the caller.
+ */
+ZHA_API zha_status zha_sparse_attn(const zha_config *cfg, const void *q, const void *K, const void *V,
+                           const int32_t *lens, const zha_selection *sel, void *out,
+                           void *workspace, int32_t *dev_status, void *stream);
+
+/*
+ * zha_decode -- one decode step of the layer: write k_new/v_new
+ * ([batch][n_kv_heads][head_dim]) at position lens[b] of K/V, increment
+ * lens[b], extend the tree (zha_tree_append with n_new = 1), route the
+ * queries q, and attend (zha_sparse_attn). lens is updated on the device.
+ * Selection written to *sel.
+ */
+ZHA_API zha_status zha_decode(const zha_config *cfg, void *tree, void *K, void *V, const void *refs,
+                      int32_t *lens, const void *q, const void *k_new, const void *v_new,
+                      const float *p_levels, const zha_selection *sel, void *out,
+                      void *workspace, int32_t *dev_status, void *stream);
+
+/*
+ * zha_dense_decode -- the comparison kernel: exact softmax attention of every
+ * query head over all lens[b] tokens (split-K flash decoding, same numerics
+ * as zha_sparse_attn).
+ */
+ZHA_API zha_status zha_dense_decode(const zha_config *cfg, const void *q, const void *K, const void *V,
+                            const int32_t *lens, void *out, void *workspace, int32_t *dev_status,
+                            void *stream);
+
+/*
+ * zha_topp_select -- one level of the routing selection on given scores,
+ * for n_sets independent candidate sets (section "How does top-p routing pick
+ * tokens"): set i has counts[i] candidates whose fp32 scores are
+ * scores[i*stride .. i*stride+counts[i]) in ascending node order; kept[i*stride+j]
+ * (uint8) is set to 1 for the kept ones and 0 otherwise. Same arithmetic as
+ * the selection inside zha_route. p as in zha_route. Device pointers.
+ */
+ZHA_API zha_status zha_topp_select(const float *scores, const int32_t *counts, int32_t n_sets,
+                           int64_t stride, float p, uint8_t *kept, int32_t *dev_status,
+                           void *stream);
+
+
+/*
+ * Instrumentation (no counterpart on the pages; for measurement only).
+ * zha_launch_count: kernels this library has launched since it was loaded.
+ * zha_profile_enable(1): from now on every kernel launch is bracketed by a
+ *   pair of CUDA events recorded on its stream; (0) stops recording.
+ * zha_profile_read: waits for the recorded events and returns, per kernel
+ *   name (names separated by '\n' in `names`, at most max_kernels entries),
+ *   the summed duration in ms and the number of launches; then clears the
+ *   record. Returns the number of kernel names written, or -1 on error.
+ */
+ZHA_API uint64_t zha_launch_count(void);
+ZHA_API zha_status zha_profile_enable(int32_t on);
+ZHA_API int32_t zha_profile_read(char *names, int32_t names_len, double *ms, int64_t *launches,
+                                 int32_t max_kernels);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZHA_H */

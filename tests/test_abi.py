@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/zha.h declares, and its layout queries agree with the
+rules they document (and with the oracle's level sizes)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "zha.h")).read()
+    return sorted(set(re.findall(r"^ZHA_API\s+[\w\s\*]+?\b(zha_\w+)\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def zha():
+    from tree_indexed_sparse_02_b200 import build
+    build.build()
+    from tree_indexed_sparse_02_b200 import zha as z
+    return z
+
+
+def test_header_declares_the_hot_path(zha):
+    names = declared_functions()
+    for required in ("zha_tree_build", "zha_tree_append", "zha_route", "zha_sparse_attn", "zha_decode",
+                     "zha_dense_decode", "zha_topp_select"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(zha):
+    lib = ctypes.CDLL(zha.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_config_checks(zha):
+    zha.config(1, 2, 1, 64, 4, 3, 16, "f32", 4096)
+    bad = [dict(head_dim=96), dict(chunk=3), dict(chunk=512), dict(levels=9), dict(n_refs=33),
+           dict(n_q_heads=34, n_kv_heads=2), dict(n_q_heads=3, n_kv_heads=2)]
+    for kw in bad:
+        args = dict(batch=1, n_q_heads=2, n_kv_heads=1, head_dim=64, chunk=4, levels=3, n_refs=16,
+                    dtype="f32", max_len=4096)
+        args.update(kw)
+        with pytest.raises(zha.ZhaError):
+            zha.config(**args)
+
+
+def test_level_sizes_match_oracle(zha, orc):
+    cfg = zha.config(1, 8, 1, 128, 4, 6, 16, "bf16", 1 << 20)
+    for n in (0, 1, 3, 4, 5, 4095, 4096, 4097, 262144, 262147, 1 << 20):
+        for level in range(1, 7):
+            assert zha.level_nodes(cfg, n, level) == orc.level_nodes(n, 4, level)
+
+
+def test_tree_and_workspace_layout(zha):
+    cfg = zha.config(4, 32, 4, 128, 4, 6, 16, "bf16", 262144 + 512)
+    total = zha.tree_bytes(cfg)
+    prev_end = 0
+    for level in range(1, 7):
+        mu_off, b_off = zha.tree_level_offsets(cfg, level)
+        cap = zha.level_nodes(cfg, cfg.max_len, level)
+        assert mu_off % 256 == 0 and b_off % 256 == 0
+        assert mu_off >= prev_end
+        assert b_off >= mu_off + 4 * 4 * cap * 16 * 128 * 2
+        prev_end = b_off + 4 * 4 * cap * 16 * 4
+    assert total >= prev_end
+    ws = zha.workspace_bytes(cfg)
+    for level in range(1, 7):
+        v = zha.workspace_level_view(cfg, level)
+        assert v.cap == zha.level_nodes(cfg, cfg.max_len, level)
+        for off in (v.cand_idx, v.cand_mask, v.scores, v.kept_mask, v.count):
+            assert off % 256 == 0 and off < ws
+
+
+def test_invalid_arguments_are_rejected_before_launch(zha):
+    """Argument errors come back synchronously; these calls launch nothing."""
+    cfg = zha.config(1, 2, 1, 64, 4, 3, 16, "f32", 4096)
+    L = zha.lib()
+    assert L.zha_tree_build(ctypes.byref(cfg), None, None, None, None, None, None) == 1
+    p = (ctypes.c_float * 3)(0.9, 0.0, 0.9)       # p <= 0 at one level
+    sel = zha.Selection(16, 16, 16, None)
+    assert L.zha_route(ctypes.byref(cfg), ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), p,
+                       ctypes.byref(sel), ctypes.c_void_p(16), None, None) == 1
+    p = (ctypes.c_float * 3)(0.9, float("nan"), 0.9)
+    assert L.zha_route(ctypes.byref(cfg), ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), p,
+                       ctypes.byref(sel), ctypes.c_void_p(16), None, None) == 1
+    assert L.zha_topp_select(None, None, 1, 8, ctypes.c_float(0.5), None, None, None) == 1
+    assert L.zha_topp_select(None, None, 0, 8, ctypes.c_float(0.5), None, None, None) == 0
+    # misaligned pointer
+    assert L.zha_dense_decode(ctypes.byref(cfg), ctypes.c_void_p(18), ctypes.c_void_p(16), ctypes.c_void_p(16),
+                              ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), None, None) == 1
+    assert L.zha_status_string(3).decode().startswith("capacity")

@@ -1,0 +1,141 @@
+"""Shared helpers of the GPU parity tests: run the oracle on the same inputs
+the CUDA path gets, and compare the two the way the method allows."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import zha_oracle as orc
+from tree_indexed_sparse_02_b200.inputs import Workload, make_inputs
+
+# tolerances, err = max|gpu - oracle| / max(max|oracle|, 1)
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def rel_err(gpu, ref) -> float:
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    if r.size == 0:
+        return 0.0
+    return float(np.max(np.abs(g - r)) / max(float(np.max(np.abs(r))), 1.0))
+
+
+def np64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def storage(w: Workload) -> str:
+    return "bf16" if w.dtype == "bf16" else "f32"
+
+
+def make_cfg(zha, w: Workload, cap: int, flags: int = 0, splits: int = 0):
+    return zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs,
+                      w.dtype, cap, flags=flags, attn_splits=splits)
+
+
+def to_device(inp, device="cuda"):
+    from tree_indexed_sparse_02_b200.inputs import Inputs
+    return Inputs(K=inp.K.to(device), V=inp.V.to(device), q=inp.q.to(device), refs=inp.refs.to(device),
+                  lens=inp.lens.to(device), needle_pos=inp.needle_pos)
+
+
+def oracle_tree(w: Workload, inp, b: int, kvh: int, N: int, s: float, cap_tokens: int | None = None):
+    K = np64(inp.K[b, kvh, :max(N, 1)])
+    refs = np64(inp.refs[kvh])
+    return orc.build_tree(K, refs, N, w.chunk, w.levels, s, storage=storage(w),
+                          cap_tokens=max(cap_tokens or N, 1))
+
+
+def gpu_level_candidates(state, b, kvh, h, n_l):
+    """GPU candidates / kept / scores of query head h (within its group) as arrays over nodes."""
+    cnt = int(state["count"][b, kvh])
+    idx = state["cand_idx"][b, kvh, :cnt].cpu().numpy().astype(np.int64)
+    cm = state["cand_mask"][b, kvh, :cnt].cpu().numpy().astype(np.uint32)
+    km = state["kept_mask"][b, kvh, :cnt].cpu().numpy().astype(np.uint32)
+    sc = state["scores"][b, kvh, h, :cnt].cpu().numpy().astype(np.float64)
+    bit = np.uint32(1 << h)
+    cand = np.zeros(n_l, dtype=bool)
+    kept = np.zeros(n_l, dtype=bool)
+    score = np.full(n_l, -np.inf)
+    member = (cm & bit) != 0
+    assert np.all(np.diff(idx) > 0), "candidate list must be strictly ascending"
+    assert idx.size == 0 or (idx.min() >= 0 and idx.max() < n_l)
+    cand[idx[member]] = True
+    kept[idx[member & ((km & bit) != 0)]] = True
+    assert not np.any((km & ~cm) != 0), "kept by a head that did not have it as a candidate"
+    score[idx] = sc
+    return cand, kept, score
+
+
+def compare_routing(route_o, states, b, kvh, G, N, w: Workload, p_levels):
+    """Level-by-level comparison of one group's routing. Flips (nodes kept by
+    one side only) are allowed only where the oracle's running mass before the
+    node is within the score-error band of p. Returns (flipped_heads, max score err)."""
+    L = w.levels
+    flipped = set()
+    worst = 0.0
+    for h in range(G):
+        diverged = False
+        for level in range(L, 0, -1):
+            n_l = orc.level_nodes(N, w.chunk, level)
+            cand_g, kept_g, score_g = gpu_level_candidates(states[level], b, kvh, h, n_l)
+            cand_o = route_o.cand[level - 1][h]
+            kept_o = route_o.kept[level - 1][h]
+            if not diverged:
+                assert np.array_equal(cand_g, cand_o), (h, level)
+            common = cand_g & cand_o
+            if not common.any():
+                continue
+            so = route_o.score[level - 1][h][common]
+            sg = score_g[common]
+            err = float(np.max(np.abs(sg - so)))
+            worst = max(worst, err / max(1.0, float(np.max(np.abs(so)))))
+            flips = np.nonzero((kept_g != kept_o) & common)[0]
+            if flips.size:
+                p = float(p_levels[level - 1])
+                band = 4.0 * err + 1e-5
+                cb = route_o.cumb[level - 1][h]
+                for n in flips:
+                    assert abs(cb[n] - p) <= band, (
+                        f"head {h} level {level} node {n}: cum {cb[n]:.6f} vs p {p} (band {band:.2e})")
+                diverged = True
+                flipped.add(h)
+    return flipped, worst
+
+
+def selection_to_masks(sel, b, kvh, G, N, c, tail_only=False):
+    """Per-head attended-token masks implied by a selection (via the oracle's token rule)."""
+    cnt = int(sel["count"][b, kvh])
+    idx = sel["leaf_idx"][b, kvh, :cnt].cpu().numpy().astype(np.int64)
+    hm = sel["head_mask"][b, kvh, :cnt].cpu().numpy().astype(np.uint32)
+    n1 = N // c
+    out = []
+    for h in range(G):
+        kl = np.zeros(n1, dtype=bool)
+        kl[idx[(hm >> np.uint32(h)) & np.uint32(1) != 0]] = True
+        out.append(orc.token_set(N, c, kl, tail_only))
+    return out
+
+
+def scale_of(w: Workload) -> float:
+    return 1.0 / math.sqrt(w.head_dim)
+
+
+def small_workloads():
+    """Parity cases small enough for the oracle: several tiles and ragged tails."""
+    from tree_indexed_sparse_02_b200.inputs import TINY_F32, WIDE_32K
+    deep = Workload("deep-small bf16 B=2 c=4 L=4", 2, 16, 2, 128, 3001, 4, 4, 16, 0.95, 16, "bf16", 11)
+    g16 = Workload("G16 R32 d64 c=8 L=3", 1, 32, 2, 64, 2500, 8, 3, 32, 0.9, 8, "bf16", 12)
+    r1 = Workload("R1 c=8 p=0.75", 1, 8, 1, 128, 5003, 8, 4, 1, 0.75, 4, "bf16", 13)
+    return [TINY_F32, deep, g16, r1, WIDE_32K]
+
+
+def build_case(zha, w: Workload, extra_cap: int = 64, lens=None, device="cuda", gen_device="cpu"):
+    cap = w.context + extra_cap
+    inp = make_inputs(w, device=gen_device, capacity=cap, lens=lens)
+    dev = to_device(inp, device)
+    cfg = make_cfg(zha, w, cap)
+    buf = zha.Buffers(cfg, device=device)
+    return cfg, inp, dev, buf

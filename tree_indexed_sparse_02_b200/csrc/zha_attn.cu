@@ -1,0 +1,481 @@
+// zha_attn.cu -- exact attention over the routed tokens (and the dense
+// comparison kernel), split-K flash decoding with a log-sum-exp merge.
+//
+// Page "Zyphra AI Introduces Zyphra Hierarchical Attention (ZHA)", explainer
+// widget step 5: exact attention over the selected raw KV entries plus the
+// first token (sink) and the current chunk; section "How does top-p routing
+// pick tokens": the first token is always kept.
+//
+// Every (sequence, KV head) group streams the union of its heads' tokens
+// once; each token carries the bit mask of query heads that attend to it, so
+// one K/V read serves all G heads of the group. The token stream of a group
+// is: the kept leaf chunks (ascending), then the sink if no kept chunk holds
+// it, then the current chunk if no kept chunk is it.
+//
+// bf16: per warp, 16 tokens at a time on tensor cores (mma.sync m16n8k16):
+// S = Q K^T with the heads as the 16 rows, online softmax in registers in
+// base 2, then O += P V with P taken straight from the S accumulators. K and V
+// rows go global -> registers in fully used 32-byte sectors (coordinates of
+// the QK product are permuted identically in Q and K; the value coordinates
+// each lane owns are a contiguous block).
+// fp32: one token per lane on CUDA cores, same partial format.
+#include "zha_common.cuh"
+
+namespace zha {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kAttnWarps = 4;
+
+// Which cache position virtual token v of a group is, and which heads see it.
+struct TokenPlan {
+    int64_t N, cur_start, n1;
+    int64_t nsel, sel_tokens;  // kept leaf chunks, their tokens
+    int64_t a_len;             // sink span [0, a_len)
+    int64_t b_start, b_len;    // current-chunk span
+    int64_t nv;                // stream length
+    int c;
+    uint32_t all;
+    const int32_t *leaf;
+    const uint32_t *hmask;
+
+    __device__ __forceinline__ void at(int64_t v, int64_t &pos, uint32_t &mask,
+                                       int32_t *status) const {
+        if (v < sel_tokens) {
+            const int64_t e = v / c;
+            const int64_t lf = leaf[e];
+            if (lf < 0 || lf >= n1) {
+                set_status(status, ZHA_ERR_INVALID_ARG);
+                pos = 0;
+                mask = 0u;
+                return;
+            }
+            pos = lf * c + (v - e * c);
+            mask = hmask[e] | ((pos == 0 || pos >= cur_start) ? all : 0u);
+            return;
+        }
+        v -= sel_tokens;
+        if (v < a_len) {
+            pos = 0;
+            mask = all;
+            return;
+        }
+        v -= a_len;
+        if (v < b_len) {
+            pos = b_start + v;
+            mask = all;
+            return;
+        }
+        pos = 0;
+        mask = 0u;
+    }
+};
+
+__device__ __forceinline__ TokenPlan make_plan(const Geo &g, const int32_t *lens, int grp,
+                                               const zha_selection *sel, bool dense,
+                                               int32_t *status) {
+    TokenPlan tp{};
+    const int b = grp / g.Hkv;
+    int64_t N = lens[b];
+    if (N < 0 || N > g.max_len) {
+        set_status(status, ZHA_ERR_CAPACITY);
+        N = 0;
+    }
+    tp.N = N;
+    tp.c = g.c;
+    tp.all = g.G >= 32 ? 0xffffffffu : ((1u << g.G) - 1u);
+    tp.n1 = N / g.c;
+    if (dense || N == 0) {
+        tp.b_start = 0;
+        tp.b_len = N;
+        tp.cur_start = 0;
+        tp.nv = N;
+        return tp;
+    }
+    tp.cur_start = current_chunk_start(N, g.c, g.flags);
+    int64_t ns = sel->count[grp];
+    if (ns < 0 || ns > g.cap[1]) {
+        set_status(status, ZHA_ERR_INVALID_ARG);
+        ns = 0;
+    }
+    tp.leaf = sel->leaf_idx + grp * g.cap[1];
+    tp.hmask = sel->head_mask + grp * g.cap[1];
+    tp.nsel = ns;
+    tp.sel_tokens = ns * g.c;
+    const bool has_leaf0 = ns > 0 && tp.leaf[0] == 0;
+    const bool cur_complete = tp.cur_start + g.c <= N;
+    const bool cur_covered = cur_complete && ns > 0 && (int64_t)tp.leaf[ns - 1] * g.c == tp.cur_start;
+    tp.a_len = (!has_leaf0 && tp.cur_start > 0) ? 1 : 0;
+    tp.b_start = tp.cur_start;
+    tp.b_len = cur_covered ? 0 : N - tp.cur_start;
+    tp.nv = tp.sel_tokens + tp.a_len + tp.b_len;
+    return tp;
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Partials: ml[((grp*S + s)*G + h)*2 + {0,1}] = (max in log2 units, sum),
+// o[((grp*S + s)*G + h)*D + dim] (unnormalised).
+template <int D>
+__global__ void __launch_bounds__(kAttnWarps * 32)
+attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
+                const int32_t *lens, zha_selection sel, int dense, float *part_ml, float *part_o,
+                int32_t *status) {
+    constexpr int KP = D / 32;      // k-pairs of the QK product
+    constexpr int NJ = D / 8;       // n-tiles of the PV product
+    constexpr int DW = D / 8;       // value coordinates per lane
+    __shared__ float sm_m[kAttnWarps][16], sm_l[kAttnWarps][16];
+    __shared__ float sm_o[kAttnWarps][16][D + 4];
+
+    const int grp = blockIdx.y, split = blockIdx.x, S = gridDim.x;
+    const int b = grp / g.Hkv, kvh = grp % g.Hkv;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gq = lane >> 2, t = lane & 3;
+    const TokenPlan tp = make_plan(g, lens, grp, &sel, dense != 0, status);
+    const __nv_bfloat16 *Kg = K + (int64_t)grp * g.max_len * D;
+    const __nv_bfloat16 *Vg = V + (int64_t)grp * g.max_len * D;
+
+    // Q as the A operand: rows gq and gq+8 are heads of this group (rows >= G are zero)
+    uint32_t qa[KP][4], qb[KP][4];  // k16 steps 2kp and 2kp+1
+    const int h0 = gq, h1 = gq + 8;
+#pragma unroll
+    for (int kp = 0; kp < KP; ++kp) {
+        uint4 w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
+        if (h0 < g.G) w0 = *reinterpret_cast<const uint4 *>(q + ((int64_t)b * g.Hq + kvh * g.G + h0) * D + kp * 32 + t * 8);
+        if (h1 < g.G) w1 = *reinterpret_cast<const uint4 *>(q + ((int64_t)b * g.Hq + kvh * g.G + h1) * D + kp * 32 + t * 8);
+        qa[kp][0] = w0.x; qa[kp][1] = w1.x; qa[kp][2] = w0.y; qa[kp][3] = w1.y;
+        qb[kp][0] = w0.z; qb[kp][1] = w1.z; qb[kp][2] = w0.w; qb[kp][3] = w1.w;
+    }
+
+    const float sl2 = g.s * kLog2e;
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    float o[NJ][4];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+
+    const int64_t W = (tp.nv + 15) / 16;
+    const int64_t w_lo = W * split / S, w_hi = W * (split + 1) / S;
+    for (int64_t wt = w_lo + warp; wt < w_hi; wt += kAttnWarps) {
+        const int64_t v0 = wt * 16;
+        // K rows this lane feeds to the QK product: tokens gq and 8+gq
+        int64_t pk0, pk1;
+        uint32_t mk0, mk1;
+        tp.at(v0 + gq, pk0, mk0, status);
+        tp.at(v0 + 8 + gq, pk1, mk1, status);
+        if (v0 + gq >= tp.nv) mk0 = 0u;
+        if (v0 + 8 + gq >= tp.nv) mk1 = 0u;
+        // tokens of this lane's S columns and V rows: 2t, 2t+1, 8+2t, 9+2t
+        int64_t pv[4];
+        uint32_t mv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t v = v0 + (u >> 1) * 8 + 2 * t + (u & 1);
+            tp.at(v, pv[u], mv[u], status);
+            if (v >= tp.nv) mv[u] = 0u;
+        }
+        uint4 kr0[KP], kr1[KP];
+#pragma unroll
+        for (int kp = 0; kp < KP; ++kp) {
+            kr0[kp] = *reinterpret_cast<const uint4 *>(Kg + pk0 * D + kp * 32 + t * 8);
+            kr1[kp] = *reinterpret_cast<const uint4 *>(Kg + pk1 * D + kp * 32 + t * 8);
+        }
+        uint4 vr[4][DW / 8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int x = 0; x < DW / 8; ++x)
+                vr[u][x] = *reinterpret_cast<const uint4 *>(Vg + pv[u] * D + gq * DW + x * 8);
+
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kp = 0; kp < KP; ++kp) {
+            mma16816(s0, qa[kp][0], qa[kp][1], qa[kp][2], qa[kp][3], kr0[kp].x, kr0[kp].y);
+            mma16816(s0, qb[kp][0], qb[kp][1], qb[kp][2], qb[kp][3], kr0[kp].z, kr0[kp].w);
+            mma16816(s1, qa[kp][0], qa[kp][1], qa[kp][2], qa[kp][3], kr1[kp].x, kr1[kp].y);
+            mma16816(s1, qb[kp][0], qb[kp][1], qb[kp][2], qb[kp][3], kr1[kp].z, kr1[kp].w);
+        }
+        // s0: (head gq, tok 2t), (gq, 2t+1), (gq+8, 2t), (gq+8, 2t+1); s1: same for tokens 8+
+        float x[2][4];  // [row][token u]
+        const uint32_t mrow[2] = {h0 < g.G ? (1u << h0) : 0u, h1 < g.G ? (1u << h1) : 0u};
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            x[r][0] = (mv[0] & mrow[r]) ? s0[2 * r + 0] * sl2 : -INFINITY;
+            x[r][1] = (mv[1] & mrow[r]) ? s0[2 * r + 1] * sl2 : -INFINITY;
+            x[r][2] = (mv[2] & mrow[r]) ? s1[2 * r + 0] * sl2 : -INFINITY;
+            x[r][3] = (mv[3] & mrow[r]) ? s1[2 * r + 1] * sl2 : -INFINITY;
+        }
+        float p[2][4];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            float mx = fmaxf(fmaxf(x[r][0], x[r][1]), fmaxf(x[r][2], x[r][3]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run[r], mx);
+            const float corr = (m_run[r] == -INFINITY) ? 0.f : exp2f(m_run[r] - m_new);
+            float ls = 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                p[r][u] = (x[r][u] == -INFINITY) ? 0.f : exp2f(x[r][u] - m_new);
+                ls += p[r][u];
+            }
+            l_run[r] = l_run[r] * corr + ls;
+            m_run[r] = m_new;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+                o[j][2 * r] *= corr;
+                o[j][2 * r + 1] *= corr;
+            }
+        }
+        const uint32_t pa0 = pack_bf16(p[0][0], p[0][1]);
+        const uint32_t pa1 = pack_bf16(p[1][0], p[1][1]);
+        const uint32_t pa2 = pack_bf16(p[0][2], p[0][3]);
+        const uint32_t pa3 = pack_bf16(p[1][2], p[1][3]);
+        // V as B: k = tokens (2t, 2t+1 | 8+2t, 9+2t), n = value coordinate gq*DW + j
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            const int x8 = j >> 3, wi = (j & 7) >> 1;
+            const uint32_t w0 = (&vr[0][x8].x)[wi], w1 = (&vr[1][x8].x)[wi];
+            const uint32_t w2 = (&vr[2][x8].x)[wi], w3 = (&vr[3][x8].x)[wi];
+            const uint32_t sel_lo = (j & 1) ? 0x7632u : 0x5410u;
+            const uint32_t b0 = __byte_perm(w0, w1, sel_lo);
+            const uint32_t b1 = __byte_perm(w2, w3, sel_lo);
+            mma16816(o[j], pa0, pa1, pa2, pa3, b0, b1);
+        }
+    }
+    // row sums across the 4 lanes of a row
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+    }
+    // o[j]: (row gq, coord (2t)*DW + j), (gq, (2t+1)*DW + j), (gq+8, ...), (gq+8, ...)
+    if (t == 0) {
+        sm_m[warp][gq] = m_run[0];
+        sm_m[warp][gq + 8] = m_run[1];
+        sm_l[warp][gq] = l_run[0];
+        sm_l[warp][gq + 8] = l_run[1];
+    }
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+        sm_o[warp][gq][(2 * t) * DW + j] = o[j][0];
+        sm_o[warp][gq][(2 * t + 1) * DW + j] = o[j][1];
+        sm_o[warp][gq + 8][(2 * t) * DW + j] = o[j][2];
+        sm_o[warp][gq + 8][(2 * t + 1) * DW + j] = o[j][3];
+    }
+    __syncthreads();
+    const int64_t pbase = ((int64_t)grp * S + split) * g.G;
+    for (int i = threadIdx.x; i < g.G * D; i += blockDim.x) {
+        const int h = i / D, dim = i % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, sm_m[w][h]);
+        float L = 0.f, acc = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kAttnWarps; ++w) {
+                if (sm_m[w][h] == -INFINITY) continue;
+                const float f = exp2f(sm_m[w][h] - M);
+                L += sm_l[w][h] * f;
+                acc += sm_o[w][h][dim] * f;
+            }
+        }
+        part_o[(pbase + h) * D + dim] = acc;
+        if (dim == 0) {
+            part_ml[(pbase + h) * 2 + 0] = M;
+            part_ml[(pbase + h) * 2 + 1] = L;
+        }
+    }
+}
+
+// CUDA-core variant (fp32 inputs, or any dtype for checking): one token per lane.
+template <typename T, int D>
+__global__ void __launch_bounds__(kAttnWarps * 32)
+attn_simt_kernel(Geo g, const T *q, const T *K, const T *V, const int32_t *lens,
+                 zha_selection sel, int dense, float *part_ml, float *part_o, int32_t *status) {
+    constexpr int DL = D / 32;
+    __shared__ float qs[16][D];
+    __shared__ float sm_m[kAttnWarps][16], sm_l[kAttnWarps][16];
+    __shared__ float sm_o[kAttnWarps][16][D];
+    const int grp = blockIdx.y, split = blockIdx.x, S = gridDim.x;
+    const int b = grp / g.Hkv, kvh = grp % g.Hkv;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int G = g.G;
+    const TokenPlan tp = make_plan(g, lens, grp, &sel, dense != 0, status);
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x)
+        qs[i / D][i % D] = to_f32(q[((int64_t)b * g.Hq + kvh * G + i / D) * D + i % D]);
+    __syncthreads();
+    const T *Kg = K + (int64_t)grp * g.max_len * D;
+    const T *Vg = V + (int64_t)grp * g.max_len * D;
+    const float sl2 = g.s * kLog2e;
+    float m_run[16], l_run[16], o[16][DL];
+#pragma unroll
+    for (int h = 0; h < 16; ++h) {
+        m_run[h] = -INFINITY;
+        l_run[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) o[h][e] = 0.f;
+    }
+    const int64_t W = (tp.nv + 31) / 32;
+    const int64_t w_lo = W * split / S, w_hi = W * (split + 1) / S;
+    for (int64_t wt = w_lo + warp; wt < w_hi; wt += kAttnWarps) {
+        const int64_t v = wt * 32 + lane;
+        int64_t pos;
+        uint32_t mask;
+        tp.at(v, pos, mask, status);
+        if (v >= tp.nv) mask = 0u;
+        float sc[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) sc[h] = 0.f;
+        const T *kr = Kg + pos * D;
+        for (int k = 0; k < D; ++k) {
+            const float kv = to_f32(kr[k]);
+#pragma unroll
+            for (int h = 0; h < 16; ++h)
+                if (h < G) sc[h] = fmaf(qs[h][k], kv, sc[h]);
+        }
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+            if (h >= G) continue;
+            const float x = ((mask >> h) & 1u) ? sc[h] * sl2 : -INFINITY;
+            const float mx = warp_max(x);
+            const float m_new = fmaxf(m_run[h], mx);
+            const float corr = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - m_new);
+            const float pw = (x == -INFINITY) ? 0.f : exp2f(x - m_new);
+            l_run[h] = l_run[h] * corr + warp_sum(pw);
+            m_run[h] = m_new;
+#pragma unroll
+            for (int e = 0; e < DL; ++e) o[h][e] *= corr;
+            sc[h] = pw;
+        }
+        for (int j = 0; j < 32; ++j) {
+            const int64_t pj = __shfl_sync(0xffffffffu, pos, j);
+            float vv[DL];
+#pragma unroll
+            for (int e = 0; e < DL; ++e) vv[e] = to_f32(Vg[pj * D + lane + 32 * e]);
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+                if (h >= G) continue;
+                const float pj_h = __shfl_sync(0xffffffffu, sc[h], j);
+#pragma unroll
+                for (int e = 0; e < DL; ++e) o[h][e] = fmaf(pj_h, vv[e], o[h][e]);
+            }
+        }
+    }
+    if (lane == 0)
+        for (int h = 0; h < G; ++h) {
+            sm_m[warp][h] = m_run[h];
+            sm_l[warp][h] = l_run[h];
+        }
+#pragma unroll
+    for (int h = 0; h < 16; ++h)
+        if (h < G)
+#pragma unroll
+            for (int e = 0; e < DL; ++e) sm_o[warp][h][lane + 32 * e] = o[h][e];
+    __syncthreads();
+    const int64_t pbase = ((int64_t)grp * S + split) * G;
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+        const int h = i / D, dim = i % D;
+        float M = -INFINITY;
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, sm_m[w][h]);
+        float L = 0.f, acc = 0.f;
+        if (M != -INFINITY)
+            for (int w = 0; w < kAttnWarps; ++w) {
+                if (sm_m[w][h] == -INFINITY) continue;
+                const float f = exp2f(sm_m[w][h] - M);
+                L += sm_l[w][h] * f;
+                acc += sm_o[w][h][dim] * f;
+            }
+        part_o[(pbase + h) * D + dim] = acc;
+        if (dim == 0) {
+            part_ml[(pbase + h) * 2 + 0] = M;
+            part_ml[(pbase + h) * 2 + 1] = L;
+        }
+    }
+}
+
+// Log-sum-exp merge of the split-K partials: one block per (group, head).
+template <typename T>
+__global__ void attn_merge_kernel(Geo g, int S, const float *part_ml, const float *part_o,
+                                  T *out) {
+    const int grp = blockIdx.x / g.G, h = blockIdx.x % g.G;
+    const int b = grp / g.Hkv, kvh = grp % g.Hkv;
+    const int D = g.d;
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, part_ml[(((int64_t)grp * S + s) * g.G + h) * 2]);
+    for (int dim = threadIdx.x; dim < D; dim += blockDim.x) {
+        float L = 0.f, acc = 0.f;
+        if (M != -INFINITY)
+            for (int s = 0; s < S; ++s) {
+                const int64_t idx = ((int64_t)grp * S + s) * g.G + h;
+                const float ms = part_ml[idx * 2];
+                if (ms == -INFINITY) continue;
+                const float f = exp2f(ms - M);
+                L += part_ml[idx * 2 + 1] * f;
+                acc += part_o[idx * D + dim] * f;
+            }
+        out[((int64_t)b * g.Hq + kvh * g.G + h) * D + dim] = from_f32<T>(L > 0.f ? acc / L : 0.f);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const void *V,
+                             const int32_t *lens, const zha_selection *sel, void *out, void *ws,
+                             int32_t *status, cudaStream_t st) {
+    float *part_ml = reinterpret_cast<float *>(static_cast<char *>(ws) + g.ws_part_ml);
+    float *part_o = reinterpret_cast<float *>(static_cast<char *>(ws) + g.ws_part_o);
+    const int S = g.splits;
+    const int dense = sel == nullptr;
+    zha_selection sv{};
+    if (sel) sv = *sel;
+    dim3 grid(S, g.groups());
+    const char *attn_name = dense ? "attn_dense" : "attn_sparse";
+    if (g.dtype == ZHA_BF16) {
+        auto qq = static_cast<const __nv_bfloat16 *>(q);
+        auto kk = static_cast<const __nv_bfloat16 *>(K);
+        auto vv = static_cast<const __nv_bfloat16 *>(V);
+        {
+        ProfScope ps(attn_name, st);
+        if (g.d == 128)
+            attn_mma_kernel<128><<<grid, kAttnWarps * 32, 0, st>>>(g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
+        else
+            attn_mma_kernel<64><<<grid, kAttnWarps * 32, 0, st>>>(g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        ProfScope pm("attn_merge", st);
+        attn_merge_kernel<__nv_bfloat16><<<g.groups() * g.G, g.d, 0, st>>>(g, S, part_ml, part_o, static_cast<__nv_bfloat16 *>(out));
+    } else {
+        auto qq = static_cast<const float *>(q);
+        auto kk = static_cast<const float *>(K);
+        auto vv = static_cast<const float *>(V);
+        {
+        ProfScope ps(attn_name, st);
+        if (g.d == 128)
+            attn_simt_kernel<float, 128><<<grid, kAttnWarps * 32, 0, st>>>(g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
+        else
+            attn_simt_kernel<float, 64><<<grid, kAttnWarps * 32, 0, st>>>(g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        ProfScope pm("attn_merge", st);
+        attn_merge_kernel<float><<<g.groups() * g.G, g.d, 0, st>>>(g, S, part_ml, part_o, static_cast<float *>(out));
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace zha

@@ -1,0 +1,176 @@
+// zha_common.cuh -- shared device helpers and the derived geometry of one
+// configuration (sizes of every tree level, offsets inside the tree buffer and
+// the workspace). Internal to libzha.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/zha.h"
+
+namespace zha {
+
+constexpr int kMaxLevels = ZHA_MAX_LEVELS;
+
+__host__ __device__ inline int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ inline int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+// Nodes at `level` (1 = leaf chunks) for n tokens: floor(n/c), then ceil(./c).
+__host__ __device__ inline int64_t level_nodes(int64_t n, int c, int level) {
+    int64_t m = n / c;
+    for (int l = 2; l <= level; ++l) m = (m + c - 1) / c;
+    return m;
+}
+
+struct Geo {
+    int B, Hq, Hkv, G, d, c, L, R, dtype, flags, splits;
+    int64_t max_len;
+    float s;
+    int64_t cap[kMaxLevels + 1];        // nodes per level at max_len (index = level)
+    size_t mu_off[kMaxLevels + 1];      // tree buffer offsets
+    size_t bias_off[kMaxLevels + 1];
+    size_t tree_bytes;
+    // workspace
+    size_t ws_cand[kMaxLevels + 1], ws_cmask[kMaxLevels + 1], ws_scores[kMaxLevels + 1],
+        ws_kept[kMaxLevels + 1], ws_count[kMaxLevels + 1];
+    size_t ws_maxkey;                   // [L][B*Hkv][G] u32
+    size_t ws_levelkept;                // [B*Hkv][G][L] i32
+    size_t ws_part_ml, ws_part_o;       // split-K partials
+    size_t ws_bytes;
+    __host__ __device__ int groups() const { return B * Hkv; }
+    __host__ __device__ int esize() const { return dtype == ZHA_BF16 ? 2 : 4; }
+};
+
+// ----------------------------------------------------------------- device helpers
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// First error wins.
+__device__ __forceinline__ void set_status(int32_t *status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// Monotone map float -> uint32 (larger float, larger key); 0 is below every
+// finite value's key, so it doubles as "no value".
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+    return __uint_as_float(u);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Load EPL consecutive elements as floats.
+template <int EPL>
+__device__ __forceinline__ void load_vec(const float *p, float (&v)[EPL]) {
+    if constexpr (EPL == 4) {
+        float4 t = *reinterpret_cast<const float4 *>(p);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    } else if constexpr (EPL == 2) {
+        float2 t = *reinterpret_cast<const float2 *>(p);
+        v[0] = t.x; v[1] = t.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) v[i] = p[i];
+    }
+}
+template <int EPL>
+__device__ __forceinline__ void load_vec(const __nv_bfloat16 *p, float (&v)[EPL]) {
+    if constexpr (EPL == 4) {
+        uint2 t = *reinterpret_cast<const uint2 *>(p);
+        __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&t.x);
+        __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&t.y);
+        float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+        v[0] = fa.x; v[1] = fa.y; v[2] = fb.x; v[3] = fb.y;
+    } else if constexpr (EPL == 2) {
+        __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(p);
+        float2 fa = __bfloat1622float2(a);
+        v[0] = fa.x; v[1] = fa.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) v[i] = __bfloat162float(p[i]);
+    }
+}
+template <int EPL>
+__device__ __forceinline__ void store_vec(float *p, const float (&v)[EPL]) {
+    if constexpr (EPL == 4) {
+        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    } else if constexpr (EPL == 2) {
+        *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) p[i] = v[i];
+    }
+}
+template <int EPL>
+__device__ __forceinline__ void store_vec(__nv_bfloat16 *p, const float (&v)[EPL]) {
+    if constexpr (EPL == 4) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+        __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+        uint2 t;
+        t.x = *reinterpret_cast<uint32_t *>(&a);
+        t.y = *reinterpret_cast<uint32_t *>(&b);
+        *reinterpret_cast<uint2 *>(p) = t;
+    } else if constexpr (EPL == 2) {
+        *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v[0], v[1]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) p[i] = __float2bfloat16_rn(v[i]);
+    }
+}
+
+// Current chunk start (explainer step 5): the chunk holding the newest token,
+// or with ZHA_FLAG_TAIL_ONLY only the incomplete tail.
+__host__ __device__ inline int64_t current_chunk_start(int64_t N, int c, int flags) {
+    if (N <= 0) return 0;
+    return (flags & ZHA_FLAG_TAIL_ONLY) ? (N / c) * c : ((N - 1) / c) * c;
+}
+
+}  // namespace zha
+
+// Every kernel launch goes through a ProfScope: it counts the launch and, when
+// profiling is on, brackets it with a pair of CUDA events on its stream.
+namespace zha {
+struct ProfScope {
+    ProfScope(const char *name, cudaStream_t st);
+    ~ProfScope();
+    int slot;
+    cudaStream_t st;
+};
+}  // namespace zha
+
+// Entry points implemented in the kernel files, called by zha_api.cu.
+namespace zha {
+cudaError_t launch_tree_update(const Geo &g, void *tree, const void *K, const void *refs,
+                               const int32_t *lens, int n_new, int32_t *status, cudaStream_t st);
+cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const int32_t *lens,
+                         const float *p_levels, const zha_selection &sel, void *ws,
+                         int32_t *status, cudaStream_t st);
+cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const void *V,
+                             const int32_t *lens, const zha_selection *sel, void *out, void *ws,
+                             int32_t *status, cudaStream_t st);
+cudaError_t launch_decode_write(const Geo &g, void *K, void *V, int32_t *lens, const void *k_new,
+                                const void *v_new, int32_t *status, cudaStream_t st);
+cudaError_t launch_topp_select(const float *scores, const int32_t *counts, int n_sets,
+                               int64_t stride, float p, uint8_t *kept, int32_t *status,
+                               cudaStream_t st);
+}  // namespace zha

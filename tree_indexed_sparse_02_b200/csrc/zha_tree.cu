@@ -1,0 +1,246 @@
+// zha_tree.cu -- building and extending the summary tree.
+//
+// Page "Zyphra AI Introduces Zyphra Hierarchical Attention (ZHA)", section
+// "Building the tree": contiguous chunks of c keys are summarised against R
+// reference queries as tangent planes of the chunk's log attention mass, and
+// the summaries are grouped and summarised again level by level.
+//
+// For reference r and points x_i with log-weights a_i (raw keys: a_i = 0;
+// children of a parent: x_i = mu_{i,r}, a_i = bias_{i,r}):
+//   l_i = s r.x_i + a_i,  F = log sum_i e^{l_i},  w_i = e^{l_i - F},
+//   mu_r = sum_i w_i x_i,  bias_r = F - s r.mu_r.
+// Since s r.mu_r = sum_i w_i (l_i - a_i), the bias is formed from the same
+// per-point dot products, in one online (running-max) pass over the points.
+//
+// Work split: one warp per (node, reference) pair; each lane owns d/32
+// consecutive coordinates, so point loads are coalesced 8/16-byte vectors and
+// the dot products end in a warp butterfly (every lane gets bitwise the same
+// sum, so all lanes agree on every branch).
+#include "zha_common.cuh"
+
+namespace zha {
+
+namespace {
+
+constexpr int kLevelWarps = 8;
+
+template <typename T, int EPL>
+__device__ __forceinline__ void warp_plane(const T *x0, int64_t xstride, const float *a0,
+                                           int64_t astride, int npts, const float (&rv)[EPL],
+                                           float s, T *mu_out, float *b_out, int lane) {
+    float m = -INFINITY, sum = 0.f, wl = 0.f;
+    float acc[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+    for (int i = 0; i < npts; ++i) {
+        float x[EPL];
+        load_vec<EPL>(x0 + (int64_t)i * xstride + lane * EPL, x);
+        float part = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) part = fmaf(rv[e], x[e], part);
+        const float rx = s * warp_sum(part);           // s r.x_i
+        const float ai = a0 ? a0[(int64_t)i * astride] : 0.f;
+        const float l = rx + ai;
+        if (l > m) {
+            const float sc = (m == -INFINITY) ? 0.f : expf(m - l);
+            sum *= sc;
+            wl *= sc;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] *= sc;
+            m = l;
+        }
+        const float w = expf(l - m);
+        sum += w;
+        wl = fmaf(w, rx, wl);
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, x[e], acc[e]);
+    }
+    const float inv = 1.f / sum;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] *= inv;
+    store_vec<EPL>(mu_out + lane * EPL, acc);
+    if (lane == 0) *b_out = (m + logf(sum)) - wl * inv;
+}
+
+struct TreePtrs {
+    void *mu[kMaxLevels + 1];
+    float *bias[kMaxLevels + 1];
+};
+
+// Plane r of node `node` at `level` of group `grp`.
+template <typename T, int EPL>
+__device__ __forceinline__ void node_plane(const Geo &g, const TreePtrs &tp, const T *K,
+                                           const T *refs, int grp, int level, int64_t node,
+                                           int64_t n_below, int r, int lane) {
+    const int kvh = grp % g.Hkv;
+    float rv[EPL];
+    load_vec<EPL>(refs + ((int64_t)kvh * g.R + r) * g.d + lane * EPL, rv);
+    T *mu = reinterpret_cast<T *>(tp.mu[level]) + ((grp * g.cap[level] + node) * g.R + r) * g.d;
+    float *bias = tp.bias[level] + (grp * g.cap[level] + node) * g.R + r;
+    if (level == 1) {
+        const T *x0 = K + ((int64_t)grp * g.max_len + node * g.c) * g.d;
+        warp_plane<T, EPL>(x0, g.d, nullptr, 0, g.c, rv, g.s, mu, bias, lane);
+    } else {
+        const int64_t c0 = node * g.c;
+        const int64_t c1 = min(c0 + g.c, n_below);
+        const T *x0 = reinterpret_cast<const T *>(tp.mu[level - 1]) +
+                      ((grp * g.cap[level - 1] + c0) * g.R + r) * g.d;
+        const float *a0 = tp.bias[level - 1] + (grp * g.cap[level - 1] + c0) * g.R + r;
+        warp_plane<T, EPL>(x0, (int64_t)g.R * g.d, a0, g.R, (int)(c1 - c0), rv, g.s, mu, bias,
+                           lane);
+    }
+}
+
+// Tokens before/after the update of sequence b; false if nothing changes.
+__device__ __forceinline__ bool update_range(const Geo &g, const int32_t *lens, int b, int n_new,
+                                             int64_t &n_old, int64_t &n_now, int32_t *status) {
+    n_now = lens[b];
+    if (n_now < 0 || n_now > g.max_len) {
+        set_status(status, ZHA_ERR_CAPACITY);
+        return false;
+    }
+    n_old = (n_new < 0) ? 0 : max64(n_now - n_new, 0);
+    return (n_now / g.c) > (n_old / g.c);
+}
+
+// One level, many nodes: grid.x covers node slots x references, grid.y groups.
+template <typename T, int EPL>
+__global__ void __launch_bounds__(kLevelWarps * 32)
+tree_level_kernel(Geo g, TreePtrs tp, const T *K, const T *refs, const int32_t *lens, int level,
+                  int n_new, int64_t slots, int32_t *status) {
+    const int grp = blockIdx.y;
+    const int b = grp / g.Hkv;
+    const int lane = threadIdx.x & 31;
+    const int64_t item = (int64_t)blockIdx.x * kLevelWarps + (threadIdx.x >> 5);
+    if (item >= slots * g.R) return;
+    int64_t n_old, n_now;
+    if (!update_range(g, lens, b, n_new, n_old, n_now, status)) return;
+    int64_t lo = n_old / g.c;
+    for (int l = 2; l <= level; ++l) lo /= g.c;
+    const int64_t node = lo + item / g.R;
+    const int r = (int)(item % g.R);
+    if (node >= level_nodes(n_now, g.c, level)) return;
+    const int64_t n_below = level > 1 ? level_nodes(n_now, g.c, level - 1) : 0;
+    node_plane<T, EPL>(g, tp, K, refs, grp, level, node, n_below, r, lane);
+}
+
+// Few new tokens (a decode step): one block per group walks every level,
+// warp r computing plane r of each changed node; levels are separated by a
+// block barrier, which also makes the children's global writes visible.
+template <typename T, int EPL>
+__global__ void tree_path_kernel(Geo g, TreePtrs tp, const T *K, const T *refs,
+                                 const int32_t *lens, int n_new, int32_t *status) {
+    const int grp = blockIdx.x;
+    const int b = grp / g.Hkv;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    int64_t n_old, n_now;
+    const bool any = update_range(g, lens, b, n_new, n_old, n_now, status);
+    if (!any) return;  // uniform across the block
+    int64_t lo = n_old / g.c;
+    for (int level = 1; level <= g.L; ++level) {
+        if (level > 1) lo /= g.c;
+        const int64_t hi = level_nodes(n_now, g.c, level);
+        const int64_t n_below = level > 1 ? level_nodes(n_now, g.c, level - 1) : 0;
+        const int64_t items = (hi - lo) * g.R;
+        for (int64_t it = warp; it < items; it += blockDim.x >> 5)
+            node_plane<T, EPL>(g, tp, K, refs, grp, level, lo + it / g.R, n_below,
+                               (int)(it % g.R), lane);
+        __syncthreads();
+    }
+}
+
+template <typename T, int EPL>
+cudaError_t tree_update_t(const Geo &g, const TreePtrs &tp, const T *K, const T *refs,
+                          const int32_t *lens, int n_new, int32_t *status, cudaStream_t st) {
+    if (n_new >= 0 && n_new <= g.c) {
+        const int warps = g.R < 4 ? 4 : g.R;
+        ProfScope ps("tree_path", st);
+        tree_path_kernel<T, EPL><<<g.groups(), warps * 32, 0, st>>>(g, tp, K, refs, lens, n_new,
+                                                                    status);
+        return cudaGetLastError();
+    }
+    int64_t bound = n_new < 0 ? g.cap[1] : (n_new + g.c - 1) / g.c;
+    for (int level = 1; level <= g.L; ++level) {
+        if (level > 1) bound = n_new < 0 ? g.cap[level] : min64(bound / g.c + 2, g.cap[level]);
+        bound = min64(bound, g.cap[level]);
+        if (bound <= 0) break;
+        const int64_t items = bound * g.R;
+        dim3 grid((unsigned)((items + kLevelWarps - 1) / kLevelWarps), g.groups());
+        {
+            static const char *names[] = {"", "tree_level[l1]", "tree_level[l2]", "tree_level[l3]",
+                                          "tree_level[l4]", "tree_level[l5]", "tree_level[l6]",
+                                          "tree_level[l7]", "tree_level[l8]"};
+            ProfScope ps(names[level], st);
+            tree_level_kernel<T, EPL><<<grid, kLevelWarps * 32, 0, st>>>(g, tp, K, refs, lens, level,
+                                                                         n_new, bound, status);
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_tree_update(const Geo &g, void *tree, const void *K, const void *refs,
+                               const int32_t *lens, int n_new, int32_t *status, cudaStream_t st) {
+    TreePtrs tp{};
+    for (int l = 1; l <= g.L; ++l) {
+        tp.mu[l] = static_cast<char *>(tree) + g.mu_off[l];
+        tp.bias[l] = reinterpret_cast<float *>(static_cast<char *>(tree) + g.bias_off[l]);
+    }
+    if (g.dtype == ZHA_BF16) {
+        auto k = static_cast<const __nv_bfloat16 *>(K);
+        auto r = static_cast<const __nv_bfloat16 *>(refs);
+        return g.d == 128 ? tree_update_t<__nv_bfloat16, 4>(g, tp, k, r, lens, n_new, status, st)
+                          : tree_update_t<__nv_bfloat16, 2>(g, tp, k, r, lens, n_new, status, st);
+    }
+    auto k = static_cast<const float *>(K);
+    auto r = static_cast<const float *>(refs);
+    return g.d == 128 ? tree_update_t<float, 4>(g, tp, k, r, lens, n_new, status, st)
+                      : tree_update_t<float, 2>(g, tp, k, r, lens, n_new, status, st);
+}
+
+// Decode step prologue: write the new token of every (sequence, KV head) at
+// position lens[b], then advance lens[b] (one block per sequence, so the
+// increment follows every read of the old length in the block).
+template <typename T>
+__global__ void decode_write_kernel(Geo g, T *K, T *V, int32_t *lens, const T *k_new,
+                                    const T *v_new, int32_t *status) {
+    const int b = blockIdx.x;
+    const int64_t n = lens[b];
+    const bool ok = n >= 0 && n < g.max_len;
+    if (ok) {
+        for (int i = threadIdx.x; i < g.Hkv * g.d; i += blockDim.x) {
+            const int kvh = i / g.d, e = i % g.d;
+            const int64_t dst = (((int64_t)b * g.Hkv + kvh) * g.max_len + n) * g.d + e;
+            K[dst] = k_new[((int64_t)b * g.Hkv + kvh) * g.d + e];
+            V[dst] = v_new[((int64_t)b * g.Hkv + kvh) * g.d + e];
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (ok)
+            lens[b] = (int32_t)(n + 1);
+        else
+            set_status(status, ZHA_ERR_CAPACITY);
+    }
+}
+
+cudaError_t launch_decode_write(const Geo &g, void *K, void *V, int32_t *lens, const void *k_new,
+                                const void *v_new, int32_t *status, cudaStream_t st) {
+    ProfScope ps("decode_write", st);
+    if (g.dtype == ZHA_BF16)
+        decode_write_kernel<__nv_bfloat16><<<g.B, 256, 0, st>>>(
+            g, static_cast<__nv_bfloat16 *>(K), static_cast<__nv_bfloat16 *>(V), lens,
+            static_cast<const __nv_bfloat16 *>(k_new), static_cast<const __nv_bfloat16 *>(v_new),
+            status);
+    else
+        decode_write_kernel<float><<<g.B, 256, 0, st>>>(
+            g, static_cast<float *>(K), static_cast<float *>(V), lens,
+            static_cast<const float *>(k_new), static_cast<const float *>(v_new), status);
+    return cudaGetLastError();
+}
+
+}  // namespace zha
