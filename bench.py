@@ -1,0 +1,476 @@
+#!/usr/bin/env python
+"""Decode benchmark of the ZHA hot path on B200: one step = append the new
+token to the cache and the summary tree, route every query head top-down with
+top-p, and attend over the routed tokens (zha_decode), for every sequence of
+the batch. Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload deep256k]
+  python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+Multi-GPU (torchrun): each rank decodes its own independent replica of the
+workload (the path shards by sequence and KV head with no exchange), timed on
+the device; the slowest rank's time is used.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s per layer & µs/step vs context; HBM GB/s on touched bytes"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="zha", choices=["zha", "reference"])
+    ap.add_argument("--workload", default="deep256k",
+                    choices=["deep256k", "deep1m", "wide32k", "tiny", "small", "medium"])
+    ap.add_argument("--refs", default="random", choices=["random", "aligned"])
+    ap.add_argument("--p", type=float, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-profile", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def workload(args):
+    import dataclasses
+
+    from tree_indexed_sparse_02_b200 import inputs as I
+    w = {"deep256k": I.DEEP_256K, "deep1m": I.DEEP_1M, "wide32k": I.WIDE_32K, "tiny": I.TINY_F32,
+         # a reduced deep-tree case (same kernels, B=1, N=64K) for detailed profiler captures
+         "small": dataclasses.replace(I.DEEP_256K, name="deep N=65536 c=4 L=6 B=1", batch=1,
+                                      context=65536, needles=64, diffuse_nodes=8),
+         # one sequence of the 256K deep workload (a quarter of its bytes)
+         "medium": dataclasses.replace(I.DEEP_256K, name="deep N=262144 c=4 L=6 B=1", batch=1)}[args.workload]
+    w = dataclasses.replace(w, refs_mode=args.refs)
+    if args.p is not None:
+        w = dataclasses.replace(w, p=args.p)
+    return w
+
+
+# ----------------------------------------------------------------- helpers
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, enabled: bool = True):
+        self.index, self.enabled, self.proc, self.path = index, enabled, None, None
+
+    def __enter__(self):
+        if not self.enabled:
+            return self
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[5], f[6], f[7], f[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "zha":
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    import torch
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    import torch
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- CPU oracle
+
+
+def oracle_sample(w, inp, steps: int, warmup: int = 0):
+    """Time the oracle's decode step (route + exact attention) for ONE
+    (sequence, KV head) group on a prebuilt oracle tree; returns (seconds per
+    whole-batch step, threads, sample description)."""
+    sys.path.insert(0, os.path.join(ROOT, "oracle"))
+    import numpy as np
+    import torch
+
+    import zha_oracle as orc
+    orc.build_library()
+    G, N, d = w.group, w.context, w.head_dim
+    s = 1.0 / math.sqrt(d)
+    K = inp.K[0, 0, :N].to("cpu", torch.float64).numpy()
+    V = inp.V[0, 0, :N].to("cpu", torch.float64).numpy()
+    refs = inp.refs[0].to("cpu", torch.float64).numpy()
+    t0 = time.perf_counter()
+    tree = orc.build_tree(K, refs, N, w.chunk, w.levels, s, storage="bf16" if w.dtype == "bf16" else "f32")
+    build_s = time.perf_counter() - t0
+    q = inp.q[0, :G].to("cpu", torch.float64).numpy()
+    rng = np.random.default_rng(0)
+    times = []
+    for i in range(warmup + steps):
+        qi = q if i == 0 else rng.normal(size=q.shape)
+        t0 = time.perf_counter()
+        orc.decode_group(tree, qi, K, V, w.p)
+        if i >= warmup:
+            times.append(time.perf_counter() - t0)
+    groups = w.batch * w.n_kv_heads
+    per_group = sum(times) / len(times)
+    sample = (f"oracle route+attend of 1 of {groups} (sequence, KV head) groups per step on a prebuilt "
+              f"oracle tree (build {build_s:.1f}s untimed), {len(times)} steps; whole-batch step time = "
+              f"{groups} x group time")
+    return per_group * groups, orc.num_threads(), sample
+
+
+def reference_arm(args, w, world, rank):
+    import torch
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    from tree_indexed_sparse_02_b200.inputs import make_inputs
+    inp = make_inputs(w, device=dev)
+    step_s, cores, sample = oracle_sample(w, inp, args.steps, args.warmup)
+    value = w.batch / step_s
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    return {"workload": w.name, "batch": w.batch, "context": w.context, "n_q_heads": w.n_q_heads,
+            "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "chunk": w.chunk, "levels": w.levels,
+            "n_refs": w.n_refs, "p": w.p, "refs": w.refs_mode, "needles_per_seq": w.needles,
+            "l2": "flushed (256 MiB write) before every timed step, outside the timed region"}
+
+
+# -------------------------------------------------------------- ZHA arm
+
+
+def zha_arm(args, w, world, rank, local):
+    import dataclasses
+
+    import torch
+
+    from tree_indexed_sparse_02_b200 import zha
+    from tree_indexed_sparse_02_b200.inputs import decode_stream, make_inputs
+
+    K_steps, W_steps = args.steps, args.warmup
+    if world > 1:
+        w = dataclasses.replace(w, seed=w.seed + 1000 * rank)   # independent replica per rank
+    n_total = W_steps + 2 * K_steps + (K_steps if not args.no_e2e else 0)
+    cap = w.context + n_total + 8
+    inp = make_inputs(w, device="cuda", capacity=cap)
+    cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs, w.dtype,
+                     cap)
+    buf = zha.Buffers(cfg)
+    K, V, refs, lens = inp.K, inp.V, inp.refs, inp.lens
+    k_new, v_new, qs = decode_stream(w, n_total, device="cuda")
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=w.torch_dtype(), device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    p = w.p
+
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    zha.tree_build(cfg, buf.tree, K, refs, lens, buf.status)
+    torch.cuda.synchronize()
+    build_ms = (time.perf_counter() - t0) * 1e3
+    buf.check_status("tree build")
+
+    count_views = [buf.level_state(l)["count"].view(-1) for l in range(1, w.levels + 1)]
+    sel_count = buf.sel["count"].view(-1)
+    step_i = 0
+
+    def decode_step(i):
+        zha.decode(cfg, buf.tree, K, V, refs, lens, qs[i], k_new[i], v_new[i], p, buf.sel, out,
+                   buf.workspace, buf.status)
+
+    # warm-up
+    for _ in range(W_steps):
+        decode_step(step_i)
+        step_i += 1
+    torch.cuda.synchronize()
+    buf.check_status("warm-up")
+
+    def timed_pass(n, hist):
+        nonlocal step_i
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for j in range(n):
+            flush.fill_(float(j))
+            ev[j][0].record(stream)
+            decode_step(step_i)
+            ev[j][1].record(stream)
+            step_i += 1
+            for l in range(w.levels):
+                hist[j, l].copy_(count_views[l], non_blocking=True)
+            hist[j, w.levels].copy_(sel_count, non_blocking=True)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    G_groups = w.batch * w.n_kv_heads
+    hist_a = torch.zeros((K_steps, w.levels + 1, G_groups), dtype=torch.int32, device="cuda")
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = zha.launch_count()
+    with Clocks(local, enabled=not args.no_clocks) as clk:
+        times_a = timed_pass(K_steps, hist_a)
+    launches = zha.launch_count() - launches0
+    barrier(world)
+    buf.check_status("timed steps")
+    clocks = clk.summary()
+
+    total_ms = max_over_ranks(sum(times_a), world)
+    ms_per_step = total_ms / K_steps
+    tokens = sum_over_ranks(float(w.batch * K_steps), world)
+    value = tokens / (total_ms / 1e3)
+
+    # bytes the step must move (algorithmic), from the routed counts of each step
+    es = 2 if w.dtype == "bf16" else 4
+    node_bytes = w.n_refs * w.head_dim * es + w.n_refs * 4          # summary keys + plane offsets
+    cand_bytes = node_bytes + 8 + w.group * 4                       # + index, head mask, G scores
+    tok_bytes = 2 * w.head_dim * es                                 # K + V row
+    h = hist_a.double().cpu()
+    cand_per_step = h[:, : w.levels, :].sum(dim=(1, 2))             # all levels, all groups
+    leaves_per_step = h[:, w.levels, :].sum(dim=1)
+    extra_tokens = G_groups * (w.chunk + 1)                          # sink + current chunk, upper bound
+    attn_tokens = leaves_per_step * w.chunk + extra_tokens
+    qo_bytes = G_groups * 2 * w.group * w.head_dim * es
+    touched = cand_per_step * cand_bytes + attn_tokens * tok_bytes + qo_bytes
+    touched_mean = float(touched.mean())
+    keys_share = float(attn_tokens.mean()) / (G_groups * (w.context + W_steps + K_steps))
+    peak, peak_kind = read_peaks()
+
+    res = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K_steps,
+           "warmup": W_steps, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": config_of(w),
+           "us_per_step": ms_per_step * 1e3, "tree_build_ms": build_ms,
+           "touched_bytes_per_step": touched_mean,
+           "touched_gbs": touched_mean / (ms_per_step / 1e3) / 1e9,
+           "touched_frac_of_hbm": touched_mean / (ms_per_step / 1e3) / 1e9 / peak,
+           "keys_attended": keys_share,
+           "candidates_per_step": float(cand_per_step.mean()),
+           "gpu_launches": int(launches), "clocks": clocks}
+
+    # per-kernel CUDA-event timing: a second pass of K steps, every launch bracketed
+    if not args.no_profile:
+        hist_b = torch.zeros_like(hist_a)
+        zha.profile_enable(True)
+        times_b = timed_pass(K_steps, hist_b)
+        zha.profile_enable(False)
+        prof = zha.profile_read()
+        buf.check_status("profiled steps")
+        hb = hist_b.double().cpu()
+        tot = sum(v[0] for v in prof.values())
+        top = max(prof, key=lambda k: prof[k][0])
+        res["kernels"] = {k: {"ms_per_step": v[0] / K_steps, "launches_per_step": v[1] / K_steps,
+                              "share": v[0] / tot} for k, v in sorted(prof.items(), key=lambda kv: -kv[1][0])}
+        res["profiled_ms_per_step"] = sum(times_b) / K_steps
+        # algorithmic bytes of the dominant kernel over the profiled pass
+        if top.startswith("score[l"):
+            lvl = int(top[len("score[l"):-1])
+            alg = float(hb[:, lvl - 1, :].sum()) * cand_bytes + K_steps * w.levels * 0
+            unit_desc = f"{cand_bytes} B per candidate node at level {lvl}"
+        elif top == "attn_sparse":
+            toks = hb[:, w.levels, :].sum() * w.chunk + K_steps * extra_tokens
+            alg = float(toks) * tok_bytes
+            unit_desc = f"{tok_bytes} B per attended (union) token"
+        else:
+            alg = None
+            unit_desc = "not an HBM-streaming kernel"
+        ms_top, n_top = prof[top]
+        if alg is not None:
+            achieved = alg / n_top / (ms_top / n_top / 1e3) / 1e9
+            res["roofline"] = {"kernel": top, "bound": "hbm", "achieved": achieved, "peak": peak,
+                               "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                               "traffic": traffic_for(top, alg / n_top), "bytes_per_launch": alg / n_top,
+                               "unit_bytes": unit_desc, "avg_launch_ms": ms_top / n_top}
+        else:
+            res["roofline"] = {"kernel": top, "bound": "latency", "achieved": None, "peak": peak,
+                               "unit": "GB/s", "frac": None, "traffic": None}
+
+    # the build's own dense flash-decoding kernel on the same cache
+    if not args.no_dense:
+        q0 = qs[0]
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_steps)]
+        for j in range(W_steps):
+            zha.dense_decode(cfg, q0, K, V, lens, out, buf.workspace, buf.status)
+        for j in range(K_steps):
+            flush.fill_(float(j))
+            ev[j][0].record(stream)
+            zha.dense_decode(cfg, q0, K, V, lens, out, buf.workspace, buf.status)
+            ev[j][1].record(stream)
+        torch.cuda.synchronize()
+        dense_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world) / K_steps
+        n_now = int(lens[0])
+        dense_bytes = G_groups * n_now * tok_bytes + qo_bytes
+        res["dense"] = {"us_per_step": dense_ms * 1e3, "tokens_per_s": w.batch / (dense_ms / 1e3),
+                        "gbs": dense_bytes / (dense_ms / 1e3) / 1e9, "frac_of_hbm": dense_bytes / (dense_ms / 1e3) / 1e9 / peak}
+        res["speedup_vs_dense"] = dense_ms / ms_per_step
+
+    # end to end through the public call with host buffers
+    if not args.no_e2e:
+        qh = qs[step_i:step_i + K_steps].cpu().pin_memory()
+        kh = k_new[step_i:step_i + K_steps].cpu().pin_memory()
+        vh = v_new[step_i:step_i + K_steps].cpu().pin_memory()
+        oh = torch.empty((K_steps,) + tuple(out.shape), dtype=out.dtype).pin_memory()
+        qd, kd, vd = torch.empty_like(qs[0]), torch.empty_like(k_new[0]), torch.empty_like(v_new[0])
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_steps)]
+        barrier(world)
+        for j in range(K_steps):
+            flush.fill_(float(j))
+            ev[j][0].record(stream)
+            qd.copy_(qh[j], non_blocking=True)
+            kd.copy_(kh[j], non_blocking=True)
+            vd.copy_(vh[j], non_blocking=True)
+            zha.decode(cfg, buf.tree, K, V, refs, lens, qd, kd, vd, p, buf.sel, out, buf.workspace, buf.status)
+            oh[j].copy_(out, non_blocking=True)
+            ev[j][1].record(stream)
+        torch.cuda.synchronize()
+        buf.check_status("e2e steps")
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
+        res["e2e"] = {"value": sum_over_ranks(float(w.batch * K_steps), world) / (e2e_ms / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": (qd.numel() + kd.numel() + vd.numel()) * qd.element_size(),
+                      "d2h_bytes_per_step": out.numel() * out.element_size()}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        step_s, cores, sample = oracle_sample(w, inp, steps=2)
+        res["cpu_baseline"] = {"value": w.batch / step_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": sample}
+    if world > 1:
+        torch.distributed.barrier()
+    return res
+
+
+def traffic_for(kernel: str, alg_bytes_per_launch: float):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; None otherwise."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        ent = d["kernels"][kernel]
+        if ent.get("source_sha") != source_sha():
+            return None
+        return ent["dram_bytes_per_alg_byte"] * alg_bytes_per_launch
+    except Exception:
+        return None
+
+
+def source_sha():
+    import hashlib
+    hsh = hashlib.sha256()
+    csrc = os.path.join(ROOT, "tree_indexed_sparse_02_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            hsh.update(open(os.path.join(csrc, name), "rb").read())
+    return hsh.hexdigest()[:16]
+
+
+def main():
+    args = parse()
+    w = workload(args)
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        reference_arm(args, w, world, rank)
+        return
+    res = zha_arm(args, w, world, rank, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

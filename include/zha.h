@@ -40,7 +40,8 @@
  *     Query head h uses KV head h / G, G = n_q_heads / n_kv_heads.
  *   - Supported: head_dim in {64, 128}; chunk a power of two in [2, 256];
  *     1 <= levels <= ZHA_MAX_LEVELS; 1 <= n_refs <= 32; G <= 16;
- *     dtype BF16 or F32. Anything else returns ZHA_ERR_UNSUPPORTED.
+ *     max_len <= 2^30 and max_len / chunk <= 2^23; dtype BF16 or F32.
+ *     Anything else returns ZHA_ERR_UNSUPPORTED.
  */
 #ifndef ZHA_H
 #define ZHA_H
@@ -113,12 +114,14 @@ typedef struct zha_selection {
 
 /* Byte offsets, inside the workspace, of the per-level routing state of the
  * last zha_route / zha_decode call (valid until the workspace is reused):
- *   cand_idx  [batch][n_kv_heads][cap_l] int32    candidate node indices, ascending
- *   cand_mask [batch][n_kv_heads][cap_l] uint32   heads for which it is a candidate
- *   scores    [batch][n_kv_heads][G][cap_l] float estimate max_r(s q.mu_r + b_r)
- *   kept_mask [batch][n_kv_heads][cap_l] uint32   heads that kept it
- *   count     [batch][n_kv_heads] int32           candidates in use
- * cap_l = nodes at level l for max_len tokens. */
+ *   cand_idx  [batch][n_kv_heads][cap] int32    candidate node indices, ascending
+ *   cand_mask [batch][n_kv_heads][cap] uint32   heads for which it is a candidate
+ *                                               (0: padding, a child past the level's end)
+ *   scores    [batch][n_kv_heads][G][cap] float estimate max_r(s q.mu_r + b_r)
+ *   kept_mask [batch][n_kv_heads][cap] uint32   heads that kept it
+ *   count     [batch][n_kv_heads] int32         entries in use
+ * cap = nodes at that level for max_len tokens, plus chunk, rounded up to a
+ * multiple of 8. */
 typedef struct zha_level_view {
     int64_t cap;
     size_t cand_idx, cand_mask, scores, kept_mask, count;

@@ -70,7 +70,7 @@ def test_tree_and_workspace_layout(zha):
     ws = zha.workspace_bytes(cfg)
     for level in range(1, 7):
         v = zha.workspace_level_view(cfg, level)
-        assert v.cap == zha.level_nodes(cfg, cfg.max_len, level)
+        assert v.cap == (zha.level_nodes(cfg, cfg.max_len, level) + cfg.chunk + 7) // 8 * 8
         for off in (v.cand_idx, v.cand_mask, v.scores, v.kept_mask, v.count):
             assert off % 256 == 0 and off < ws
 

@@ -55,12 +55,16 @@ def gpu_level_candidates(state, b, kvh, h, n_l):
     cm = state["cand_mask"][b, kvh, :cnt].cpu().numpy().astype(np.uint32)
     km = state["kept_mask"][b, kvh, :cnt].cpu().numpy().astype(np.uint32)
     sc = state["scores"][b, kvh, h, :cnt].cpu().numpy().astype(np.float64)
+    assert np.all(np.diff(idx) > 0), "candidate list must be strictly ascending"
+    # entries with an empty head mask are padding (children past the level's end)
+    real = cm != 0
+    assert not np.any(km[~real]), "padding entry kept"
+    idx, cm, km, sc = idx[real], cm[real], km[real], sc[real]
     bit = np.uint32(1 << h)
     cand = np.zeros(n_l, dtype=bool)
     kept = np.zeros(n_l, dtype=bool)
     score = np.full(n_l, -np.inf)
     member = (cm & bit) != 0
-    assert np.all(np.diff(idx) > 0), "candidate list must be strictly ascending"
     assert idx.size == 0 or (idx.min() >= 0 and idx.max() < n_l)
     cand[idx[member]] = True
     kept[idx[member & ((km & bit) != 0)]] = True

@@ -25,8 +25,8 @@ zha_status check_config(const zha_config *c) {
     if (c->levels > ZHA_MAX_LEVELS || c->n_refs > 32) return ZHA_ERR_UNSUPPORTED;
     if (c->dtype != ZHA_BF16 && c->dtype != ZHA_F32) return ZHA_ERR_UNSUPPORTED;
     if (c->flags & ~ZHA_FLAG_TAIL_ONLY) return ZHA_ERR_UNSUPPORTED;
-    // int32 indices of tokens and leaves; fixed-point mass sums need <= 2^23 candidates
-    if (c->max_len > INT32_MAX || c->max_len / c->chunk > (1 << 23)) return ZHA_ERR_UNSUPPORTED;
+    // int32 token and leaf indices; fixed-point mass sums need <= 2^23 candidates
+    if (c->max_len > (1 << 30) || c->max_len / c->chunk > (1 << 23)) return ZHA_ERR_UNSUPPORTED;
     if (c->attn_splits < 0 || c->attn_splits > 4096) return ZHA_ERR_INVALID_ARG;
     if (!(c->scale == c->scale)) return ZHA_ERR_INVALID_ARG;
     return ZHA_OK;
@@ -59,21 +59,28 @@ Geo make_geo(const zha_config *c) {
     g.tree_bytes = off;
     off = 0;
     for (int l = 1; l <= g.L; ++l) {
-        const size_t n = groups * g.cap[l];
+        g.capv[l] = (g.cap[l] + g.c + 7) & ~int64_t(7);
+        const size_t n = groups * g.capv[l];
         g.ws_cand[l] = off;   off = align256(off + n * 4);
         g.ws_cmask[l] = off;  off = align256(off + n * 4);
         g.ws_kept[l] = off;   off = align256(off + n * 4);
         g.ws_scores[l] = off; off = align256(off + n * g.G * 4);
         g.ws_count[l] = off;  off = align256(off + groups * 4);
+        const size_t k = groups * g.cap[l];
+        g.ws_plist[l] = off;  off = align256(off + k * 4);
+        g.ws_pmask[l] = off;  off = align256(off + k * 4);
+        g.ws_pcount[l] = off; off = align256(off + groups * 4);
     }
     g.ws_maxkey = off;
     off = align256(off + (size_t)g.L * groups * g.G * 4);
-    g.ws_levelkept = off;
-    off = align256(off + groups * g.G * g.L * 4);
+    g.ws_minkey = off;
+    off = align256(off + (size_t)g.L * groups * g.G * 4);
+    g.ws_done = off;
+    off = align256(off + (size_t)g.L * groups * 4);
     int splits = c->attn_splits;
     if (splits == 0) {
-        // about four CTAs per SM over all groups, no more than one per 64 tokens
-        const int64_t want = (148 * 4 + (int64_t)groups - 1) / (int64_t)groups;
+        // one wave of two resident CTAs per SM over all groups, at most one per 64 tokens
+        const int64_t want = (148 * 2) / (int64_t)groups;
         const int64_t most = (g.max_len + 63) / 64;
         splits = (int)(want < most ? want : most);
         if (splits < 1) splits = 1;
@@ -152,7 +159,7 @@ zha_status zha_workspace_level_view(const zha_config *cfg, int32_t level, zha_le
     if (s != ZHA_OK) return s;
     if (level < 1 || level > cfg->levels || !v) return ZHA_ERR_INVALID_ARG;
     Geo g = make_geo(cfg);
-    v->cap = g.cap[level];
+    v->cap = g.capv[level];
     v->cand_idx = g.ws_cand[level];
     v->cand_mask = g.ws_cmask[level];
     v->scores = g.ws_scores[level];

@@ -29,30 +29,30 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kAttnWarps = 4;
 
 // Which cache position virtual token v of a group is, and which heads see it.
+// All token counts fit in int32 (max_len <= 2^30).
 struct TokenPlan {
-    int64_t N, cur_start, n1;
-    int64_t nsel, sel_tokens;  // kept leaf chunks, their tokens
-    int64_t a_len;             // sink span [0, a_len)
-    int64_t b_start, b_len;    // current-chunk span
-    int64_t nv;                // stream length
-    int c;
+    int N, cur_start, n1;
+    int nsel, sel_tokens;  // kept leaf chunks, their tokens
+    int a_len;             // sink span [0, a_len)
+    int b_start, b_len;    // current-chunk span
+    int nv;                // stream length
+    int lc;                // log2(c)
     uint32_t all;
     const int32_t *leaf;
     const uint32_t *hmask;
 
-    __device__ __forceinline__ void at(int64_t v, int64_t &pos, uint32_t &mask,
-                                       int32_t *status) const {
+    __device__ __forceinline__ void at(int v, int &pos, uint32_t &mask, int32_t *status) const {
         if (v < sel_tokens) {
-            const int64_t e = v / c;
-            const int64_t lf = leaf[e];
-            if (lf < 0 || lf >= n1) {
+            const int e = v >> lc;
+            const int lf = __ldg(&leaf[e]);
+            if ((unsigned)lf >= (unsigned)n1) {
                 set_status(status, ZHA_ERR_INVALID_ARG);
                 pos = 0;
                 mask = 0u;
                 return;
             }
-            pos = lf * c + (v - e * c);
-            mask = hmask[e] | ((pos == 0 || pos >= cur_start) ? all : 0u);
+            pos = (lf << lc) | (v & ((1 << lc) - 1));
+            mask = __ldg(&hmask[e]) | ((pos == 0 || pos >= cur_start) ? all : 0u);
             return;
         }
         v -= sel_tokens;
@@ -77,15 +77,15 @@ __device__ __forceinline__ TokenPlan make_plan(const Geo &g, const int32_t *lens
                                                int32_t *status) {
     TokenPlan tp{};
     const int b = grp / g.Hkv;
-    int64_t N = lens[b];
+    int N = lens[b];
     if (N < 0 || N > g.max_len) {
         set_status(status, ZHA_ERR_CAPACITY);
         N = 0;
     }
     tp.N = N;
-    tp.c = g.c;
+    tp.lc = __ffs(g.c) - 1;
     tp.all = g.G >= 32 ? 0xffffffffu : ((1u << g.G) - 1u);
-    tp.n1 = N / g.c;
+    tp.n1 = N >> tp.lc;
     if (dense || N == 0) {
         tp.b_start = 0;
         tp.b_len = N;
@@ -93,8 +93,8 @@ __device__ __forceinline__ TokenPlan make_plan(const Geo &g, const int32_t *lens
         tp.nv = N;
         return tp;
     }
-    tp.cur_start = current_chunk_start(N, g.c, g.flags);
-    int64_t ns = sel->count[grp];
+    tp.cur_start = (int)current_chunk_start(N, g.c, g.flags);
+    int ns = sel->count[grp];
     if (ns < 0 || ns > g.cap[1]) {
         set_status(status, ZHA_ERR_INVALID_ARG);
         ns = 0;
@@ -102,10 +102,10 @@ __device__ __forceinline__ TokenPlan make_plan(const Geo &g, const int32_t *lens
     tp.leaf = sel->leaf_idx + grp * g.cap[1];
     tp.hmask = sel->head_mask + grp * g.cap[1];
     tp.nsel = ns;
-    tp.sel_tokens = ns * g.c;
+    tp.sel_tokens = ns << tp.lc;
     const bool has_leaf0 = ns > 0 && tp.leaf[0] == 0;
     const bool cur_complete = tp.cur_start + g.c <= N;
-    const bool cur_covered = cur_complete && ns > 0 && (int64_t)tp.leaf[ns - 1] * g.c == tp.cur_start;
+    const bool cur_covered = cur_complete && ns > 0 && (tp.leaf[ns - 1] << tp.lc) == tp.cur_start;
     tp.a_len = (!has_leaf0 && tp.cur_start > 0) ? 1 : 0;
     tp.b_start = tp.cur_start;
     tp.b_len = cur_covered ? 0 : N - tp.cur_start;
@@ -129,16 +129,54 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 // Partials: ml[((grp*S + s)*G + h)*2 + {0,1}] = (max in log2 units, sum),
 // o[((grp*S + s)*G + h)*D + dim] (unnormalised).
+
+constexpr int kTile = 64;    // tokens per pipeline stage (16 per warp)
+constexpr int kStages = 3;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+                 "r"(valid ? 16 : 0));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                          uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+template <int D>
+constexpr int attn_smem_bytes() {
+    return kStages * 2 * kTile * D * 2;
+}
+
+// bf16 split-K attention. The CTA's 128 threads stream 64-token tiles of the
+// group's token list (K and V rows, gathered by position) into a 3-stage
+// shared-memory ring with cp.async; rows are stored with their 16-byte
+// chunks XOR-swizzled by (row & 7) so that ldmatrix reads of 8 rows at one
+// column are bank-conflict free. Each warp then computes its 16 tokens.
 template <int D>
 __global__ void __launch_bounds__(kAttnWarps * 32)
 attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
                 const int32_t *lens, zha_selection sel, int dense, float *part_ml, float *part_o,
                 int32_t *status) {
-    constexpr int KP = D / 32;      // k-pairs of the QK product
-    constexpr int NJ = D / 8;       // n-tiles of the PV product
-    constexpr int DW = D / 8;       // value coordinates per lane
-    __shared__ float sm_m[kAttnWarps][16], sm_l[kAttnWarps][16];
-    __shared__ float sm_o[kAttnWarps][16][D + 4];
+    constexpr int ROWB = D * 2;            // bytes per token row
+    constexpr int CH = ROWB / 16;          // 16-byte chunks per row
+    constexpr int TILE_B = kTile * ROWB;
+    constexpr int STAGE_B = 2 * TILE_B;    // K tile then V tile
+    constexpr int NJ = D / 8;              // n-tiles of the PV product
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
 
     const int grp = blockIdx.y, split = blockIdx.x, S = gridDim.x;
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
@@ -149,16 +187,53 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     const __nv_bfloat16 *Vg = V + (int64_t)grp * g.max_len * D;
 
     // Q as the A operand: rows gq and gq+8 are heads of this group (rows >= G are zero)
-    uint32_t qa[KP][4], qb[KP][4];  // k16 steps 2kp and 2kp+1
+    uint32_t qf[D / 16][4];
     const int h0 = gq, h1 = gq + 8;
+    {
+        const uint32_t *q0 = reinterpret_cast<const uint32_t *>(q + ((int64_t)b * g.Hq + kvh * g.G + h0) * D);
+        const uint32_t *q1 = reinterpret_cast<const uint32_t *>(q + ((int64_t)b * g.Hq + kvh * g.G + h1) * D);
 #pragma unroll
-    for (int kp = 0; kp < KP; ++kp) {
-        uint4 w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
-        if (h0 < g.G) w0 = *reinterpret_cast<const uint4 *>(q + ((int64_t)b * g.Hq + kvh * g.G + h0) * D + kp * 32 + t * 8);
-        if (h1 < g.G) w1 = *reinterpret_cast<const uint4 *>(q + ((int64_t)b * g.Hq + kvh * g.G + h1) * D + kp * 32 + t * 8);
-        qa[kp][0] = w0.x; qa[kp][1] = w1.x; qa[kp][2] = w0.y; qa[kp][3] = w1.y;
-        qb[kp][0] = w0.z; qb[kp][1] = w1.z; qb[kp][2] = w0.w; qb[kp][3] = w1.w;
+        for (int st = 0; st < D / 16; ++st) {
+            qf[st][0] = h0 < g.G ? q0[st * 8 + t] : 0u;
+            qf[st][1] = h1 < g.G ? q1[st * 8 + t] : 0u;
+            qf[st][2] = h0 < g.G ? q0[st * 8 + 4 + t] : 0u;
+            qf[st][3] = h1 < g.G ? q1[st * 8 + 4 + t] : 0u;
+        }
     }
+
+    const int ntiles = (tp.nv + kTile - 1) / kTile;
+    const int t_lo = (int)((int64_t)ntiles * split / S), t_hi = (int)((int64_t)ntiles * (split + 1) / S);
+
+    // Cache positions and head masks of the next tiles, resolved one iteration
+    // ahead of their copies (by threads 0..63, one row each) so that the
+    // lookups' latency overlaps a whole tile of compute.
+    constexpr int kSlots = kStages + 1;
+    __shared__ int spos[kSlots][kTile];
+    __shared__ uint32_t smask[kSlots][kTile];
+    auto resolve = [&](int tile, int slot) {
+        if (threadIdx.x < kTile) {
+            const int v = tile * kTile + threadIdx.x;
+            int pos;
+            uint32_t m;
+            tp.at(v, pos, m, status);
+            spos[slot][threadIdx.x] = pos;
+            smask[slot][threadIdx.x] = v < tp.nv ? m : 0u;
+        }
+    };
+    // 16 threads per row of a tile: one 16-byte chunk of K and of V each
+    auto issue = [&](int tile, int stage, int slot) {
+        const uint32_t kb = sbase + stage * STAGE_B, vb = kb + TILE_B;
+#pragma unroll
+        for (int k = 0; k < kTile * CH / (kAttnWarps * 32); ++k) {
+            const int c = threadIdx.x + k * kAttnWarps * 32;
+            const int row = c / CH, ch = c % CH;
+            const int pos = spos[slot][row];
+            const bool valid = tile * kTile + row < tp.nv;
+            const uint32_t off = row * ROWB + ((ch ^ (row & 7)) << 4);
+            cp_async16(kb + off, Kg + (int64_t)pos * D + ch * 8, valid);
+            cp_async16(vb + off, Vg + (int64_t)pos * D + ch * 8, valid);
+        }
+    };
 
     const float sl2 = g.s * kLog2e;
     float m_run[2] = {-INFINITY, -INFINITY};
@@ -166,51 +241,50 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     float o[NJ][4];
 #pragma unroll
     for (int j = 0; j < NJ; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    const uint32_t mrow[2] = {h0 < g.G ? (1u << h0) : 0u, h1 < g.G ? (1u << h1) : 0u};
 
-    const int64_t W = (tp.nv + 15) / 16;
-    const int64_t w_lo = W * split / S, w_hi = W * (split + 1) / S;
-    for (int64_t wt = w_lo + warp; wt < w_hi; wt += kAttnWarps) {
-        const int64_t v0 = wt * 16;
-        // K rows this lane feeds to the QK product: tokens gq and 8+gq
-        int64_t pk0, pk1;
-        uint32_t mk0, mk1;
-        tp.at(v0 + gq, pk0, mk0, status);
-        tp.at(v0 + 8 + gq, pk1, mk1, status);
-        if (v0 + gq >= tp.nv) mk0 = 0u;
-        if (v0 + 8 + gq >= tp.nv) mk1 = 0u;
-        // tokens of this lane's S columns and V rows: 2t, 2t+1, 8+2t, 9+2t
-        int64_t pv[4];
+    // tile t_lo + i: copies in stage i % kStages, positions in slot i % kSlots
+#pragma unroll
+    for (int st = 0; st < kStages; ++st)
+        if (t_lo + st < t_hi) resolve(t_lo + st, st);
+    __syncthreads();
+#pragma unroll
+    for (int st = 0; st < kStages - 1; ++st) {
+        if (t_lo + st < t_hi) issue(t_lo + st, st, st);
+        cp_async_commit();
+    }
+    for (int it = 0; t_lo + it < t_hi; ++it) {
+        cp_async_wait<kStages - 2>();
+        __syncthreads();
+        {
+            const int nt = t_lo + it + kStages - 1;
+            if (nt < t_hi) issue(nt, (it + kStages - 1) % kStages, (it + kStages - 1) % kSlots);
+            cp_async_commit();
+        }
+        // look up the tile after that now; its slot was last read by tile it - 1
+        if (t_lo + it + kStages < t_hi) resolve(t_lo + it + kStages, (it + kStages) % kSlots);
+        const int stage = it % kStages;
+        const uint32_t kb = sbase + stage * STAGE_B, vb = kb + TILE_B;
+        const int row0 = warp * 16;
+        // heads that see this lane's S columns / V rows: tokens 2t, 2t+1, 8+2t, 9+2t
         uint32_t mv[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int64_t v = v0 + (u >> 1) * 8 + 2 * t + (u & 1);
-            tp.at(v, pv[u], mv[u], status);
-            if (v >= tp.nv) mv[u] = 0u;
-        }
-        uint4 kr0[KP], kr1[KP];
-#pragma unroll
-        for (int kp = 0; kp < KP; ++kp) {
-            kr0[kp] = *reinterpret_cast<const uint4 *>(Kg + pk0 * D + kp * 32 + t * 8);
-            kr1[kp] = *reinterpret_cast<const uint4 *>(Kg + pk1 * D + kp * 32 + t * 8);
-        }
-        uint4 vr[4][DW / 8];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-            for (int x = 0; x < DW / 8; ++x)
-                vr[u][x] = *reinterpret_cast<const uint4 *>(Vg + pv[u] * D + gq * DW + x * 8);
-
+        for (int u = 0; u < 4; ++u) mv[u] = smask[it % kSlots][row0 + (u >> 1) * 8 + 2 * t + (u & 1)];
         float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int kp = 0; kp < KP; ++kp) {
-            mma16816(s0, qa[kp][0], qa[kp][1], qa[kp][2], qa[kp][3], kr0[kp].x, kr0[kp].y);
-            mma16816(s0, qb[kp][0], qb[kp][1], qb[kp][2], qb[kp][3], kr0[kp].z, kr0[kp].w);
-            mma16816(s1, qa[kp][0], qa[kp][1], qa[kp][2], qa[kp][3], kr1[kp].x, kr1[kp].y);
-            mma16816(s1, qb[kp][0], qb[kp][1], qb[kp][2], qb[kp][3], kr1[kp].z, kr1[kp].w);
+        for (int kp = 0; kp < D / 32; ++kp) {
+            uint32_t b0, b1, b2, b3;
+            const int ch = 4 * kp + (lane >> 3);
+            int row = row0 + (lane & 7);
+            ldsm_x4(kb + row * ROWB + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
+            mma16816(s0, qf[2 * kp][0], qf[2 * kp][1], qf[2 * kp][2], qf[2 * kp][3], b0, b1);
+            mma16816(s0, qf[2 * kp + 1][0], qf[2 * kp + 1][1], qf[2 * kp + 1][2], qf[2 * kp + 1][3], b2, b3);
+            row += 8;
+            ldsm_x4(kb + row * ROWB + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
+            mma16816(s1, qf[2 * kp][0], qf[2 * kp][1], qf[2 * kp][2], qf[2 * kp][3], b0, b1);
+            mma16816(s1, qf[2 * kp + 1][0], qf[2 * kp + 1][1], qf[2 * kp + 1][2], qf[2 * kp + 1][3], b2, b3);
         }
-        // s0: (head gq, tok 2t), (gq, 2t+1), (gq+8, 2t), (gq+8, 2t+1); s1: same for tokens 8+
-        float x[2][4];  // [row][token u]
-        const uint32_t mrow[2] = {h0 < g.G ? (1u << h0) : 0u, h1 < g.G ? (1u << h1) : 0u};
+        float x[2][4];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             x[r][0] = (mv[0] & mrow[r]) ? s0[2 * r + 0] * sl2 : -INFINITY;
@@ -244,37 +318,40 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
         const uint32_t pa1 = pack_bf16(p[1][0], p[1][1]);
         const uint32_t pa2 = pack_bf16(p[0][2], p[0][3]);
         const uint32_t pa3 = pack_bf16(p[1][2], p[1][3]);
-        // V as B: k = tokens (2t, 2t+1 | 8+2t, 9+2t), n = value coordinate gq*DW + j
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-            const int x8 = j >> 3, wi = (j & 7) >> 1;
-            const uint32_t w0 = (&vr[0][x8].x)[wi], w1 = (&vr[1][x8].x)[wi];
-            const uint32_t w2 = (&vr[2][x8].x)[wi], w3 = (&vr[3][x8].x)[wi];
-            const uint32_t sel_lo = (j & 1) ? 0x7632u : 0x5410u;
-            const uint32_t b0 = __byte_perm(w0, w1, sel_lo);
-            const uint32_t b1 = __byte_perm(w2, w3, sel_lo);
-            mma16816(o[j], pa0, pa1, pa2, pa3, b0, b1);
+        for (int jp = 0; jp < NJ / 2; ++jp) {
+            uint32_t b0, b1, b2, b3;
+            const int row = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int ch = 2 * jp + (lane >> 4);
+            ldsm_x4_t(vb + row * ROWB + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
+            mma16816(o[2 * jp], pa0, pa1, pa2, pa3, b0, b1);
+            mma16816(o[2 * jp + 1], pa0, pa1, pa2, pa3, b2, b3);
         }
     }
-    // row sums across the 4 lanes of a row
+    cp_async_wait<0>();
+    __syncthreads();
+    // row sums across the 4 lanes of a row, then the 4 warps' partials via shared memory
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
         l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
     }
-    // o[j]: (row gq, coord (2t)*DW + j), (gq, (2t+1)*DW + j), (gq+8, ...), (gq+8, ...)
+    float *sm_m = reinterpret_cast<float *>(smem);                 // [warps][16]
+    float *sm_l = sm_m + kAttnWarps * 16;                           // [warps][16]
+    float *sm_o = sm_l + kAttnWarps * 16;                           // [warps][16][D + 4]
+    constexpr int OS = D + 4;
     if (t == 0) {
-        sm_m[warp][gq] = m_run[0];
-        sm_m[warp][gq + 8] = m_run[1];
-        sm_l[warp][gq] = l_run[0];
-        sm_l[warp][gq + 8] = l_run[1];
+        sm_m[warp * 16 + gq] = m_run[0];
+        sm_m[warp * 16 + gq + 8] = m_run[1];
+        sm_l[warp * 16 + gq] = l_run[0];
+        sm_l[warp * 16 + gq + 8] = l_run[1];
     }
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
-        sm_o[warp][gq][(2 * t) * DW + j] = o[j][0];
-        sm_o[warp][gq][(2 * t + 1) * DW + j] = o[j][1];
-        sm_o[warp][gq + 8][(2 * t) * DW + j] = o[j][2];
-        sm_o[warp][gq + 8][(2 * t + 1) * DW + j] = o[j][3];
+        sm_o[(warp * 16 + gq) * OS + 8 * j + 2 * t] = o[j][0];
+        sm_o[(warp * 16 + gq) * OS + 8 * j + 2 * t + 1] = o[j][1];
+        sm_o[(warp * 16 + gq + 8) * OS + 8 * j + 2 * t] = o[j][2];
+        sm_o[(warp * 16 + gq + 8) * OS + 8 * j + 2 * t + 1] = o[j][3];
     }
     __syncthreads();
     const int64_t pbase = ((int64_t)grp * S + split) * g.G;
@@ -282,15 +359,16 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
         const int h = i / D, dim = i % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, sm_m[w][h]);
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, sm_m[w * 16 + h]);
         float L = 0.f, acc = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < kAttnWarps; ++w) {
-                if (sm_m[w][h] == -INFINITY) continue;
-                const float f = exp2f(sm_m[w][h] - M);
-                L += sm_l[w][h] * f;
-                acc += sm_o[w][h][dim] * f;
+                const float mw = sm_m[w * 16 + h];
+                if (mw == -INFINITY) continue;
+                const float f = exp2f(mw - M);
+                L += sm_l[w * 16 + h] * f;
+                acc += sm_o[(w * 16 + h) * OS + dim] * f;
             }
         }
         part_o[(pbase + h) * D + dim] = acc;
@@ -329,18 +407,18 @@ attn_simt_kernel(Geo g, const T *q, const T *K, const T *V, const int32_t *lens,
 #pragma unroll
         for (int e = 0; e < DL; ++e) o[h][e] = 0.f;
     }
-    const int64_t W = (tp.nv + 31) / 32;
-    const int64_t w_lo = W * split / S, w_hi = W * (split + 1) / S;
-    for (int64_t wt = w_lo + warp; wt < w_hi; wt += kAttnWarps) {
-        const int64_t v = wt * 32 + lane;
-        int64_t pos;
+    const int W = (tp.nv + 31) / 32;
+    const int w_lo = (int)((int64_t)W * split / S), w_hi = (int)((int64_t)W * (split + 1) / S);
+    for (int wt = w_lo + warp; wt < w_hi; wt += kAttnWarps) {
+        const int v = wt * 32 + lane;
+        int pos;
         uint32_t mask;
         tp.at(v, pos, mask, status);
         if (v >= tp.nv) mask = 0u;
         float sc[16];
 #pragma unroll
         for (int h = 0; h < 16; ++h) sc[h] = 0.f;
-        const T *kr = Kg + pos * D;
+        const T *kr = Kg + (int64_t)pos * D;
         for (int k = 0; k < D; ++k) {
             const float kv = to_f32(kr[k]);
 #pragma unroll
@@ -449,11 +527,24 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
         auto kk = static_cast<const __nv_bfloat16 *>(K);
         auto vv = static_cast<const __nv_bfloat16 *>(V);
         {
-        ProfScope ps(attn_name, st);
-        if (g.d == 128)
-            attn_mma_kernel<128><<<grid, kAttnWarps * 32, 0, st>>>(g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
-        else
-            attn_mma_kernel<64><<<grid, kAttnWarps * 32, 0, st>>>(g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
+            // the shared-memory opt-in is a per-device function attribute
+            static bool attr_set[64] = {};
+            int dev = 0;
+            cudaGetDevice(&dev);
+            if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+                cudaFuncSetAttribute(attn_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     attn_smem_bytes<128>());
+                cudaFuncSetAttribute(attn_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     attn_smem_bytes<64>());
+                attr_set[dev] = true;
+            }
+            ProfScope ps(attn_name, st);
+            if (g.d == 128)
+                attn_mma_kernel<128><<<grid, kAttnWarps * 32, attn_smem_bytes<128>(), st>>>(
+                    g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
+            else
+                attn_mma_kernel<64><<<grid, kAttnWarps * 32, attn_smem_bytes<64>(), st>>>(
+                    g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;

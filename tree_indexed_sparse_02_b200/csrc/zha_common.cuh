@@ -28,14 +28,16 @@ struct Geo {
     int64_t max_len;
     float s;
     int64_t cap[kMaxLevels + 1];        // nodes per level at max_len (index = level)
+    int64_t capv[kMaxLevels + 1];       // candidate slots per level: cap + c (padding children)
     size_t mu_off[kMaxLevels + 1];      // tree buffer offsets
     size_t bias_off[kMaxLevels + 1];
     size_t tree_bytes;
     // workspace
     size_t ws_cand[kMaxLevels + 1], ws_cmask[kMaxLevels + 1], ws_scores[kMaxLevels + 1],
-        ws_kept[kMaxLevels + 1], ws_count[kMaxLevels + 1];
-    size_t ws_maxkey;                   // [L][B*Hkv][G] u32
-    size_t ws_levelkept;                // [B*Hkv][G][L] i32
+        ws_kept[kMaxLevels + 1], ws_count[kMaxLevels + 1];     // candidates of a level
+    size_t ws_plist[kMaxLevels + 1], ws_pmask[kMaxLevels + 1], ws_pcount[kMaxLevels + 1];  // kept
+    size_t ws_maxkey, ws_minkey;        // [L][B*Hkv][G] u32 ordered keys of the scores
+    size_t ws_done;                     // [L][B*Hkv] u32 finished select CTAs
     size_t ws_part_ml, ws_part_o;       // split-K partials
     size_t ws_bytes;
     __host__ __device__ int groups() const { return B * Hkv; }

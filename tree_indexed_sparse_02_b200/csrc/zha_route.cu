@@ -7,16 +7,21 @@
 // KV entries. Section "Building the tree": a node's estimate is the max over
 // its reference planes, E = max_r (s q.mu_r + bias_r).
 //
-// Per level, for all (sequence, KV head) groups at once:
-//   score  -- every candidate node of a group is read once and scored for all
-//             G query heads of the group (mma.sync bf16 tiles: planes x heads);
+// Per level, for all (sequence, KV head) groups at once, two launches:
+//   score  -- candidate i of a group is child i % c of the (i / c)-th node
+//             the group kept one level up (all nodes at the top level); each
+//             candidate's summary is read once and scored for all G query
+//             heads of the group on tensor cores (mma.sync bf16: planes x
+//             heads), and the per-head max and min score are kept;
 //   select -- one CTA per (group, query head): exact threshold search for the
 //             shortest (score desc, index asc) prefix holding p of the mass,
-//             as a 3-pass radix select on the fp32 score bits with masses
-//             summed in 2^-40 fixed point (exact, order-independent sums);
-//   expand -- one CTA per group: the existing children of the nodes kept by
-//             any head become the next level's candidates (ascending), each
-//             carrying the bit mask of heads that kept its parent.
+//             a radix select over the score's distance below the max (the
+//             range is known, so 12-bit digits are spread over buckets that
+//             are actually used) with masses summed in 2^-31 fixed point
+//             (exact and order-independent); kept bits are OR-ed per
+//             candidate, and the last CTA of a group to finish compacts the
+//             candidates some head kept into the next level's parent list
+//             (or, at level 1, into the selection).
 #include "zha_common.cuh"
 
 namespace zha {
@@ -26,47 +31,78 @@ namespace {
 // ------------------------------------------------------------------ level views
 
 struct LevelWs {
-    int32_t *cand;
-    uint32_t *cmask;
-    float *scores;
-    uint32_t *kept;
-    int32_t *count;
+    int32_t *cand;      // [groups][capv] node index of candidate i
+    uint32_t *cmask;    // [groups][capv] heads that have it as a candidate (0 = padding)
+    float *scores;      // [groups][G][capv]
+    uint32_t *kept;     // [groups][capv] heads that kept it
+    int32_t *count;     // [groups] candidate entries in use
+    int32_t *plist;     // [groups][cap] nodes kept by some head, ascending
+    uint32_t *pmask;    // [groups][cap] heads that kept them
+    int32_t *pcount;    // [groups]
+    uint32_t *maxkey;   // [groups][G]
+    uint32_t *minkey;   // [groups][G]
+    uint32_t *done;     // [groups]
 };
 
-__host__ __device__ inline LevelWs level_ws(const Geo &g, void *ws, int l) {
+inline LevelWs level_ws(const Geo &g, void *ws, int l) {
     char *base = static_cast<char *>(ws);
+    const size_t lg = (size_t)(l - 1) * g.groups();
     LevelWs v;
     v.cand = reinterpret_cast<int32_t *>(base + g.ws_cand[l]);
     v.cmask = reinterpret_cast<uint32_t *>(base + g.ws_cmask[l]);
     v.scores = reinterpret_cast<float *>(base + g.ws_scores[l]);
     v.kept = reinterpret_cast<uint32_t *>(base + g.ws_kept[l]);
     v.count = reinterpret_cast<int32_t *>(base + g.ws_count[l]);
+    v.plist = reinterpret_cast<int32_t *>(base + g.ws_plist[l]);
+    v.pmask = reinterpret_cast<uint32_t *>(base + g.ws_pmask[l]);
+    v.pcount = reinterpret_cast<int32_t *>(base + g.ws_pcount[l]);
+    v.maxkey = reinterpret_cast<uint32_t *>(base + g.ws_maxkey) + lg * g.G;
+    v.minkey = reinterpret_cast<uint32_t *>(base + g.ws_minkey) + lg * g.G;
+    v.done = reinterpret_cast<uint32_t *>(base + g.ws_done) + lg;
     return v;
 }
 
 __device__ __forceinline__ uint32_t all_heads(int G) { return G >= 32 ? 0xffffffffu : ((1u << G) - 1u); }
 
+// Candidate i of a group at a level: its node and the heads it is a candidate for.
+struct CandSource {
+    int lc;                   // log2(c)
+    int top;                  // top level: candidate i is node i, for every head
+    int n_here;               // nodes at this level
+    const int32_t *plist;     // nodes kept one level up
+    const uint32_t *pmask;
+    __device__ __forceinline__ void at(int i, int &node, uint32_t &mask, uint32_t all) const {
+        if (top) {
+            node = i;
+            mask = all;
+            return;
+        }
+        const int j = i >> lc;
+        node = (__ldg(&plist[j]) << lc) | (i & ((1 << lc) - 1));
+        mask = node < n_here ? __ldg(&pmask[j]) : 0u;
+    }
+};
+
+__device__ __forceinline__ int64_t group_len(const Geo &g, const int32_t *lens, int grp) {
+    const int64_t N = lens[grp / g.Hkv];
+    return (N < 0 || N > g.max_len) ? 0 : N;
+}
+
 // ----------------------------------------------------------------------- init
 
-__global__ void route_init_kernel(Geo g, LevelWs top, const int32_t *lens, uint32_t *maxkey,
-                                  int32_t *status) {
+__global__ void route_init_kernel(Geo g, uint32_t *maxkey, uint32_t *minkey, uint32_t *done,
+                                  const int32_t *lens, int32_t *status) {
     const int grp = blockIdx.x;
-    const int b = grp / g.Hkv;
-    int64_t N = lens[b];
-    if (N < 0 || N > g.max_len) {
-        if (threadIdx.x == 0) set_status(status, ZHA_ERR_CAPACITY);
-        N = 0;
+    if (threadIdx.x == 0) {
+        const int64_t N = lens[grp / g.Hkv];
+        if (N < 0 || N > g.max_len) set_status(status, ZHA_ERR_CAPACITY);
     }
-    const int64_t nL = level_nodes(N, g.c, g.L);
-    const int64_t cap = g.cap[g.L];
-    for (int64_t i = threadIdx.x; i < nL; i += blockDim.x) {
-        top.cand[grp * cap + i] = (int32_t)i;
-        top.cmask[grp * cap + i] = all_heads(g.G);
-        top.kept[grp * cap + i] = 0u;
+    for (int i = threadIdx.x; i < g.L * g.G; i += blockDim.x) {
+        const int64_t at = ((int64_t)(i / g.G) * g.groups() + grp) * g.G + i % g.G;
+        maxkey[at] = 0u;
+        minkey[at] = 0xffffffffu;
     }
-    if (threadIdx.x == 0) top.count[grp] = (int32_t)nL;
-    for (int i = threadIdx.x; i < g.L * g.G; i += blockDim.x)
-        maxkey[((int64_t)(i / g.G) * g.groups() + grp) * g.G + i % g.G] = 0u;
+    for (int l = threadIdx.x; l < g.L; l += blockDim.x) done[(int64_t)l * g.groups() + grp] = 0u;
 }
 
 // ---------------------------------------------------------------------- score
@@ -86,7 +122,19 @@ __device__ __forceinline__ uint4 ldg16(const void *p) {
 
 constexpr int kScoreWarps = 4;
 
-// bf16 scoring on tensor cores. One warp scores one node per iteration:
+__device__ __forceinline__ CandSource cand_source(const Geo &g, const LevelWs &up, int level,
+                                                  int grp, int64_t N) {
+    const int64_t cap_up = level < g.L ? g.cap[level + 1] : 0;
+    return CandSource{__ffs(g.c) - 1, level == g.L, (int)level_nodes(N, g.c, level),
+                      up.plist + grp * cap_up, up.pmask + grp * cap_up};
+}
+
+__device__ __forceinline__ int64_t cand_count(const Geo &g, const LevelWs &up, int level, int grp,
+                                              int64_t n_here) {
+    return level == g.L ? n_here : (int64_t)up.pcount[grp] * g.c;
+}
+
+// bf16 scoring on tensor cores. One warp scores one candidate per iteration:
 // A = the node's planes (16 rows per m-tile, K = head_dim), B = the group's
 // query heads (8 columns per n-tile). Coordinates are permuted identically in
 // A and B so that each lane fetches 16 contiguous bytes per row and k-pair
@@ -94,14 +142,17 @@ constexpr int kScoreWarps = 4;
 template <int D, int MT, int NT>
 __global__ void __launch_bounds__(kScoreWarps * 32)
 score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_bfloat16 *q,
-                 LevelWs lw, int level, uint32_t *maxkey) {
+                 const int32_t *lens, LevelWs lw, LevelWs up, int level) {
     constexpr int KP = D / 32;
     const int grp = blockIdx.y;
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gq = lane >> 2, t = lane & 3;
-    const int64_t cap = g.cap[level];
-    const int n = lw.count[grp];
+    const int64_t cap = g.cap[level], capv = g.capv[level];
+    const CandSource src = cand_source(g, up, level, grp, group_len(g, lens, grp));
+    const int n = (int)cand_count(g, up, level, grp, src.n_here);
+    if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
+    const uint32_t all = all_heads(g.G);
 
     uint32_t bq[NT][KP][4];
 #pragma unroll
@@ -114,74 +165,112 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
             bq[nt][kp][0] = w.x; bq[nt][kp][1] = w.y; bq[nt][kp][2] = w.z; bq[nt][kp][3] = w.w;
         }
     }
-    float runmax[NT][2];
+    float runmax[NT][2], runmin[NT][2];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) runmax[nt][0] = runmax[nt][1] = -INFINITY;
+    for (int nt = 0; nt < NT; ++nt) {
+        runmax[nt][0] = runmax[nt][1] = -INFINITY;
+        runmin[nt][0] = runmin[nt][1] = INFINITY;
+    }
 
     const float s = g.s;
-    for (int i = blockIdx.x * kScoreWarps + warp; i < n; i += gridDim.x * kScoreWarps) {
-        const int64_t node = lw.cand[grp * cap + i];
-        const uint32_t hm = lw.cmask[grp * cap + i];
-        const __nv_bfloat16 *base = mu + (grp * cap + node) * (int64_t)g.R * D;
-        const float *bb = bias + (grp * cap + node) * (int64_t)g.R;
-        uint4 ra[MT][KP], rb[MT][KP];
+    // U candidates per warp and iteration, their loads issued together
+    constexpr int U = 2;
+    const int stride = gridDim.x * kScoreWarps * U;
+    for (int i0 = (blockIdx.x * kScoreWarps + warp) * U; i0 < n; i0 += stride) {
+        int node[U];
+        uint32_t hm[U];
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            const int r0 = mt * 16 + gq, r1 = r0 + 8;
-#pragma unroll
-            for (int kp = 0; kp < KP; ++kp) {
-                ra[mt][kp] = r0 < g.R ? ldg16(base + (int64_t)r0 * D + kp * 32 + t * 8) : make_uint4(0, 0, 0, 0);
-                rb[mt][kp] = r1 < g.R ? ldg16(base + (int64_t)r1 * D + kp * 32 + t * 8) : make_uint4(0, 0, 0, 0);
-            }
-        }
-        float e[NT][2];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) e[nt][0] = e[nt][1] = -INFINITY;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            float acc[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll
-            for (int kp = 0; kp < KP; ++kp) {
-                const uint32_t a0[4] = {ra[mt][kp].x, rb[mt][kp].x, ra[mt][kp].y, rb[mt][kp].y};
-                const uint32_t a1[4] = {ra[mt][kp].z, rb[mt][kp].z, ra[mt][kp].w, rb[mt][kp].w};
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    mma_bf16_16816(acc[nt], a0, bq[nt][kp][0], bq[nt][kp][1]);
-                    mma_bf16_16816(acc[nt], a1, bq[nt][kp][2], bq[nt][kp][3]);
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u;
+            node[u] = 0;
+            hm[u] = 0u;
+            if (i < n) {
+                src.at(i, node[u], hm[u], all);
+                if (lane == 0) {
+                    lw.cand[grp * capv + i] = node[u];
+                    lw.cmask[grp * capv + i] = hm[u];
+                    lw.kept[grp * capv + i] = 0u;
                 }
             }
-            const int r0 = mt * 16 + gq, r1 = r0 + 8;
-            const float b0 = r0 < g.R ? bb[r0] : -INFINITY;
-            const float b1 = r1 < g.R ? bb[r1] : -INFINITY;
+        }
+        uint4 ra[U][MT][KP], rb[U][MT][KP];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                e[nt][0] = fmaxf(e[nt][0], fmaxf(fmaf(s, acc[nt][0], b0), fmaf(s, acc[nt][2], b1)));
-                e[nt][1] = fmaxf(e[nt][1], fmaxf(fmaf(s, acc[nt][1], b0), fmaf(s, acc[nt][3], b1)));
+        for (int u = 0; u < U; ++u) {
+            const __nv_bfloat16 *base = mu + (grp * cap + node[u]) * (int64_t)g.R * D;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int r0 = mt * 16 + gq, r1 = r0 + 8;
+#pragma unroll
+                for (int kp = 0; kp < KP; ++kp) {
+                    ra[u][mt][kp] = (hm[u] && r0 < g.R) ? ldg16(base + (int64_t)r0 * D + kp * 32 + t * 8)
+                                                        : make_uint4(0, 0, 0, 0);
+                    rb[u][mt][kp] = (hm[u] && r1 < g.R) ? ldg16(base + (int64_t)r1 * D + kp * 32 + t * 8)
+                                                        : make_uint4(0, 0, 0, 0);
+                }
             }
         }
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                float v = e[nt][j];
-                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-                e[nt][j] = v;
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u;
+            if (i >= n) break;
+            if (hm[u] == 0u) {
+                if (lane < g.G) lw.scores[(grp * g.G + lane) * capv + i] = -INFINITY;
+                continue;
             }
-        if (gq == 0) {
+            const float *bb = bias + (grp * cap + node[u]) * (int64_t)g.R;
+            float e[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) e[nt][0] = e[nt][1] = -INFINITY;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                float acc[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+                for (int kp = 0; kp < KP; ++kp) {
+                    const uint4 &xa = ra[u][mt][kp], &xb = rb[u][mt][kp];
+                    const uint32_t a0[4] = {xa.x, xb.x, xa.y, xb.y};
+                    const uint32_t a1[4] = {xa.z, xb.z, xa.w, xb.w};
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        mma_bf16_16816(acc[nt], a0, bq[nt][kp][0], bq[nt][kp][1]);
+                        mma_bf16_16816(acc[nt], a1, bq[nt][kp][2], bq[nt][kp][3]);
+                    }
+                }
+                const int r0 = mt * 16 + gq, r1 = r0 + 8;
+                const float b0 = r0 < g.R ? bb[r0] : -INFINITY;
+                const float b1 = r1 < g.R ? bb[r1] : -INFINITY;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    e[nt][0] = fmaxf(e[nt][0], fmaxf(fmaf(s, acc[nt][0], b0), fmaf(s, acc[nt][2], b1)));
+                    e[nt][1] = fmaxf(e[nt][1], fmaxf(fmaf(s, acc[nt][1], b0), fmaf(s, acc[nt][3], b1)));
+                }
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int h = nt * 8 + 2 * t + j;
-                    if (h < g.G) {
-                        lw.scores[(grp * g.G + h) * cap + i] = e[nt][j];
-                        if ((hm >> h) & 1u) runmax[nt][j] = fmaxf(runmax[nt][j], e[nt][j]);
-                    }
+                    float v = e[nt][j];
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                    e[nt][j] = v;
                 }
+            if (gq == 0) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int h = nt * 8 + 2 * t + j;
+                        if (h < g.G) {
+                            lw.scores[(grp * g.G + h) * capv + i] = e[nt][j];
+                            if ((hm[u] >> h) & 1u) {
+                                runmax[nt][j] = fmaxf(runmax[nt][j], e[nt][j]);
+                                runmin[nt][j] = fminf(runmin[nt][j], e[nt][j]);
+                            }
+                        }
+                    }
+            }
         }
     }
     if (gq == 0) {
@@ -190,30 +279,45 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int h = nt * 8 + 2 * t + j;
-                if (h < g.G && runmax[nt][j] > -INFINITY)
-                    atomicMax(&maxkey[(int64_t)grp * g.G + h], ordered_key(runmax[nt][j]));
+                if (h < g.G && runmax[nt][j] > -INFINITY) {
+                    atomicMax(&lw.maxkey[(int64_t)grp * g.G + h], ordered_key(runmax[nt][j]));
+                    atomicMin(&lw.minkey[(int64_t)grp * g.G + h], ordered_key(runmin[nt][j]));
+                }
             }
     }
 }
 
-// fp32 scoring on CUDA cores: one block per node per iteration, one thread
-// per (plane, head) dot product.
+// fp32 scoring on CUDA cores: one block per candidate per iteration, one
+// thread per (plane, head) dot product.
 template <int D>
 __global__ void score_f32_kernel(Geo g, const float *mu, const float *bias, const float *q,
-                                 LevelWs lw, int level, uint32_t *maxkey) {
+                                 const int32_t *lens, LevelWs lw, LevelWs up, int level) {
     __shared__ float qs[16][D];
     __shared__ float es[32][16];
     const int grp = blockIdx.y;
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
-    const int64_t cap = g.cap[level];
-    const int n = lw.count[grp];
+    const int64_t cap = g.cap[level], capv = g.capv[level];
+    const CandSource src = cand_source(g, up, level, grp, group_len(g, lens, grp));
+    const int n = (int)cand_count(g, up, level, grp, src.n_here);
+    if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
+    const uint32_t all = all_heads(g.G);
     for (int i = threadIdx.x; i < g.G * D; i += blockDim.x)
         qs[i / D][i % D] = q[((int64_t)b * g.Hq + kvh * g.G + i / D) * D + i % D];
-    float runmax = -INFINITY;
+    float runmax = -INFINITY, runmin = INFINITY;
     __syncthreads();
     for (int i = blockIdx.x; i < n; i += gridDim.x) {
-        const int64_t node = lw.cand[grp * cap + i];
-        const uint32_t hm = lw.cmask[grp * cap + i];
+        int node;
+        uint32_t hm;
+        src.at(i, node, hm, all);
+        if (threadIdx.x == 0) {
+            lw.cand[grp * capv + i] = (int32_t)node;
+            lw.cmask[grp * capv + i] = hm;
+            lw.kept[grp * capv + i] = 0u;
+        }
+        if (hm == 0u) {
+            if (threadIdx.x < g.G) lw.scores[(grp * g.G + threadIdx.x) * capv + i] = -INFINITY;
+            continue;  // uniform across the block
+        }
         const float *base = mu + (grp * cap + node) * (int64_t)g.R * D;
         const float *bb = bias + (grp * cap + node) * (int64_t)g.R;
         for (int pr = threadIdx.x; pr < g.R * g.G; pr += blockDim.x) {
@@ -227,25 +331,39 @@ __global__ void score_f32_kernel(Geo g, const float *mu, const float *bias, cons
             const int h = threadIdx.x;
             float e = -INFINITY;
             for (int r = 0; r < g.R; ++r) e = fmaxf(e, es[r][h]);
-            lw.scores[(grp * g.G + h) * cap + i] = e;
-            if ((hm >> h) & 1u) runmax = fmaxf(runmax, e);
+            lw.scores[(grp * g.G + h) * capv + i] = e;
+            if ((hm >> h) & 1u) {
+                runmax = fmaxf(runmax, e);
+                runmin = fminf(runmin, e);
+            }
         }
         __syncthreads();
     }
-    if (threadIdx.x < g.G && runmax > -INFINITY)
-        atomicMax(&maxkey[(int64_t)grp * g.G + threadIdx.x], ordered_key(runmax));
+    if (threadIdx.x < g.G && runmax > -INFINITY) {
+        atomicMax(&lw.maxkey[(int64_t)grp * g.G + threadIdx.x], ordered_key(runmax));
+        atomicMin(&lw.minkey[(int64_t)grp * g.G + threadIdx.x], ordered_key(runmin));
+    }
 }
 
 // --------------------------------------------------------------------- select
 
 constexpr int kSelThreads = 512;
-constexpr int kBuckets = 2048;
+constexpr int kDigitBits = 12;
+constexpr int kBuckets = 1 << kDigitBits;
 constexpr int kMaxTies = 1024;
-// masses e^{E - max} in (0, 1] are summed as integers in units of 2^-40
-constexpr float kMassScale = 1099511627776.0f;
+// masses e^{E - max} in (0, 1] are summed exactly as integers in units of
+// 2^-31 (per-candidate rounding error <= 2^-32)
+constexpr float kMassScale = 2147483648.0f;
 
-__device__ __forceinline__ unsigned long long fixed_mass(float e, float m) {
-    return __float2ull_rn(expf(e - m) * kMassScale);
+__device__ __forceinline__ uint32_t fixed_mass(float e, float m) {
+    return __float2uint_rn(expf(e - m) * kMassScale);
+}
+
+// 64-bit histogram bucket from native 32-bit shared atomics: the low word
+// accumulates, and the one addition that wraps it bumps the carry word.
+__device__ __forceinline__ void hist_add(uint32_t *lo, uint32_t *carry, int b, uint32_t w) {
+    const uint32_t old = atomicAdd(&lo[b], w);
+    if (old > 0xffffffffu - w) atomicAdd(&carry[b], 1u);
 }
 
 template <typename V>
@@ -287,111 +405,147 @@ __device__ __forceinline__ V block_exclusive_scan(V v, V *red, V *total) {
 }
 
 struct SelShared {
-    unsigned long long hist[kBuckets];
+    uint32_t hist_lo[kBuckets];
+    uint32_t hist_hi[kBuckets];
     unsigned long long red[kSelThreads / 32];
     int32_t ties[kMaxTies];
     int32_t sorted_ties[kMaxTies];
     unsigned long long above, target;
-    uint32_t digit;
-    uint32_t maxkey;
+    uint32_t digit, kmax, kmin;
     int ntie;
+    int last;
 };
 
-// Exact top-p over the members of one candidate set:
-//   member(i)  -- candidate i belongs to this head's set
-//   score(i)   -- its fp32 estimate
-//   emit(i)    -- called once for every kept candidate
-// Returns (in every thread) the number kept.
-template <class Member, class Score, class Emit>
-__device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t maxkey_in, Member member,
-                         Score score, Emit emit) {
+// Exact top-p over the members of one candidate set, read 8 consecutive
+// candidates at a time:
+//   load8(i0, e) -- fills e[0..8) with the scores of candidates i0..i0+7 and
+//                   returns a bit mask of those that are members (and < n)
+//   emit(i)      -- called once for every kept candidate
+// kmax_in / kmin_in: ordered keys of the members' max / min score (kmax_in = 0:
+// unknown, found here). Returns (in every thread) the number kept.
+template <class Load8, class Emit>
+__device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, uint32_t kmin_in,
+                         Load8 load8, Emit emit) {
     const int tid = threadIdx.x;
-    // max over the members (passed in when the scorer already has it)
-    if (tid == 0) sh.maxkey = maxkey_in;
+    const int64_t nblk = (n + 7) >> 3;
+    if (tid == 0) {
+        sh.kmax = kmax_in;
+        sh.kmin = kmax_in ? kmin_in : 0xffffffffu;
+    }
     __syncthreads();
-    if (maxkey_in == 0u) {
-        uint32_t mk = 0u;
-        for (int64_t i = tid; i < n; i += blockDim.x)
-            if (member(i)) mk = max(mk, ordered_key(score(i)));
-        if (mk) atomicMax(&sh.maxkey, mk);
-        __syncthreads();
-    }
-    const uint32_t mk = sh.maxkey;
-    if (mk == 0u) return 0;  // no member
-    int kept = 0;
-    if (p >= 1.f) {
-        for (int64_t i = tid; i < n; i += blockDim.x)
-            if (member(i)) {
-                emit(i);
-                ++kept;
-            }
-        return (int)block_sum<unsigned long long>((unsigned long long)kept, sh.red);
-    }
-    const float m = key_to_float(mk);
-    // three radix passes (11, 11, 10 bits) find tau, the key of the crossing
-    // candidate, and `above`, the mass of all candidates with larger keys.
-    uint32_t prefix = 0u;
-    int hi_shift = 32;
-    if (tid == 0) sh.above = 0ull;
-    for (int pass = 0; pass < 3; ++pass) {
-        const int bits = pass < 2 ? 11 : 10;
-        const int shift = hi_shift - bits;
-        for (int i = tid; i < kBuckets; i += blockDim.x) sh.hist[i] = 0ull;
-        __syncthreads();
-        for (int64_t i = tid; i < n; i += blockDim.x) {
-            if (!member(i)) continue;
-            const float e = score(i);
-            const uint32_t k = ordered_key(e);
-            if (hi_shift < 32 && (k >> hi_shift) != (prefix >> hi_shift)) continue;
-            atomicAdd(&sh.hist[(k >> shift) & ((1u << bits) - 1u)], fixed_mass(e, m));
+    if (kmax_in == 0u) {
+        uint32_t mx = 0u, mn = 0xffffffffu;
+        for (int64_t blk = tid; blk < nblk; blk += blockDim.x) {
+            float e[8];
+            const uint32_t mb = load8(blk << 3, e);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+                if ((mb >> v) & 1u) {
+                    const uint32_t k = ordered_key(e[v]);
+                    mx = max(mx, k);
+                    mn = min(mn, k);
+                }
+        }
+        if (mx) {
+            atomicMax(&sh.kmax, mx);
+            atomicMin(&sh.kmin, mn);
         }
         __syncthreads();
-        if (pass == 0) {
+    }
+    const uint32_t kmax = sh.kmax, kmin = sh.kmin;
+    if (kmax == 0u) return 0;  // no member (uniform)
+    int kept = 0;
+    if (p >= 1.f) {
+        for (int64_t blk = tid; blk < nblk; blk += blockDim.x) {
+            float e[8];
+            const uint32_t mb = load8(blk << 3, e);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+                if ((mb >> v) & 1u) {
+                    emit((blk << 3) + v);
+                    ++kept;
+                }
+        }
+        return (int)block_sum<unsigned long long>((unsigned long long)kept, sh.red);
+    }
+    const float m = key_to_float(kmax);
+    // u = kmax - key: 0 for the best candidate, growing as the score falls.
+    const uint32_t span = kmax - kmin;
+    int hi = span ? 32 - __clz(span) : 0;  // bits of u that can be non-zero
+    uint32_t prefix = 0u;                   // known bits of the crossing u (bits >= hi)
+    if (tid == 0) sh.above = 0ull;
+    bool first = true;
+    do {
+        const int bits = hi < kDigitBits ? hi : kDigitBits;
+        const int shift = hi - bits;
+        for (int i = tid; i < kBuckets; i += blockDim.x) sh.hist_lo[i] = sh.hist_hi[i] = 0u;
+        __syncthreads();
+        for (int64_t blk = tid; blk < nblk; blk += blockDim.x) {
+            float e[8];
+            const uint32_t mb = load8(blk << 3, e);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                if (!((mb >> v) & 1u)) continue;
+                const uint32_t u = kmax - ordered_key(e[v]);
+                if (hi < 32 && (u >> hi) != (prefix >> hi)) continue;
+                hist_add(sh.hist_lo, sh.hist_hi, (int)((u >> shift) & ((1u << bits) - 1u)),
+                         fixed_mass(e[v], m));
+            }
+        }
+        __syncthreads();
+        if (first) {
             unsigned long long z = 0ull;
-            for (int i = tid; i < kBuckets; i += blockDim.x) z += sh.hist[i];
+            for (int i = tid; i < kBuckets; i += blockDim.x)
+                z += ((unsigned long long)sh.hist_hi[i] << 32) | sh.hist_lo[i];
             z = block_sum<unsigned long long>(z, sh.red);
             if (tid == 0) sh.target = (unsigned long long)ceil((double)p * (double)z);
             __syncthreads();
+            first = false;
         }
-        // crossing bucket: running mass from the top bucket down first reaches target
+        // crossing digit: running mass from digit 0 (best) upward first reaches target
         constexpr int per = kBuckets / kSelThreads;
         unsigned long long mine = 0ull;
 #pragma unroll
-        for (int j = 0; j < per; ++j) mine += sh.hist[tid * per + j];
-        // suffix sum over threads of higher index = total - inclusive prefix
+        for (int j = 0; j < per; ++j)
+            mine += ((unsigned long long)sh.hist_hi[tid * per + j] << 32) | sh.hist_lo[tid * per + j];
         unsigned long long tot;
         const unsigned long long excl = block_exclusive_scan<unsigned long long>(mine, sh.red, &tot);
-        unsigned long long run = sh.above + (tot - excl - mine);
+        unsigned long long run = sh.above + excl;
         const unsigned long long target = sh.target;
         __syncthreads();
 #pragma unroll
-        for (int j = per - 1; j >= 0; --j) {
+        for (int j = 0; j < per; ++j) {
             const int dgt = tid * per + j;
-            const unsigned long long hgt = sh.hist[dgt];
+            const unsigned long long hgt = ((unsigned long long)sh.hist_hi[dgt] << 32) | sh.hist_lo[dgt];
             if (hgt && run < target && run + hgt >= target) {
                 sh.digit = (uint32_t)dgt;
-                sh.above = run;  // mass strictly above this bucket
+                sh.above = run;  // mass of the candidates with smaller u
             }
             run += hgt;
         }
         __syncthreads();
         prefix |= sh.digit << shift;
-        hi_shift = shift;
-    }
+        hi = shift;
+    } while (hi > 0);
     const uint32_t tau = prefix;
     const unsigned long long above = sh.above, target = sh.target;
     if (tid == 0) sh.ntie = 0;
     __syncthreads();
-    // keys above tau are kept; ties at tau are resolved in index order
-    for (int64_t i = tid; i < n; i += blockDim.x) {
-        if (!member(i)) continue;
-        const uint32_t k = ordered_key(score(i));
-        if (k > tau) {
-            emit(i);
-            ++kept;
-        } else if (k == tau) {
-            const int slot = atomicAdd(&sh.ntie, 1);
-            if (slot < kMaxTies) sh.ties[slot] = (int32_t)i;
+    // smaller u kept; ties at tau resolved in index order
+    for (int64_t blk = tid; blk < nblk; blk += blockDim.x) {
+        float e[8];
+        const uint32_t mb = load8(blk << 3, e);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            if (!((mb >> v) & 1u)) continue;
+            const uint32_t u = kmax - ordered_key(e[v]);
+            if (u < tau) {
+                emit((blk << 3) + v);
+                ++kept;
+            } else if (u == tau) {
+                const int slot = atomicAdd(&sh.ntie, 1);
+                if (slot < kMaxTies) sh.ties[slot] = (int32_t)((blk << 3) + v);
+            }
         }
     }
     __syncthreads();
@@ -400,7 +554,7 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t maxkey_in, 
         for (int j = tid; j < ntie; j += blockDim.x) {
             int rank = 0;
             const int32_t v = sh.ties[j];
-            for (int u = 0; u < ntie; ++u) rank += sh.ties[u] < v;
+            for (int w = 0; w < ntie; ++w) rank += sh.ties[w] < v;
             sh.sorted_ties[rank] = v;
         }
         __syncthreads();
@@ -408,42 +562,119 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t maxkey_in, 
             unsigned long long cum = above;
             for (int j = 0; j < ntie && cum < target; ++j) {
                 const int32_t i = sh.sorted_ties[j];
+                float e[8];
+                load8((int64_t)i & ~int64_t(7), e);
                 emit(i);
                 ++kept;
-                cum += fixed_mass(score(i), m);
+                cum += fixed_mass(e[i & 7], m);
             }
         }
     } else if (tid == 0) {
         // more exact ties than fit: walk the whole set in index order
         unsigned long long cum = above;
-        for (int64_t i = 0; i < n && cum < target; ++i) {
-            if (!member(i) || ordered_key(score(i)) != tau) continue;
-            emit(i);
-            ++kept;
-            cum += fixed_mass(score(i), m);
+        for (int64_t blk = 0; blk < nblk && cum < target; ++blk) {
+            float e[8];
+            const uint32_t mb = load8(blk << 3, e);
+            for (int v = 0; v < 8 && cum < target; ++v) {
+                if (!((mb >> v) & 1u) || kmax - ordered_key(e[v]) != tau) continue;
+                emit((blk << 3) + v);
+                ++kept;
+                cum += fixed_mass(e[v], m);
+            }
         }
     }
     return (int)block_sum<unsigned long long>((unsigned long long)kept, sh.red);
 }
 
+// Compacts the candidates with a non-zero kept mask, in order, into
+// (out_idx, out_mask); returns the number written (every thread). The kept
+// rows are padded to a multiple of 8 entries.
+__device__ int64_t compact_kept(const uint32_t *kept, const int32_t *cand, int64_t n,
+                                int32_t *out_idx, uint32_t *out_mask, unsigned long long *red) {
+    constexpr int V = 8;
+    int64_t run = 0;
+    for (int64_t base = 0; base < n; base += (int64_t)blockDim.x * V) {
+        const int64_t i0 = base + (int64_t)threadIdx.x * V;
+        uint32_t km[V];
+        int cnt = 0;
+        if (i0 < n) {
+            const uint4 a = __ldcg(reinterpret_cast<const uint4 *>(kept + i0));
+            const uint4 b = __ldcg(reinterpret_cast<const uint4 *>(kept + i0) + 1);
+            km[0] = a.x; km[1] = a.y; km[2] = a.z; km[3] = a.w;
+            km[4] = b.x; km[5] = b.y; km[6] = b.z; km[7] = b.w;
+        } else {
+#pragma unroll
+            for (int v = 0; v < V; ++v) km[v] = 0u;
+        }
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            if (i0 + v >= n) km[v] = 0u;
+            cnt += km[v] != 0u;
+        }
+        unsigned long long tot;
+        int64_t o = run + (int64_t)block_exclusive_scan<unsigned long long>((unsigned long long)cnt, red, &tot);
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+            if (km[v]) {
+                out_idx[o] = cand[i0 + v];
+                out_mask[o] = km[v];
+                ++o;
+            }
+        run += (int64_t)tot;
+    }
+    return run;
+}
+
 __global__ void __launch_bounds__(kSelThreads)
-select_kernel(Geo g, LevelWs lw, int level, float p, const uint32_t *maxkey, int32_t *level_kept) {
+select_kernel(Geo g, LevelWs lw, int level, float p, int32_t *level_kept, zha_selection sel) {
     __shared__ SelShared sh;
     const int h = blockIdx.x, grp = blockIdx.y;
-    const int64_t cap = g.cap[level];
+    const int64_t capv = g.capv[level];
     const int64_t n = lw.count[grp];
     const uint32_t bit = 1u << h;
-    const uint32_t *cmask = lw.cmask + grp * cap;
-    const float *sc = lw.scores + (grp * g.G + h) * cap;
-    uint32_t *kept = lw.kept + grp * cap;
-    const uint32_t mk = maxkey[(int64_t)grp * g.G + h];
+    const uint32_t *cmask = lw.cmask + grp * capv;
+    const float *sc = lw.scores + (grp * g.G + h) * capv;
+    uint32_t *kept = lw.kept + grp * capv;
+    const uint32_t kmax = lw.maxkey[(int64_t)grp * g.G + h];
+    const uint32_t kmin = lw.minkey[(int64_t)grp * g.G + h];
+    // rows are padded to a multiple of 8 entries, so 8-wide loads stay in bounds
     const int nk = topp_core(
-        sh, n, p, mk, [&](int64_t i) { return (cmask[i] & bit) != 0u; },
-        [&](int64_t i) { return sc[i]; }, [&](int64_t i) { atomicOr(&kept[i], bit); });
+        sh, n, p, kmax, kmin,
+        [&](int64_t i0, float (&e)[8]) {
+            const float4 e0 = __ldg(reinterpret_cast<const float4 *>(sc + i0));
+            const float4 e1 = __ldg(reinterpret_cast<const float4 *>(sc + i0) + 1);
+            const uint4 m0 = __ldg(reinterpret_cast<const uint4 *>(cmask + i0));
+            const uint4 m1 = __ldg(reinterpret_cast<const uint4 *>(cmask + i0) + 1);
+            e[0] = e0.x; e[1] = e0.y; e[2] = e0.z; e[3] = e0.w;
+            e[4] = e1.x; e[5] = e1.y; e[6] = e1.z; e[7] = e1.w;
+            const uint32_t mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+            uint32_t mb = 0u;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) mb |= ((mm[v] & bit) != 0u && i0 + v < n) ? (1u << v) : 0u;
+            return mb;
+        },
+        [&](int64_t i) { atomicOr(&kept[i], bit); });
     if (level_kept && threadIdx.x == 0) {
         const int b = grp / g.Hkv, kvh = grp % g.Hkv;
-        level_kept[((int64_t)b * g.Hq + kvh * g.G + h) * g.L + (level - 1)] = mk ? nk : 0;
+        level_kept[((int64_t)b * g.Hq + kvh * g.G + h) * g.L + (level - 1)] = nk;
     }
+    // the last of the group's G CTAs compacts the union of the kept candidates
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) sh.last = atomicAdd(&lw.done[grp], 1u) == (uint32_t)(g.G - 1);
+    __syncthreads();
+    if (!sh.last) return;
+    __threadfence();
+    if (level > 1) {
+        const int64_t m = compact_kept(kept, lw.cand + grp * capv, n, lw.plist + grp * g.cap[level],
+                                       lw.pmask + grp * g.cap[level], sh.red);
+        if (threadIdx.x == 0) lw.pcount[grp] = (int32_t)m;
+    } else {
+        const int64_t m = compact_kept(kept, lw.cand + grp * capv, n, sel.leaf_idx + grp * g.cap[1],
+                                       sel.head_mask + grp * g.cap[1], sh.red);
+        if (threadIdx.x == 0) sel.count[grp] = (int32_t)m;
+    }
+    if (threadIdx.x == 0) lw.done[grp] = 0u;
 }
 
 __global__ void __launch_bounds__(kSelThreads)
@@ -461,57 +692,18 @@ select_sets_kernel(const float *scores, const int32_t *counts, int64_t stride, f
     for (int64_t i = threadIdx.x; i < n; i += blockDim.x) kp[i] = 0;
     __syncthreads();
     topp_core(
-        sh, n, p, 0u, [&](int64_t) { return true; }, [&](int64_t i) { return sc[i]; },
-        [&](int64_t i) { kp[i] = 1; });
-}
-
-// --------------------------------------------------------------------- expand
-
-constexpr int kExpThreads = 1024;
-
-__global__ void __launch_bounds__(kExpThreads)
-expand_kernel(Geo g, LevelWs cur, LevelWs nxt, int level, const int32_t *lens,
-              zha_selection sel) {
-    __shared__ int64_t red[kExpThreads / 32];
-    const int grp = blockIdx.x;
-    const int b = grp / g.Hkv;
-    int64_t N = lens[b];
-    if (N < 0 || N > g.max_len) N = 0;
-    const int64_t cap = g.cap[level];
-    const int64_t n = cur.count[grp];
-    const int64_t n_below = level > 1 ? level_nodes(N, g.c, level - 1) : 0;
-    const int64_t cap_next = level > 1 ? g.cap[level - 1] : g.cap[1];
-    int64_t run = 0;
-    for (int64_t base = 0; base < n; base += blockDim.x) {
-        const int64_t i = base + threadIdx.x;
-        uint32_t km = 0u;
-        int64_t node = 0;
-        if (i < n) {
-            km = cur.kept[grp * cap + i];
-            node = cur.cand[grp * cap + i];
-        }
-        int64_t nch = 0;
-        if (km) nch = level > 1 ? min64(g.c, n_below - node * g.c) : 1;
-        int64_t tot;
-        const int64_t off = run + block_exclusive_scan<int64_t>(nch, red, &tot);
-        if (level > 1) {
-            for (int64_t j = 0; j < nch; ++j) {
-                nxt.cand[grp * cap_next + off + j] = (int32_t)(node * g.c + j);
-                nxt.cmask[grp * cap_next + off + j] = km;
-                nxt.kept[grp * cap_next + off + j] = 0u;
+        sh, n, p, 0u, 0xffffffffu,
+        [&](int64_t i0, float (&e)[8]) {
+            uint32_t mb = 0u;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const bool in = i0 + v < n;
+                e[v] = in ? sc[i0 + v] : 0.f;
+                mb |= in ? (1u << v) : 0u;
             }
-        } else if (nch) {
-            sel.leaf_idx[grp * cap_next + off] = (int32_t)node;
-            sel.head_mask[grp * cap_next + off] = km;
-        }
-        run += tot;
-    }
-    if (threadIdx.x == 0) {
-        if (level > 1)
-            nxt.count[grp] = (int32_t)run;
-        else
-            sel.count[grp] = (int32_t)run;
-    }
+            return mb;
+        },
+        [&](int64_t i) { kp[i] = 1; });
 }
 
 }  // namespace
@@ -519,72 +711,68 @@ expand_kernel(Geo g, LevelWs cur, LevelWs nxt, int level, const int32_t *lens,
 cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const int32_t *lens,
                          const float *p_levels, const zha_selection &sel, void *ws,
                          int32_t *status, cudaStream_t st) {
-    uint32_t *maxkey = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + g.ws_maxkey);
-    const int groups = g.groups();
     static const char *score_names[] = {"", "score[l1]", "score[l2]", "score[l3]", "score[l4]",
                                         "score[l5]", "score[l6]", "score[l7]", "score[l8]"};
     static const char *select_names[] = {"", "select[l1]", "select[l2]", "select[l3]", "select[l4]",
                                          "select[l5]", "select[l6]", "select[l7]", "select[l8]"};
-    static const char *expand_names[] = {"", "expand[l1]", "expand[l2]", "expand[l3]", "expand[l4]",
-                                         "expand[l5]", "expand[l6]", "expand[l7]", "expand[l8]"};
+    const int groups = g.groups();
     {
         ProfScope ps("route_init", st);
-        route_init_kernel<<<groups, 256, 0, st>>>(g, level_ws(g, ws, g.L), lens, maxkey, status);
+        char *base = static_cast<char *>(ws);
+        route_init_kernel<<<groups, 64, 0, st>>>(
+            g, reinterpret_cast<uint32_t *>(base + g.ws_maxkey),
+            reinterpret_cast<uint32_t *>(base + g.ws_minkey),
+            reinterpret_cast<uint32_t *>(base + g.ws_done), lens, status);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    const char *tb = static_cast<const char *>(tree);
     for (int level = g.L; level >= 1; --level) {
         LevelWs lw = level_ws(g, ws, level);
-        uint32_t *mk = maxkey + (int64_t)(level - 1) * groups * g.G;
-        const char *tb = static_cast<const char *>(tree);
-        const int64_t cap = g.cap[level];
-        if (g.dtype == ZHA_BF16) {
+        LevelWs up = level < g.L ? level_ws(g, ws, level + 1) : lw;
+        const int64_t capv = g.capv[level];
+        {
             ProfScope ps(score_names[level], st);
-            const auto *mu = reinterpret_cast<const __nv_bfloat16 *>(tb + g.mu_off[level]);
-            const auto *bias = reinterpret_cast<const float *>(tb + g.bias_off[level]);
-            const auto *qq = static_cast<const __nv_bfloat16 *>(q);
-            const int64_t want = (cap + kScoreWarps - 1) / kScoreWarps;
-            const int per_group = (int)max64(1, min64(want, (148 * 8 + groups - 1) / groups));
-            dim3 grid(per_group, groups);
-            const int mt = g.R > 16 ? 2 : 1, nt = g.G > 8 ? 2 : 1;
-#define ZHA_SCORE(D, MT, NT) score_mma_kernel<D, MT, NT><<<grid, kScoreWarps * 32, 0, st>>>(g, mu, bias, qq, lw, level, mk)
-            if (g.d == 128) {
-                if (mt == 1 && nt == 1) ZHA_SCORE(128, 1, 1);
-                else if (mt == 1) ZHA_SCORE(128, 1, 2);
-                else if (nt == 1) ZHA_SCORE(128, 2, 1);
-                else ZHA_SCORE(128, 2, 2);
-            } else {
-                if (mt == 1 && nt == 1) ZHA_SCORE(64, 1, 1);
-                else if (mt == 1) ZHA_SCORE(64, 1, 2);
-                else if (nt == 1) ZHA_SCORE(64, 2, 1);
-                else ZHA_SCORE(64, 2, 2);
-            }
+            if (g.dtype == ZHA_BF16) {
+                const auto *mu = reinterpret_cast<const __nv_bfloat16 *>(tb + g.mu_off[level]);
+                const auto *bias = reinterpret_cast<const float *>(tb + g.bias_off[level]);
+                const auto *qq = static_cast<const __nv_bfloat16 *>(q);
+                const int64_t want = (capv + kScoreWarps - 1) / kScoreWarps;
+                const int per_group = (int)max64(1, min64(want, (148 * 8 + groups - 1) / groups));
+                dim3 grid(per_group, groups);
+                const int mt = g.R > 16 ? 2 : 1, nt = g.G > 8 ? 2 : 1;
+#define ZHA_SCORE(D, MT, NT) \
+    score_mma_kernel<D, MT, NT><<<grid, kScoreWarps * 32, 0, st>>>(g, mu, bias, qq, lens, lw, up, level)
+                if (g.d == 128) {
+                    if (mt == 1 && nt == 1) ZHA_SCORE(128, 1, 1);
+                    else if (mt == 1) ZHA_SCORE(128, 1, 2);
+                    else if (nt == 1) ZHA_SCORE(128, 2, 1);
+                    else ZHA_SCORE(128, 2, 2);
+                } else {
+                    if (mt == 1 && nt == 1) ZHA_SCORE(64, 1, 1);
+                    else if (mt == 1) ZHA_SCORE(64, 1, 2);
+                    else if (nt == 1) ZHA_SCORE(64, 2, 1);
+                    else ZHA_SCORE(64, 2, 2);
+                }
 #undef ZHA_SCORE
-        } else {
-            ProfScope ps(score_names[level], st);
-            const auto *mu = reinterpret_cast<const float *>(tb + g.mu_off[level]);
-            const auto *bias = reinterpret_cast<const float *>(tb + g.bias_off[level]);
-            const auto *qq = static_cast<const float *>(q);
-            const int per_group = (int)max64(1, min64(cap, (148 * 8 + groups - 1) / groups));
-            dim3 grid(per_group, groups);
-            if (g.d == 128)
-                score_f32_kernel<128><<<grid, 128, 0, st>>>(g, mu, bias, qq, lw, level, mk);
-            else
-                score_f32_kernel<64><<<grid, 128, 0, st>>>(g, mu, bias, qq, lw, level, mk);
+            } else {
+                const auto *mu = reinterpret_cast<const float *>(tb + g.mu_off[level]);
+                const auto *bias = reinterpret_cast<const float *>(tb + g.bias_off[level]);
+                const auto *qq = static_cast<const float *>(q);
+                const int per_group = (int)max64(1, min64(capv, (148 * 8 + groups - 1) / groups));
+                dim3 grid(per_group, groups);
+                if (g.d == 128)
+                    score_f32_kernel<128><<<grid, 128, 0, st>>>(g, mu, bias, qq, lens, lw, up, level);
+                else
+                    score_f32_kernel<64><<<grid, 128, 0, st>>>(g, mu, bias, qq, lens, lw, up, level);
+            }
         }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         {
             ProfScope ps(select_names[level], st);
             select_kernel<<<dim3(g.G, groups), kSelThreads, 0, st>>>(g, lw, level, p_levels[level - 1],
-                                                                     mk, sel.level_kept);
-        }
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-        LevelWs nx = level > 1 ? level_ws(g, ws, level - 1) : lw;
-        {
-            ProfScope ps(expand_names[level], st);
-            expand_kernel<<<groups, kExpThreads, 0, st>>>(g, lw, nx, level, lens, sel);
+                                                                     sel.level_kept, sel);
         }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
