@@ -152,22 +152,36 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def _all_reduce(x: float, world: int, op) -> float:
     import torch
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    import torch
+    return _all_reduce(x, world, torch.distributed.ReduceOp.MAX)
 
 
 def sum_over_ranks(x: float, world: int) -> float:
     import torch
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t)
-    return float(t.item())
+    return _all_reduce(x, world, torch.distributed.ReduceOp.SUM)
+
+
+def job_throughput(tokens_local: float, ms_local: float, world: int):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    ms = max_over_ranks(ms_local, world)
+    return sum_over_ranks(tokens_local, world) / (ms / 1e3), ms
+
+
+def replica(w, rank: int):
+    """The workload a rank decodes: the same shapes, its own seed."""
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank) if rank else w
 
 
 # --------------------------------------------------------------- CPU oracle
@@ -246,8 +260,7 @@ def zha_arm(args, w, world, rank, local):
     from tree_indexed_sparse_02_b200.inputs import decode_stream, make_inputs
 
     K_steps, W_steps = args.steps, args.warmup
-    if world > 1:
-        w = dataclasses.replace(w, seed=w.seed + 1000 * rank)   # independent replica per rank
+    w = replica(w, rank)   # independent replica per rank
     n_total = W_steps + 2 * K_steps + (K_steps if not args.no_e2e else 0)
     cap = w.context + n_total + 8
     inp = make_inputs(w, device="cuda", capacity=cap)
@@ -310,10 +323,8 @@ def zha_arm(args, w, world, rank, local):
     buf.check_status("timed steps")
     clocks = clk.summary()
 
-    total_ms = max_over_ranks(sum(times_a), world)
+    value, total_ms = job_throughput(float(w.batch * K_steps), sum(times_a), world)
     ms_per_step = total_ms / K_steps
-    tokens = sum_over_ranks(float(w.batch * K_steps), world)
-    value = tokens / (total_ms / 1e3)
 
     # bytes the step must move (algorithmic), from the routed counts of each step
     es = 2 if w.dtype == "bf16" else 4
@@ -418,8 +429,8 @@ def zha_arm(args, w, world, rank, local):
             ev[j][1].record(stream)
         torch.cuda.synchronize()
         buf.check_status("e2e steps")
-        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
-        res["e2e"] = {"value": sum_over_ranks(float(w.batch * K_steps), world) / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e_value, _ = job_throughput(float(w.batch * K_steps), sum(a.elapsed_time(b) for a, b in ev), world)
+        res["e2e"] = {"value": e2e_value, "unit": "tokens/s",
                       "h2d_bytes_per_step": (qd.numel() + kd.numel() + vd.numel()) * qd.element_size(),
                       "d2h_bytes_per_step": out.numel() * out.element_size()}
 
