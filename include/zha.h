@@ -223,6 +223,28 @@ ZHA_API zha_status zha_dense_decode(const zha_config *cfg, const void *q, const 
                             void *stream);
 
 /*
+ * zha_dense_decode_noalloc -- zha_dense_decode for callers that cannot
+ * allocate device memory (no counterpart on the method's pages). Some callers
+ * cannot call cudaMalloc or hand over a workspace: code embedded in a host
+ * framework that owns every device allocation through its own arena, or a
+ * latency-critical loop that must not pay for cudaMalloc, which can
+ * synchronise the device. This entry point takes the same inputs and output
+ * as zha_dense_decode and no workspace: its split-K scratch is a fixed 4 MiB
+ * array compiled into the library, which every device that loads the library
+ * keeps reserved until the process exits. Configurations whose split-K
+ * partials (batch * n_kv_heads * splits * G * (head_dim + 2) floats, each
+ * part rounded up to 256 bytes) exceed 4 MiB return ZHA_ERR_CAPACITY.
+ * All calls share the array, so calls whose kernels overlap on the GPU (for
+ * example on two streams at once) race and must be serialised by the caller.
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture. It allocates nothing, in the library or in any library it calls.
+ */
+ZHA_API zha_status zha_dense_decode_noalloc(const zha_config *cfg, const void *q, const void *K,
+                                            const void *V, const int32_t *lens, void *out,
+                                            int32_t *dev_status, void *stream);
+
+/*
  * zha_topp_select -- one level of the routing selection on given scores,
  * for n_sets independent candidate sets (section "How does top-p routing pick
  * tokens"): set i has counts[i] candidates whose fp32 scores are

@@ -112,6 +112,11 @@ zha_status check_sel(const zha_selection *sel) {
 
 }  // namespace
 
+namespace zha {
+// The geometry of a configuration, for entry points defined in other files.
+Geo make_geo_for(const zha_config *c) { return make_geo(c); }
+}  // namespace zha
+
 extern "C" {
 
 const char *zha_status_string(zha_status s) {

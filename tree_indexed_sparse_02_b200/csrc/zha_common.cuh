@@ -172,6 +172,7 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
                              int32_t *status, cudaStream_t st);
 cudaError_t launch_decode_write(const Geo &g, void *K, void *V, int32_t *lens, const void *k_new,
                                 const void *v_new, int32_t *status, cudaStream_t st);
+Geo make_geo_for(const zha_config *c);
 cudaError_t launch_topp_select(const float *scores, const int32_t *counts, int n_sets,
                                int64_t stride, float p, uint8_t *kept, int32_t *status,
                                cudaStream_t st);
