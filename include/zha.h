@@ -6,17 +6,19 @@
  *
  * Method (page "Zyphra AI Introduces Zyphra Hierarchical Attention (ZHA)",
  * MarkTechPost article):
- *   - section "Building the tree": keys are cut into contiguous chunks of c;
- *     each chunk is summarised against R learned reference queries as tangent
- *     planes of the chunk's log attention mass; summaries are grouped and
- *     summarised again, level by level; a node's estimate is the max over its
- *     planes.
- *   - section "How does top-p routing pick tokens": a decode query scores the
- *     top-level nodes, keeps the smallest set that holds a fraction p of the
- *     estimated mass, expands only their children, and repeats down to the
- *     raw KV; token 0 is always kept as the attention sink.
- *   - explainer widget, step 5: exact attention over the selected raw KV, the
- *     sink and the current chunk; the full KV cache stays stored.
+ *   - section "Building the tree": the cache is cut into contiguous chunks of c
+ *     keys; R learned reference queries each give a chunk a tangent plane of
+ *     its log attention mass; c sibling summaries are in turn summarised into
+ *     a parent, one level at a time; the largest plane value is the node's
+ *     estimate.
+ *   - section "How does top-p routing pick tokens": a decode query rates the
+ *     nodes of the top level, retains the fewest whose estimated mass adds up
+ *     to at least p of the total, rates only the children of those, and goes
+ *     on down to the raw KV; token 0 (the attention sink) is attended in
+ *     every case.
+ *   - explainer widget, step 5: the final attention is exact, over the raw KV
+ *     that routing picked plus the sink and the chunk being written; the
+ *     whole cache is kept.
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller. The library

@@ -10,21 +10,20 @@
  * What each function follows (page title, then section):
  *   "Zyphra AI Introduces Zyphra Hierarchical Attention (ZHA)" (MarkTechPost
  *   article, tradepoint.io copy):
- *     - "Building the tree": keys are cut into contiguous chunks of c; every
- *       chunk is compressed to summaries; summaries are grouped and compressed
- *       again, level by level (c = 4 with 6 levels gives 4,096 tokens per top
- *       node). Each learned reference query gives a tangent-plane estimate of
- *       a chunk's log attention mass; the max over the planes is the node's
- *       estimate.
- *     - "How does top-p routing pick tokens": a query scores the top-level
- *       nodes, keeps the smallest set holding a fraction p of the estimated
- *       mass, expands only the kept nodes' children, and repeats down to the
- *       raw KV entries; the first token is always kept (attention sink).
- *     - explainer widget, step 5 caption: exact attention runs over the
- *       selected raw KV entries plus the sink and the current chunk.
- *   "ZHA" (kongchang.com notes): upper-level nodes are compressed
- *       representations of their children; tree depth grows as the cache
- *       grows.
+ *     - "Building the tree": the cache is cut into contiguous chunks of c
+ *       keys and each chunk is summarised; c sibling summaries are summarised
+ *       into a parent, one level at a time (c = 4 and 6 levels put 4,096
+ *       tokens under a top node). Every learned reference query gives a chunk
+ *       a tangent plane of its log attention mass; the largest plane value is
+ *       the node's estimate.
+ *     - "How does top-p routing pick tokens": a decode query rates the top
+ *       level's nodes, retains the fewest whose estimated mass reaches p of
+ *       the total, rates only their children next, and so on down to raw
+ *       keys; token 0 (the attention sink) is attended in every case.
+ *     - explainer widget, step 5 caption: the final attention is exact, over
+ *       the routed raw KV plus the sink and the chunk being written.
+ *   "ZHA" (kongchang.com notes): a parent summarises its children, and the
+ *       tree grows as the cache does.
  *
  * Readings taken where the pages are loose (each is also listed in the
  * design notes of the repository):

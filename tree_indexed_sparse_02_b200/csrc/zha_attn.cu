@@ -2,9 +2,9 @@
 // comparison kernel), split-K flash decoding with a log-sum-exp merge.
 //
 // Page "Zyphra AI Introduces Zyphra Hierarchical Attention (ZHA)", explainer
-// widget step 5: exact attention over the selected raw KV entries plus the
-// first token (sink) and the current chunk; section "How does top-p routing
-// pick tokens": the first token is always kept.
+// widget step 5: the final attention is exact, over the routed raw KV plus
+// token 0 (the sink, section "How does top-p routing pick tokens") and the
+// chunk being written.
 //
 // Every (sequence, KV head) group streams the union of its heads' tokens
 // once; each token carries the bit mask of query heads that attend to it, so

@@ -1,11 +1,11 @@
 // zha_route.cu -- top-p routing down the summary tree.
 //
 // Page "Zyphra AI Introduces Zyphra Hierarchical Attention (ZHA)", section
-// "How does top-p routing pick tokens": a decode query scores the top-level
-// nodes, keeps the smallest set that holds a fraction p of the estimated
-// attention mass, expands only their children, and repeats down to the raw
-// KV entries. Section "Building the tree": a node's estimate is the max over
-// its reference planes, E = max_r (s q.mu_r + bias_r).
+// "How does top-p routing pick tokens": a decode query rates the top level's
+// nodes, retains the fewest whose estimated attention mass reaches p of the
+// total, rates only their children next, and so on down to raw keys. Section
+// "Building the tree": a node's estimate is its largest reference-plane
+// value, E = max_r (s q.mu_r + bias_r).
 //
 // Per level, for all (sequence, KV head) groups at once, two launches:
 //   score  -- candidate i of a group is child i % c of the (i / c)-th node

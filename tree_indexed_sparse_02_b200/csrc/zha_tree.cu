@@ -1,9 +1,9 @@
 // zha_tree.cu -- building and extending the summary tree.
 //
 // Page "Zyphra AI Introduces Zyphra Hierarchical Attention (ZHA)", section
-// "Building the tree": contiguous chunks of c keys are summarised against R
-// reference queries as tangent planes of the chunk's log attention mass, and
-// the summaries are grouped and summarised again level by level.
+// "Building the tree": each contiguous chunk of c keys gets, from each of R
+// reference queries, a tangent plane of its log attention mass; c sibling
+// summaries are then summarised into a parent, one level at a time.
 //
 // For reference r and points x_i with log-weights a_i (raw keys: a_i = 0;
 // children of a parent: x_i = mu_{i,r}, a_i = bias_{i,r}):
