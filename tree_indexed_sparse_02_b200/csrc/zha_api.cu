@@ -65,6 +65,7 @@ Geo make_geo(const zha_config *c) {
         g.ws_cmask[l] = off;  off = align256(off + n * 4);
         g.ws_kept[l] = off;   off = align256(off + n * 4);
         g.ws_scores[l] = off; off = align256(off + n * g.G * 4);
+        g.ws_keptbits[l] = off; off = align256(off + n * g.G / 8);
         g.ws_count[l] = off;  off = align256(off + groups * 4);
         const size_t k = groups * g.cap[l];
         g.ws_plist[l] = off;  off = align256(off + k * 4);

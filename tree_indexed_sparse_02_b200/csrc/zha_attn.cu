@@ -41,6 +41,29 @@ struct TokenPlan {
     const int32_t *leaf;
     const uint32_t *hmask;
 
+    // Split form of at(): fetch() issues the selection loads, finish() uses them.
+    __device__ __forceinline__ void fetch(int v, int &lf, uint32_t &hm) const {
+        if (v < sel_tokens) {
+            lf = __ldg(&leaf[v >> lc]);
+            hm = __ldg(&hmask[v >> lc]);
+        }
+    }
+    __device__ __forceinline__ void finish(int v, int lf, uint32_t hm, int &pos, uint32_t &mask,
+                                           int32_t *status) const {
+        if (v < sel_tokens) {
+            if ((unsigned)lf >= (unsigned)n1) {
+                set_status(status, ZHA_ERR_INVALID_ARG);
+                pos = 0;
+                mask = 0u;
+                return;
+            }
+            pos = (lf << lc) | (v & ((1 << lc) - 1));
+            mask = hm | ((pos == 0 || pos >= cur_start) ? all : 0u);
+            return;
+        }
+        at(v, pos, mask, status);
+    }
+
     __device__ __forceinline__ void at(int v, int &pos, uint32_t &mask, int32_t *status) const {
         if (v < sel_tokens) {
             const int e = v >> lc;
@@ -261,8 +284,13 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
             if (nt < t_hi) issue(nt, (it + kStages - 1) % kStages, (it + kStages - 1) % kSlots);
             cp_async_commit();
         }
-        // look up the tile after that now; its slot was last read by tile it - 1
-        if (t_lo + it + kStages < t_hi) resolve(t_lo + it + kStages, (it + kStages) % kSlots);
+        // look up the tile after that: loads now, results stored after this
+        // tile's compute (its slot was last read by tile it - 1)
+        const int rt = t_lo + it + kStages;
+        const bool look = threadIdx.x < kTile && rt < t_hi;
+        int f_leaf = 0;
+        uint32_t f_hm = 0u;
+        if (look) tp.fetch(rt * kTile + threadIdx.x, f_leaf, f_hm);
         const int stage = it % kStages;
         const uint32_t kb = sbase + stage * STAGE_B, vb = kb + TILE_B;
         const int row0 = warp * 16;
@@ -326,6 +354,14 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
             ldsm_x4_t(vb + row * ROWB + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
             mma16816(o[2 * jp], pa0, pa1, pa2, pa3, b0, b1);
             mma16816(o[2 * jp + 1], pa0, pa1, pa2, pa3, b2, b3);
+        }
+        if (look) {
+            const int v = rt * kTile + threadIdx.x;
+            int pos;
+            uint32_t m;
+            tp.finish(v, f_leaf, f_hm, pos, m, status);
+            spos[(it + kStages) % kSlots][threadIdx.x] = pos;
+            smask[(it + kStages) % kSlots][threadIdx.x] = v < tp.nv ? m : 0u;
         }
     }
     cp_async_wait<0>();

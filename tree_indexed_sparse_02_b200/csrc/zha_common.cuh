@@ -36,6 +36,7 @@ struct Geo {
     size_t ws_cand[kMaxLevels + 1], ws_cmask[kMaxLevels + 1], ws_scores[kMaxLevels + 1],
         ws_kept[kMaxLevels + 1], ws_count[kMaxLevels + 1];     // candidates of a level
     size_t ws_plist[kMaxLevels + 1], ws_pmask[kMaxLevels + 1], ws_pcount[kMaxLevels + 1];  // kept
+    size_t ws_keptbits[kMaxLevels + 1];  // [B*Hkv][G][capv/8] bytes: each head's kept bitmap
     size_t ws_maxkey, ws_minkey;        // [L][B*Hkv][G] u32 ordered keys of the scores
     size_t ws_done;                     // [L][B*Hkv] u32 finished select CTAs
     size_t ws_part_ml, ws_part_o;       // split-K partials

@@ -18,10 +18,11 @@
 //             a radix select over the score's distance below the max (the
 //             range is known, so 12-bit digits are spread over buckets that
 //             are actually used) with masses summed in 2^-31 fixed point
-//             (exact and order-independent); kept bits are OR-ed per
-//             candidate, and the last CTA of a group to finish compacts the
-//             candidates some head kept into the next level's parent list
-//             (or, at level 1, into the selection).
+//             (exact and order-independent); each head writes a kept bitmap,
+//             and the last CTA of a group to finish joins the G bitmaps into
+//             per-candidate head masks and compacts the candidates some head
+//             kept into the next level's parent list (or, at level 1, into
+//             the selection).
 #include "zha_common.cuh"
 
 namespace zha {
@@ -189,7 +190,6 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
                 if (lane == 0) {
                     lw.cand[grp * capv + i] = node[u];
                     lw.cmask[grp * capv + i] = hm[u];
-                    lw.kept[grp * capv + i] = 0u;
                 }
             }
         }
@@ -312,7 +312,6 @@ __global__ void score_f32_kernel(Geo g, const float *mu, const float *bias, cons
         if (threadIdx.x == 0) {
             lw.cand[grp * capv + i] = (int32_t)node;
             lw.cmask[grp * capv + i] = hm;
-            lw.kept[grp * capv + i] = 0u;
         }
         if (hm == 0u) {
             if (threadIdx.x < g.G) lw.scores[(grp * g.G + threadIdx.x) * capv + i] = -INFINITY;
@@ -347,7 +346,7 @@ __global__ void score_f32_kernel(Geo g, const float *mu, const float *bias, cons
 
 // --------------------------------------------------------------------- select
 
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = 1024;
 constexpr int kDigitBits = 12;
 constexpr int kBuckets = 1 << kDigitBits;
 constexpr int kMaxTies = 1024;
@@ -416,18 +415,23 @@ struct SelShared {
     int last;
 };
 
-// Exact top-p over the members of one candidate set, read 8 consecutive
-// candidates at a time:
-//   load8(i0, e) -- fills e[0..8) with the scores of candidates i0..i0+7 and
-//                   returns a bit mask of those that are members (and < n)
-//   emit(i)      -- called once for every kept candidate
+// Exact top-p over the members of one candidate set, visited in blocks of 8
+// consecutive candidates (two blocks in flight per thread):
+//   load8(blk, e)    -- fills e[0..8) with the scores of candidates 8 blk ..
+//                       8 blk + 7 and returns the bit mask of those that are
+//                       members (and < n)
+//   store8(blk, m)   -- records the kept bits m of block blk (called once for
+//                       every block)
+//   add_kept(i)      -- marks one more candidate kept (thread 0 only, after
+//                       every store8)
 // kmax_in / kmin_in: ordered keys of the members' max / min score (kmax_in = 0:
 // unknown, found here). Returns (in every thread) the number kept.
-template <class Load8, class Emit>
+template <class Load8, class Store8, class AddKept>
 __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, uint32_t kmin_in,
-                         Load8 load8, Emit emit) {
+                         Load8 load8, Store8 store8, AddKept add_kept) {
     const int tid = threadIdx.x;
     const int64_t nblk = (n + 7) >> 3;
+    const int64_t step = blockDim.x;
     if (tid == 0) {
         sh.kmax = kmax_in;
         sh.kmin = kmax_in ? kmin_in : 0xffffffffu;
@@ -435,9 +439,9 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
     __syncthreads();
     if (kmax_in == 0u) {
         uint32_t mx = 0u, mn = 0xffffffffu;
-        for (int64_t blk = tid; blk < nblk; blk += blockDim.x) {
+        for (int64_t blk = tid; blk < nblk; blk += step) {
             float e[8];
-            const uint32_t mb = load8(blk << 3, e);
+            const uint32_t mb = load8(blk, e);
 #pragma unroll
             for (int v = 0; v < 8; ++v)
                 if ((mb >> v) & 1u) {
@@ -453,18 +457,13 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
         __syncthreads();
     }
     const uint32_t kmax = sh.kmax, kmin = sh.kmin;
-    if (kmax == 0u) return 0;  // no member (uniform)
     int kept = 0;
-    if (p >= 1.f) {
-        for (int64_t blk = tid; blk < nblk; blk += blockDim.x) {
+    if (kmax == 0u || p >= 1.f) {  // no member, or keep every member (uniform)
+        for (int64_t blk = tid; blk < nblk; blk += step) {
             float e[8];
-            const uint32_t mb = load8(blk << 3, e);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-                if ((mb >> v) & 1u) {
-                    emit((blk << 3) + v);
-                    ++kept;
-                }
+            const uint32_t mb = kmax ? load8(blk, e) : 0u;
+            store8(blk, mb);
+            kept += __popc(mb);
         }
         return (int)block_sum<unsigned long long>((unsigned long long)kept, sh.red);
     }
@@ -480,9 +479,7 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
         const int shift = hi - bits;
         for (int i = tid; i < kBuckets; i += blockDim.x) sh.hist_lo[i] = sh.hist_hi[i] = 0u;
         __syncthreads();
-        for (int64_t blk = tid; blk < nblk; blk += blockDim.x) {
-            float e[8];
-            const uint32_t mb = load8(blk << 3, e);
+        auto add_block = [&](uint32_t mb, const float (&e)[8]) {
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
                 if (!((mb >> v) & 1u)) continue;
@@ -491,6 +488,13 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
                 hist_add(sh.hist_lo, sh.hist_hi, (int)((u >> shift) & ((1u << bits) - 1u)),
                          fixed_mass(e[v], m));
             }
+        };
+        for (int64_t blk = tid; blk < nblk; blk += 2 * step) {
+            float e0[8], e1[8];
+            const uint32_t m0 = load8(blk, e0);
+            const uint32_t m1 = blk + step < nblk ? load8(blk + step, e1) : 0u;
+            add_block(m0, e0);
+            add_block(m1, e1);
         }
         __syncthreads();
         if (first) {
@@ -531,22 +535,24 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
     const unsigned long long above = sh.above, target = sh.target;
     if (tid == 0) sh.ntie = 0;
     __syncthreads();
-    // smaller u kept; ties at tau resolved in index order
-    for (int64_t blk = tid; blk < nblk; blk += blockDim.x) {
+    // smaller u kept; ties at tau resolved in index order below
+    for (int64_t blk = tid; blk < nblk; blk += step) {
         float e[8];
-        const uint32_t mb = load8(blk << 3, e);
+        const uint32_t mb = load8(blk, e);
+        uint32_t kb = 0u;
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
             if (!((mb >> v) & 1u)) continue;
             const uint32_t u = kmax - ordered_key(e[v]);
             if (u < tau) {
-                emit((blk << 3) + v);
-                ++kept;
+                kb |= 1u << v;
             } else if (u == tau) {
                 const int slot = atomicAdd(&sh.ntie, 1);
                 if (slot < kMaxTies) sh.ties[slot] = (int32_t)((blk << 3) + v);
             }
         }
+        store8(blk, kb);
+        kept += __popc(kb);
     }
     __syncthreads();
     const int ntie = sh.ntie;
@@ -563,8 +569,8 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
             for (int j = 0; j < ntie && cum < target; ++j) {
                 const int32_t i = sh.sorted_ties[j];
                 float e[8];
-                load8((int64_t)i & ~int64_t(7), e);
-                emit(i);
+                load8((int64_t)i >> 3, e);
+                add_kept(i);
                 ++kept;
                 cum += fixed_mass(e[i & 7], m);
             }
@@ -574,10 +580,10 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
         unsigned long long cum = above;
         for (int64_t blk = 0; blk < nblk && cum < target; ++blk) {
             float e[8];
-            const uint32_t mb = load8(blk << 3, e);
+            const uint32_t mb = load8(blk, e);
             for (int v = 0; v < 8 && cum < target; ++v) {
                 if (!((mb >> v) & 1u) || kmax - ordered_key(e[v]) != tau) continue;
-                emit((blk << 3) + v);
+                add_kept((blk << 3) + v);
                 ++kept;
                 cum += fixed_mass(e[v], m);
             }
@@ -586,61 +592,71 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
     return (int)block_sum<unsigned long long>((unsigned long long)kept, sh.red);
 }
 
-// Compacts the candidates with a non-zero kept mask, in order, into
-// (out_idx, out_mask); returns the number written (every thread). The kept
-// rows are padded to a multiple of 8 entries.
-__device__ int64_t compact_kept(const uint32_t *kept, const int32_t *cand, int64_t n,
-                                int32_t *out_idx, uint32_t *out_mask, unsigned long long *red) {
-    constexpr int V = 8;
+// Joins the G heads' kept bitmaps of a group (bits[h][blk], byte per 8
+// candidates) into per-candidate head masks (written to kept[]) and compacts
+// the candidates some head kept, in order, into (out_idx, out_mask). Returns
+// the number written (every thread). Rows are padded to 8 entries.
+__device__ int64_t join_and_compact(const uint8_t *bits, int64_t bits_stride, int G,
+                                    uint32_t *kept, const int32_t *cand, int64_t n,
+                                    int32_t *out_idx, uint32_t *out_mask, unsigned long long *red) {
+    const int64_t nblk = (n + 7) >> 3;
     int64_t run = 0;
-    for (int64_t base = 0; base < n; base += (int64_t)blockDim.x * V) {
-        const int64_t i0 = base + (int64_t)threadIdx.x * V;
-        uint32_t km[V];
+    for (int64_t base = 0; base < nblk; base += blockDim.x) {
+        const int64_t blk = base + threadIdx.x;
+        uint32_t km[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) km[v] = 0u;
+        if (blk < nblk) {
+            for (int h = 0; h < G; ++h) {
+                const uint32_t b = __ldcg(bits + h * bits_stride + blk);
+#pragma unroll
+                for (int v = 0; v < 8; ++v) km[v] |= ((b >> v) & 1u) << h;
+            }
+            uint4 *kp = reinterpret_cast<uint4 *>(kept + (blk << 3));
+            kp[0] = make_uint4(km[0], km[1], km[2], km[3]);
+            kp[1] = make_uint4(km[4], km[5], km[6], km[7]);
+        }
         int cnt = 0;
-        if (i0 < n) {
-            const uint4 a = __ldcg(reinterpret_cast<const uint4 *>(kept + i0));
-            const uint4 b = __ldcg(reinterpret_cast<const uint4 *>(kept + i0) + 1);
-            km[0] = a.x; km[1] = a.y; km[2] = a.z; km[3] = a.w;
-            km[4] = b.x; km[5] = b.y; km[6] = b.z; km[7] = b.w;
-        } else {
 #pragma unroll
-            for (int v = 0; v < V; ++v) km[v] = 0u;
-        }
-#pragma unroll
-        for (int v = 0; v < V; ++v) {
-            if (i0 + v >= n) km[v] = 0u;
-            cnt += km[v] != 0u;
-        }
+        for (int v = 0; v < 8; ++v) cnt += km[v] != 0u;
         unsigned long long tot;
         int64_t o = run + (int64_t)block_exclusive_scan<unsigned long long>((unsigned long long)cnt, red, &tot);
+        if (cnt) {
+            const int4 c0 = *reinterpret_cast<const int4 *>(cand + (blk << 3));
+            const int4 c1 = *reinterpret_cast<const int4 *>(cand + (blk << 3) + 4);
+            const int32_t cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-        for (int v = 0; v < V; ++v)
-            if (km[v]) {
-                out_idx[o] = cand[i0 + v];
-                out_mask[o] = km[v];
-                ++o;
-            }
+            for (int v = 0; v < 8; ++v)
+                if (km[v]) {
+                    out_idx[o] = cv[v];
+                    out_mask[o] = km[v];
+                    ++o;
+                }
+        }
         run += (int64_t)tot;
     }
     return run;
 }
 
 __global__ void __launch_bounds__(kSelThreads)
-select_kernel(Geo g, LevelWs lw, int level, float p, int32_t *level_kept, zha_selection sel) {
+select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t *level_kept,
+              zha_selection sel) {
     __shared__ SelShared sh;
     const int h = blockIdx.x, grp = blockIdx.y;
     const int64_t capv = g.capv[level];
+    const int64_t bstride = capv >> 3;  // bytes of one head's bitmap
     const int64_t n = lw.count[grp];
     const uint32_t bit = 1u << h;
     const uint32_t *cmask = lw.cmask + grp * capv;
     const float *sc = lw.scores + (grp * g.G + h) * capv;
-    uint32_t *kept = lw.kept + grp * capv;
+    uint8_t *mybits = keptbits + ((int64_t)grp * g.G + h) * bstride;
     const uint32_t kmax = lw.maxkey[(int64_t)grp * g.G + h];
     const uint32_t kmin = lw.minkey[(int64_t)grp * g.G + h];
     // rows are padded to a multiple of 8 entries, so 8-wide loads stay in bounds
     const int nk = topp_core(
         sh, n, p, kmax, kmin,
-        [&](int64_t i0, float (&e)[8]) {
+        [&](int64_t blk, float (&e)[8]) {
+            const int64_t i0 = blk << 3;
             const float4 e0 = __ldg(reinterpret_cast<const float4 *>(sc + i0));
             const float4 e1 = __ldg(reinterpret_cast<const float4 *>(sc + i0) + 1);
             const uint4 m0 = __ldg(reinterpret_cast<const uint4 *>(cmask + i0));
@@ -653,25 +669,30 @@ select_kernel(Geo g, LevelWs lw, int level, float p, int32_t *level_kept, zha_se
             for (int v = 0; v < 8; ++v) mb |= ((mm[v] & bit) != 0u && i0 + v < n) ? (1u << v) : 0u;
             return mb;
         },
-        [&](int64_t i) { atomicOr(&kept[i], bit); });
+        [&](int64_t blk, uint32_t kb) { mybits[blk] = (uint8_t)kb; },
+        [&](int64_t i) { mybits[i >> 3] |= (uint8_t)(1u << (i & 7)); });
     if (level_kept && threadIdx.x == 0) {
         const int b = grp / g.Hkv, kvh = grp % g.Hkv;
         level_kept[((int64_t)b * g.Hq + kvh * g.G + h) * g.L + (level - 1)] = nk;
     }
-    // the last of the group's G CTAs compacts the union of the kept candidates
+    // the last of the group's G CTAs joins the heads' bitmaps and compacts
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) sh.last = atomicAdd(&lw.done[grp], 1u) == (uint32_t)(g.G - 1);
     __syncthreads();
     if (!sh.last) return;
     __threadfence();
+    const uint8_t *gbits = keptbits + (int64_t)grp * g.G * bstride;
+    uint32_t *kept = lw.kept + grp * capv;
     if (level > 1) {
-        const int64_t m = compact_kept(kept, lw.cand + grp * capv, n, lw.plist + grp * g.cap[level],
-                                       lw.pmask + grp * g.cap[level], sh.red);
+        const int64_t m = join_and_compact(gbits, bstride, g.G, kept, lw.cand + grp * capv, n,
+                                           lw.plist + grp * g.cap[level], lw.pmask + grp * g.cap[level],
+                                           sh.red);
         if (threadIdx.x == 0) lw.pcount[grp] = (int32_t)m;
     } else {
-        const int64_t m = compact_kept(kept, lw.cand + grp * capv, n, sel.leaf_idx + grp * g.cap[1],
-                                       sel.head_mask + grp * g.cap[1], sh.red);
+        const int64_t m = join_and_compact(gbits, bstride, g.G, kept, lw.cand + grp * capv, n,
+                                           sel.leaf_idx + grp * g.cap[1], sel.head_mask + grp * g.cap[1],
+                                           sh.red);
         if (threadIdx.x == 0) sel.count[grp] = (int32_t)m;
     }
     if (threadIdx.x == 0) lw.done[grp] = 0u;
@@ -689,19 +710,23 @@ select_sets_kernel(const float *scores, const int32_t *counts, int64_t stride, f
     }
     const float *sc = scores + set * stride;
     uint8_t *kp = kept + set * stride;
-    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) kp[i] = 0;
-    __syncthreads();
     topp_core(
         sh, n, p, 0u, 0xffffffffu,
-        [&](int64_t i0, float (&e)[8]) {
+        [&](int64_t blk, float (&e)[8]) {
             uint32_t mb = 0u;
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
-                const bool in = i0 + v < n;
-                e[v] = in ? sc[i0 + v] : 0.f;
+                const int64_t i = (blk << 3) + v;
+                const bool in = i < n;
+                e[v] = in ? sc[i] : 0.f;
                 mb |= in ? (1u << v) : 0u;
             }
             return mb;
+        },
+        [&](int64_t blk, uint32_t kb) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+                if ((blk << 3) + v < n) kp[(blk << 3) + v] = (uint8_t)((kb >> v) & 1u);
         },
         [&](int64_t i) { kp[i] = 1; });
 }
@@ -771,8 +796,9 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
         if (e != cudaSuccess) return e;
         {
             ProfScope ps(select_names[level], st);
-            select_kernel<<<dim3(g.G, groups), kSelThreads, 0, st>>>(g, lw, level, p_levels[level - 1],
-                                                                     sel.level_kept, sel);
+            uint8_t *keptbits = reinterpret_cast<uint8_t *>(static_cast<char *>(ws) + g.ws_keptbits[level]);
+            select_kernel<<<dim3(g.G, groups), kSelThreads, 0, st>>>(g, lw, keptbits, level,
+                                                                     p_levels[level - 1], sel.level_kept, sel);
         }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
