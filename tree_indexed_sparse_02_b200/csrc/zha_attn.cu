@@ -286,11 +286,13 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
         }
         // look up the tile after that: loads now, results stored after this
         // tile's compute (its slot was last read by tile it - 1)
+        // (16 lanes of every warp, one row each, so no warp lags at the barrier)
         const int rt = t_lo + it + kStages;
-        const bool look = threadIdx.x < kTile && rt < t_hi;
+        const int lrow = (threadIdx.x >> 5) * 16 + (threadIdx.x & 15);
+        const bool look = (threadIdx.x & 31) < 16 && rt < t_hi;
         int f_leaf = 0;
         uint32_t f_hm = 0u;
-        if (look) tp.fetch(rt * kTile + threadIdx.x, f_leaf, f_hm);
+        if (look) tp.fetch(rt * kTile + lrow, f_leaf, f_hm);
         const int stage = it % kStages;
         const uint32_t kb = sbase + stage * STAGE_B, vb = kb + TILE_B;
         const int row0 = warp * 16;
@@ -356,12 +358,12 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
             mma16816(o[2 * jp + 1], pa0, pa1, pa2, pa3, b2, b3);
         }
         if (look) {
-            const int v = rt * kTile + threadIdx.x;
+            const int v = rt * kTile + lrow;
             int pos;
             uint32_t m;
             tp.finish(v, f_leaf, f_hm, pos, m, status);
-            spos[(it + kStages) % kSlots][threadIdx.x] = pos;
-            smask[(it + kStages) % kSlots][threadIdx.x] = v < tp.nv ? m : 0u;
+            spos[(it + kStages) % kSlots][lrow] = pos;
+            smask[(it + kStages) % kSlots][lrow] = v < tp.nv ? m : 0u;
         }
     }
     cp_async_wait<0>();
