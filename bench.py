@@ -47,6 +47,11 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-profile", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="context sweep vs dense (deep and wide trees, random and aligned references)")
+    ap.add_argument("--sweep-n", default="8192,32768,65536,131072,524288,2097152,4194304")
+    ap.add_argument("--incremental", action="store_true",
+                    help="build the tree by 4,096-token appends, then decode at p = 0.9, 0.95, 0.99")
     return ap.parse_args()
 
 
@@ -468,12 +473,168 @@ def source_sha():
     return hsh.hexdigest()[:16]
 
 
+# ------------------------------------------------- extra modes (one GPU)
+
+
+def _timed_decode(zha, cfg, buf, K, V, refs, lens, qs, k_new, v_new, p, out, flush, first, n, warmup,
+                  w, with_counts=True):
+    """Decode steps first .. first+warmup+n; returns (ms of the n timed steps, mean
+    candidates scored, mean attended tokens) with an L2 flush before each timed step."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        zha.decode(cfg, buf.tree, K, V, refs, lens, qs[first + i], k_new[first + i], v_new[first + i], p,
+                   buf.sel, out, buf.workspace, buf.status)
+    counts = [buf.level_state(l)["count"].view(-1) for l in range(1, w.levels + 1)]
+    hist = torch.zeros((n, w.levels + 1, w.batch * w.n_kv_heads), dtype=torch.int32, device="cuda")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for j in range(n):
+        i = first + warmup + j
+        flush.fill_(float(j))
+        ev[j][0].record(stream)
+        zha.decode(cfg, buf.tree, K, V, refs, lens, qs[i], k_new[i], v_new[i], p, buf.sel, out,
+                   buf.workspace, buf.status)
+        ev[j][1].record(stream)
+        if with_counts:
+            for l in range(w.levels):
+                hist[j, l].copy_(counts[l], non_blocking=True)
+            hist[j, w.levels].copy_(buf.sel["count"].view(-1), non_blocking=True)
+    torch.cuda.synchronize()
+    buf.check_status("decode steps")
+    h = hist.double().cpu()
+    return (sum(a.elapsed_time(b) for a, b in ev), float(h[:, :w.levels].sum(dim=(1, 2)).mean()),
+            float(h[:, w.levels].sum(dim=1).mean()) * w.chunk + w.batch * w.n_kv_heads * (w.chunk + 1))
+
+
+def _timed_dense(zha, cfg, buf, q, K, V, lens, out, flush, n, warmup):
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        zha.dense_decode(cfg, q, K, V, lens, out, buf.workspace, buf.status)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for j in range(n):
+        flush.fill_(float(j))
+        ev[j][0].record(stream)
+        zha.dense_decode(cfg, q, K, V, lens, out, buf.workspace, buf.status)
+        ev[j][1].record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev) / n
+
+
+def _bytes(w, cand, tokens):
+    es = 2 if w.dtype == "bf16" else 4
+    cand_bytes = w.n_refs * w.head_dim * es + w.n_refs * 4 + 8 + w.group * 4
+    return cand * cand_bytes + tokens * 2 * w.head_dim * es + w.batch * w.n_kv_heads * 2 * w.group * w.head_dim * es
+
+
+def sweep_mode(args):
+    """Context sweep: ZHA decode vs the dense kernel on identical caches, deep and
+    wide trees, random and aligned references; one JSON line per point."""
+    import dataclasses
+
+    import torch
+
+    from tree_indexed_sparse_02_b200 import zha
+    from tree_indexed_sparse_02_b200.inputs import decode_stream, make_inputs, sweep_workload
+    peak, _ = read_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    Ns = [int(x) for x in args.sweep_n.split(",")]
+    for tree in ("deep", "wide"):
+        for refs_mode in ("random", "aligned"):
+            for N in Ns:
+                w = dataclasses.replace(sweep_workload(N, tree), refs_mode=refs_mode)
+                n, W = args.steps, args.warmup
+                cap = N + n + W + 8
+                inp = make_inputs(w, device="cuda", capacity=cap)
+                cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs,
+                                 w.dtype, cap)
+                buf = zha.Buffers(cfg)
+                zha.tree_build(cfg, buf.tree, inp.K, inp.refs, inp.lens, buf.status)
+                k_new, v_new, qs = decode_stream(w, n + W, device="cuda")
+                out = torch.empty_like(qs[0])
+                ms, cand, toks = _timed_decode(zha, cfg, buf, inp.K, inp.V, inp.refs, inp.lens, qs, k_new, v_new,
+                                               w.p, out, flush, 0, n, W, w)
+                dense_ms = _timed_dense(zha, cfg, buf, qs[0], inp.K, inp.V, inp.lens, out, flush, n, W)
+                us = ms / n * 1e3
+                touched = _bytes(w, cand, toks)
+                print(json.dumps({"mode": "sweep", "tree": tree, "refs": refs_mode, "context": N, "p": w.p,
+                                  "zha_us_per_step": us, "dense_us_per_step": dense_ms * 1e3,
+                                  "speedup_vs_dense": dense_ms * 1e3 / us,
+                                  "keys_attended": toks / (w.batch * w.n_kv_heads * (N + W + n)),
+                                  "touched_gbs": touched / (us / 1e6) / 1e9,
+                                  "touched_frac_of_hbm": touched / (us / 1e6) / 1e9 / peak,
+                                  "dense_frac_of_hbm": (w.batch * w.n_kv_heads * N * 2 * w.head_dim * 2) /
+                                  dense_ms * 1e3 / 1e9 / peak}), flush=True)
+                del inp, buf, k_new, v_new, qs, out
+                torch.cuda.empty_cache()
+
+
+def incremental_mode(args, w):
+    """The 1M deep-tree workload built by zha_tree_append in 4,096-token blocks
+    (append throughput), then decode steps at p = 0.9, 0.95 and 0.99."""
+    import dataclasses
+
+    import torch
+
+    from tree_indexed_sparse_02_b200 import zha
+    from tree_indexed_sparse_02_b200.inputs import decode_stream, make_inputs
+    peak, peak_kind = read_peaks()
+    ps = (0.9, 0.95, 0.99)
+    n, W = args.steps, args.warmup
+    N = w.context
+    cap = N + len(ps) * (n + W) + 8
+    inp = make_inputs(w, device="cuda", capacity=cap)
+    cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs, w.dtype, cap)
+    buf = zha.Buffers(cfg)
+    lens = torch.zeros_like(inp.lens)
+    block = 4096
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for start in range(0, N, block):
+        lens.fill_(min(start + block, N))
+        zha.tree_append(cfg, buf.tree, inp.K, inp.refs, lens, min(block, N - start), buf.status)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    buf.check_status("appends")
+    append_ms = e0.elapsed_time(e1)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    k_new, v_new, qs = decode_stream(w, len(ps) * (n + W), device="cuda")
+    out = torch.empty_like(qs[0])
+    per_p = {}
+    for k, p in enumerate(ps):
+        ms, cand, toks = _timed_decode(zha, cfg, buf, inp.K, inp.V, inp.refs, lens, qs, k_new, v_new, p, out,
+                                       flush, k * (n + W), n, W, w)
+        us = ms / n * 1e3
+        touched = _bytes(w, cand, toks)
+        per_p[str(p)] = {"tokens_per_s": w.batch / (us / 1e6), "us_per_step": us,
+                         "keys_attended": toks / (w.batch * w.n_kv_heads * int(lens[0])),
+                         "touched_bytes_per_step": touched, "touched_gbs": touched / (us / 1e6) / 1e9,
+                         "touched_frac_of_hbm": touched / (us / 1e6) / 1e9 / peak}
+    dense_ms = _timed_dense(zha, cfg, buf, qs[0], inp.K, inp.V, lens, out, flush, n, W)
+    main_p = per_p["0.95"]
+    res = {"metric": METRIC, "value": main_p["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1, "steps": n,
+           "warmup": W, "ms_per_step": main_p["us_per_step"] / 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": config_of(w),
+           "append": {"block_tokens": block, "tokens_per_s": N * w.batch / (append_ms / 1e3), "ms": append_ms},
+           "per_p": per_p, "dense": {"us_per_step": dense_ms * 1e3},
+           "speedup_vs_dense_p095": dense_ms * 1e3 / main_p["us_per_step"], "peak_kind": peak_kind}
+    print(json.dumps(res), flush=True)
+
+
 def main():
     args = parse()
     w = workload(args)
     world, rank, local = dist_setup(args)
     if args.impl == "reference":
         reference_arm(args, w, world, rank)
+        return
+    if args.sweep:
+        sweep_mode(args)
+        return
+    if args.incremental:
+        incremental_mode(args, w)
         return
     res = zha_arm(args, w, world, rank, local)
     if rank == 0:
