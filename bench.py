@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-profile", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
+                    help="replay each decode step from a captured CUDA graph (default on)")
     ap.add_argument("--sweep", action="store_true",
                     help="context sweep vs dense (deep and wide trees, random and aligned references)")
     ap.add_argument("--sweep-n", default="8192,32768,65536,131072,524288,2097152,4194304")
@@ -290,9 +292,15 @@ def zha_arm(args, w, world, rank, local):
     sel_count = buf.sel["count"].view(-1)
     step_i = 0
 
+    graph = zha.DecodeGraph(cfg, buf, K, V, refs, lens, p) if args.graph else None
+    use_graph = [graph is not None]
+
     def decode_step(i):
-        zha.decode(cfg, buf.tree, K, V, refs, lens, qs[i], k_new[i], v_new[i], p, buf.sel, out,
-                   buf.workspace, buf.status)
+        if use_graph[0]:
+            graph.step(qs[i], k_new[i], v_new[i])
+        else:
+            zha.decode(cfg, buf.tree, K, V, refs, lens, qs[i], k_new[i], v_new[i], p, buf.sel, out,
+                       buf.workspace, buf.status)
 
     # warm-up
     for _ in range(W_steps):
@@ -324,6 +332,8 @@ def zha_arm(args, w, world, rank, local):
     with Clocks(local, enabled=not args.no_clocks) as clk:
         times_a = timed_pass(K_steps, hist_a)
     launches = zha.launch_count() - launches0
+    if graph is not None:   # replays launch the captured kernels without going through the library
+        launches = graph.kernels_per_step * K_steps
     barrier(world)
     buf.check_status("timed steps")
     clocks = clk.summary()
@@ -356,11 +366,12 @@ def zha_arm(args, w, world, rank, local):
            "touched_frac_of_hbm": touched_mean / (ms_per_step / 1e3) / 1e9 / peak,
            "keys_attended": keys_share,
            "candidates_per_step": float(cand_per_step.mean()),
-           "gpu_launches": int(launches), "clocks": clocks}
+           "gpu_launches": int(launches), "cuda_graph": graph is not None, "clocks": clocks}
 
     # per-kernel CUDA-event timing: a second pass of K steps, every launch bracketed
     if not args.no_profile:
         hist_b = torch.zeros_like(hist_a)
+        use_graph[0] = False   # per-launch events need ordinary launches
         zha.profile_enable(True)
         times_b = timed_pass(K_steps, hist_b)
         zha.profile_enable(False)
@@ -426,11 +437,19 @@ def zha_arm(args, w, world, rank, local):
         for j in range(K_steps):
             flush.fill_(float(j))
             ev[j][0].record(stream)
-            qd.copy_(qh[j], non_blocking=True)
-            kd.copy_(kh[j], non_blocking=True)
-            vd.copy_(vh[j], non_blocking=True)
-            zha.decode(cfg, buf.tree, K, V, refs, lens, qd, kd, vd, p, buf.sel, out, buf.workspace, buf.status)
-            oh[j].copy_(out, non_blocking=True)
+            if graph is not None:   # host -> the graph's input buffers, replay, result -> host
+                graph.q.copy_(qh[j], non_blocking=True)
+                graph.k_new.copy_(kh[j], non_blocking=True)
+                graph.v_new.copy_(vh[j], non_blocking=True)
+                graph.graph.replay()
+                oh[j].copy_(graph.out, non_blocking=True)
+            else:
+                qd.copy_(qh[j], non_blocking=True)
+                kd.copy_(kh[j], non_blocking=True)
+                vd.copy_(vh[j], non_blocking=True)
+                zha.decode(cfg, buf.tree, K, V, refs, lens, qd, kd, vd, p, buf.sel, out, buf.workspace,
+                           buf.status)
+                oh[j].copy_(out, non_blocking=True)
             ev[j][1].record(stream)
         torch.cuda.synchronize()
         buf.check_status("e2e steps")
