@@ -39,19 +39,24 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="zha", choices=["zha", "reference"])
     ap.add_argument("--workload", default="deep256k",
-                    choices=["deep256k", "deep1m", "wide32k", "tiny", "small", "medium"])
+                    choices=["deep256k", "deep1m", "wide32k", "tiny", "small", "medium", "speed256k"])
     ap.add_argument("--refs", default="random", choices=["random", "aligned"])
     ap.add_argument("--p", type=float, default=None)
+    ap.add_argument("--p-schedule", default="fixed", choices=["fixed", "root"],
+                    help="per-level p: fixed p, or p^(1/L) at every level")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-profile", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--scorer", default="mma", choices=["tcgen05", "mma"],
+                    help="node-scoring kernel: tcgen05 (tensor memory) where it applies, or mma.sync")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="replay each decode step from a captured CUDA graph (default on)")
     ap.add_argument("--sweep", action="store_true",
                     help="context sweep vs dense (deep and wide trees, random and aligned references)")
     ap.add_argument("--sweep-n", default="8192,32768,65536,131072,524288,2097152,4194304")
+    ap.add_argument("--sweep-trees", default="deep,wide", help="comma list of deep, wide, speed")
     ap.add_argument("--incremental", action="store_true",
                     help="build the tree by 4,096-token appends, then decode at p = 0.9, 0.95, 0.99")
     return ap.parse_args()
@@ -62,12 +67,13 @@ def workload(args):
 
     from tree_indexed_sparse_02_b200 import inputs as I
     w = {"deep256k": I.DEEP_256K, "deep1m": I.DEEP_1M, "wide32k": I.WIDE_32K, "tiny": I.TINY_F32,
+         "speed256k": I.SPEED_256K,
          # a reduced deep-tree case (same kernels, B=1, N=64K) for detailed profiler captures
          "small": dataclasses.replace(I.DEEP_256K, name="deep N=65536 c=4 L=6 B=1", batch=1,
                                       context=65536, needles=64, diffuse_nodes=8),
          # one sequence of the 256K deep workload (a quarter of its bytes)
          "medium": dataclasses.replace(I.DEEP_256K, name="deep N=262144 c=4 L=6 B=1", batch=1)}[args.workload]
-    w = dataclasses.replace(w, refs_mode=args.refs)
+    w = dataclasses.replace(w, refs_mode=args.refs, p_schedule=args.p_schedule)
     if args.p is not None:
         w = dataclasses.replace(w, p=args.p)
     return w
@@ -218,7 +224,7 @@ def oracle_sample(w, inp, steps: int, warmup: int = 0):
     for i in range(warmup + steps):
         qi = q if i == 0 else rng.normal(size=q.shape)
         t0 = time.perf_counter()
-        orc.decode_group(tree, qi, K, V, w.p)
+        orc.decode_group(tree, qi, K, V, oracle_p(orc, w))
         if i >= warmup:
             times.append(time.perf_counter() - t0)
     groups = w.batch * w.n_kv_heads
@@ -248,10 +254,16 @@ def reference_arm(args, w, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def oracle_p(orc, w):
+    """Per-level p of the workload, by the oracle's own schedule rule."""
+    return w.p if w.p_schedule == "fixed" else orc.depth_root_schedule(w.p, w.levels)
+
+
 def config_of(w):
     return {"workload": w.name, "batch": w.batch, "context": w.context, "n_q_heads": w.n_q_heads,
             "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "chunk": w.chunk, "levels": w.levels,
-            "n_refs": w.n_refs, "p": w.p, "refs": w.refs_mode, "needles_per_seq": w.needles,
+            "n_refs": w.n_refs, "p": w.p, "p_schedule": w.p_schedule, "refs": w.refs_mode,
+            "needles_per_seq": w.needles,
             "l2": "flushed (256 MiB write) before every timed step, outside the timed region"}
 
 
@@ -272,14 +284,14 @@ def zha_arm(args, w, world, rank, local):
     cap = w.context + n_total + 8
     inp = make_inputs(w, device="cuda", capacity=cap)
     cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs, w.dtype,
-                     cap)
+                     cap, flags=zha.ZHA_FLAG_TCGEN05 if args.scorer == "tcgen05" else 0)
     buf = zha.Buffers(cfg)
     K, V, refs, lens = inp.K, inp.V, inp.refs, inp.lens
     k_new, v_new, qs = decode_stream(w, n_total, device="cuda")
     out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=w.torch_dtype(), device="cuda")
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
-    p = w.p
+    p = zha.p_schedule(w.p, w.levels, w.p_schedule)
 
     torch.cuda.synchronize()
     t0 = time.perf_counter()
@@ -366,7 +378,8 @@ def zha_arm(args, w, world, rank, local):
            "touched_frac_of_hbm": touched_mean / (ms_per_step / 1e3) / 1e9 / peak,
            "keys_attended": keys_share,
            "candidates_per_step": float(cand_per_step.mean()),
-           "gpu_launches": int(launches), "cuda_graph": graph is not None, "clocks": clocks}
+           "gpu_launches": int(launches), "cuda_graph": graph is not None, "scorer": args.scorer,
+           "clocks": clocks}
 
     # per-kernel CUDA-event timing: a second pass of K steps, every launch bracketed
     if not args.no_profile:
@@ -558,10 +571,10 @@ def sweep_mode(args):
     peak, _ = read_peaks()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     Ns = [int(x) for x in args.sweep_n.split(",")]
-    for tree in ("deep", "wide"):
+    for tree in args.sweep_trees.split(","):
         for refs_mode in ("random", "aligned"):
             for N in Ns:
-                w = dataclasses.replace(sweep_workload(N, tree), refs_mode=refs_mode)
+                w = dataclasses.replace(sweep_workload(N, tree), refs_mode=refs_mode, p_schedule=args.p_schedule)
                 n, W = args.steps, args.warmup
                 cap = N + n + W + 8
                 inp = make_inputs(w, device="cuda", capacity=cap)
@@ -572,11 +585,13 @@ def sweep_mode(args):
                 k_new, v_new, qs = decode_stream(w, n + W, device="cuda")
                 out = torch.empty_like(qs[0])
                 ms, cand, toks = _timed_decode(zha, cfg, buf, inp.K, inp.V, inp.refs, inp.lens, qs, k_new, v_new,
-                                               w.p, out, flush, 0, n, W, w)
+                                               zha.p_schedule(w.p, w.levels, w.p_schedule), out, flush, 0, n,
+                                               W, w)
                 dense_ms = _timed_dense(zha, cfg, buf, qs[0], inp.K, inp.V, inp.lens, out, flush, n, W)
                 us = ms / n * 1e3
                 touched = _bytes(w, cand, toks)
                 print(json.dumps({"mode": "sweep", "tree": tree, "refs": refs_mode, "context": N, "p": w.p,
+                                  "p_schedule": w.p_schedule,
                                   "zha_us_per_step": us, "dense_us_per_step": dense_ms * 1e3,
                                   "speedup_vs_dense": dense_ms * 1e3 / us,
                                   "keys_attended": toks / (w.batch * w.n_kv_heads * (N + W + n)),

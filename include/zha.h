@@ -76,7 +76,13 @@ enum { ZHA_BF16 = 0, ZHA_F32 = 1 };
 enum {
     /* current chunk = only the incomplete tail [c*floor(N/c), N) instead of the
      * chunk holding the newest token [c*floor((N-1)/c), N) */
-    ZHA_FLAG_TAIL_ONLY = 1
+    ZHA_FLAG_TAIL_ONLY = 1,
+    /* score candidate nodes with the tcgen05 kernel (TMA-fed tensor-core MMAs
+     * accumulating in tensor memory) where it applies: bf16, head_dim 128,
+     * n_refs 16, G <= 16, batch * n_kv_heads <= 16. The default is the
+     * mma.sync kernel, which streams the summaries at a higher fraction of
+     * HBM bandwidth on this path */
+    ZHA_FLAG_TCGEN05 = 2
 };
 
 #define ZHA_MAX_LEVELS 8
@@ -258,6 +264,26 @@ ZHA_API zha_status zha_topp_select(const float *scores, const int32_t *counts, i
                            int64_t stride, float p, uint8_t *kept, int32_t *dev_status,
                            void *stream);
 
+
+/* schedules of zha_p_schedule */
+enum { ZHA_P_FIXED = 0, ZHA_P_DEPTH_ROOT = 1 };
+
+/*
+ * zha_p_schedule -- per-level routing fractions for zha_route / zha_decode,
+ * written to p_levels[0..levels-1] (index l-1 is level l); host memory, no
+ * device work. The caveat cards of the MarkTechPost explainer (tab 5, "Top-p
+ * must scale with depth") warn that one p used at every level lets coverage
+ * shrink as the tree deepens: where mass is spread evenly, each level keeps
+ * about a fraction p of what reaches it, so the kept leaves hold about p^L.
+ *   ZHA_P_FIXED       p at every level (the pages' configurations).
+ *   ZHA_P_DEPTH_ROOT  p^(1/L) at every level, whose product over the L levels
+ *                     is p. The pages name no schedule; this is the plainest
+ *                     one that undoes the p^L shrinkage.
+ * p >= 1 gives 1 at every level. p <= 0 or NaN, levels outside
+ * 1..ZHA_MAX_LEVELS, a null p_levels or an unknown schedule:
+ * ZHA_ERR_INVALID_ARG (nothing written).
+ */
+ZHA_API zha_status zha_p_schedule(float p, int32_t levels, int32_t schedule, float *p_levels);
 
 /*
  * Instrumentation (no counterpart on the pages; for measurement only).

@@ -213,6 +213,15 @@ def route(tree: Tree, q: np.ndarray, p) -> Route:
     return out
 
 
+def depth_root_schedule(p: float, L: int) -> list:
+    """Per-level fractions p^(1/L) (level 1 first), so that their product over the
+    L levels is p. The explainer's caveat cards (MarkTechPost, tab 5) warn that
+    one fixed p per level shrinks coverage with depth; the pages name no
+    schedule, and this is the plainest one that undoes the p^L shrinkage."""
+    v = 1.0 if p >= 1.0 else float(p) ** (1.0 / L)
+    return [v] * L
+
+
 def token_set(N: int, c: int, kept_leaf: np.ndarray, tail_only: bool = False) -> np.ndarray:
     """Attended tokens: sink, kept leaf chunks, current chunk -> bool[N]."""
     kl = np.ascontiguousarray(kept_leaf, dtype=np.uint8)

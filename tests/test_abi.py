@@ -93,3 +93,20 @@ def test_invalid_arguments_are_rejected_before_launch(zha):
     assert L.zha_dense_decode(ctypes.byref(cfg), ctypes.c_void_p(18), ctypes.c_void_p(16), ctypes.c_void_p(16),
                               ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), None, None) == 1
     assert L.zha_status_string(3).decode().startswith("capacity")
+
+
+def test_p_schedule_host_rule(zha, orc):
+    """zha_p_schedule is host-only: fixed = p everywhere; depth-root = the
+    oracle's p^(1/L) rounded once to fp32; invalid arguments are refused."""
+    import numpy as np
+    for p in (0.5, 0.75, 0.95, 0.999):
+        for L in (1, 3, 6, 8):
+            assert zha.p_schedule(p, L, "fixed") == [float(np.float32(p))] * L
+            want = [float(np.float32(v)) for v in orc.depth_root_schedule(float(np.float32(p)), L)]
+            assert zha.p_schedule(p, L, "root") == want
+    assert zha.p_schedule(1.5, 4, "root") == [1.0] * 4
+    out = (ctypes.c_float * 8)()
+    L = zha.lib()
+    for args in ((0.0, 3, 1), (float("nan"), 3, 1), (0.9, 0, 1), (0.9, 9, 1), (0.9, 3, 7)):
+        assert L.zha_p_schedule(ctypes.c_float(args[0]), args[1], args[2], out) == 1
+    assert L.zha_p_schedule(ctypes.c_float(0.9), 3, 1, None) == 1

@@ -164,6 +164,39 @@ def test_route_matches_oracle(zha, w):
         assert total_flipped <= max(2, heads // 8), total_flipped
 
 
+@pytest.mark.parametrize("w", CASES[1:4], ids=IDS[1:4])
+def test_route_depth_schedule_matches_oracle(zha, w):
+    """Routing with the depth-root schedule p^(1/L) per level (from zha_p_schedule)
+    equals the oracle's routing with the same per-level fractions."""
+    cfg, inp, dev, buf = T.build_case(zha, w, lens=_lens_for(w))
+    zha.tree_build(cfg, buf.tree, dev.K, dev.refs, dev.lens, buf.status)
+    p_levels = zha.p_schedule(w.p, w.levels, "root")
+    assert all(p > w.p for p in p_levels)
+    zha.route(cfg, buf.tree, dev.q, dev.lens, p_levels, buf.sel, buf.workspace, buf.status)
+    torch.cuda.synchronize()
+    buf.check_status()
+    states = {l: buf.level_state(l) for l in range(1, w.levels + 1)}
+    s = T.scale_of(w)
+    G = w.group
+    total_flipped = 0
+    for b in range(w.batch):
+        N = int(inp.lens[b])
+        for kvh in range(w.n_kv_heads):
+            t = T.oracle_tree(w, inp, b, kvh, N, s)
+            q = T.np64(inp.q[b, kvh * G:(kvh + 1) * G])
+            r = orc.route(t, q, p_levels)
+            flipped, worst = T.compare_routing(r, states, b, kvh, G, N, w, p_levels)
+            assert worst <= T.TOL[w.dtype], worst
+            total_flipped += len(flipped)
+            for h in range(G):
+                if h in flipped:
+                    continue
+                lk = buf.sel["level_kept"][b, kvh * G + h].cpu().numpy()
+                for level in range(1, w.levels + 1):
+                    assert lk[level - 1] == r.kept[level - 1][h].sum()
+    assert total_flipped <= max(2, w.batch * w.n_q_heads // 8), total_flipped
+
+
 # ------------------------------------------------------------------ attention
 
 

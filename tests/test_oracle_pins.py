@@ -360,3 +360,62 @@ def test_route_invariants_random(orc):
                 # the kept mass reaches p of the candidates' mass
                 w = np.exp(E - E.max())
                 assert w[kept[cand]].sum() >= p * w.sum() * (1 - 1e-12)
+
+
+# ------------------------------------------------------------------ per-level p
+
+
+def _uniform_tree(orc, m, d, c, L, R, G, seed):
+    """Identical keys everywhere and N = m * c^L: every node of a level has the
+    same planes, so all candidates of a level tie and top-p keeps the first
+    ceil(p * count) of them in index order."""
+    N = m * c ** L
+    g = rng(seed)
+    K = np.tile(g.normal(size=d), (N, 1))
+    refs = g.normal(size=(R, d)) / math.sqrt(d)
+    q = g.normal(size=(G, d))
+    return orc.build_tree(K, refs, N, c, L), q
+
+
+def _uniform_counts(m, c, p_levels):
+    """Closed form of the kept count per level (level L first) on a uniform tree."""
+    counts, n_cand = [], m
+    for level in range(len(p_levels), 0, -1):
+        k = math.ceil(p_levels[level - 1] * n_cand)
+        counts.append((level, n_cand, k))
+        n_cand = k * c
+    return counts
+
+
+def test_per_level_p_closed_form_on_uniform_tree(orc):
+    """Distinct p per level: each level keeps exactly its own ceil(p_l * candidates)
+    (which list entry serves which level is pinned by the distinct counts)."""
+    m, d, c, L, R, G = 5, 16, 4, 3, 2, 2
+    t, q = _uniform_tree(orc, m, d, c, L, R, G, 80)
+    p_levels = [0.3, 0.55, 0.7]          # levels 1, 2, 3
+    r = orc.route(t, q, p_levels)
+    for h in range(G):
+        for level, n_cand, k in _uniform_counts(m, c, p_levels):
+            cand = np.nonzero(r.cand[level - 1][h])[0]
+            kept = np.nonzero(r.kept[level - 1][h])[0]
+            assert np.array_equal(cand, np.arange(n_cand)), (h, level)
+            assert np.array_equal(kept, np.arange(k)), (h, level)
+    # reversed list gives other counts: the pin separates the levels
+    assert _uniform_counts(m, c, p_levels[::-1]) != _uniform_counts(m, c, p_levels)
+
+
+@pytest.mark.parametrize("p", [0.6, 0.8, 0.95])
+def test_depth_root_schedule_restores_coverage(orc, p):
+    """On a tree with evenly spread mass the kept share of leaves is about p^L
+    under one fixed p and about p under p^(1/L) per level (the depth caveat of
+    the explainer, tab 5)."""
+    m, d, c, L, R, G = 64, 8, 4, 3, 2, 1
+    t, q = _uniform_tree(orc, m, d, c, L, R, G, 81)
+    n1 = m * c ** (L - 1)
+    sched = orc.depth_root_schedule(p, L)
+    assert len(sched) == L and math.prod(sched) == pytest.approx(p, rel=1e-12)
+    assert orc.depth_root_schedule(1.0, L) == [1.0] * L
+    fixed = orc.route(t, q, p).kept[0][0].sum() / n1
+    root = orc.route(t, q, sched).kept[0][0].sum() / n1
+    assert fixed == pytest.approx(p ** L, abs=0.02)
+    assert root == pytest.approx(p, abs=0.02)

@@ -24,7 +24,7 @@ zha_status check_config(const zha_config *c) {
     if (!pow2(c->chunk) || c->chunk < 2 || c->chunk > 256) return ZHA_ERR_UNSUPPORTED;
     if (c->levels > ZHA_MAX_LEVELS || c->n_refs > 32) return ZHA_ERR_UNSUPPORTED;
     if (c->dtype != ZHA_BF16 && c->dtype != ZHA_F32) return ZHA_ERR_UNSUPPORTED;
-    if (c->flags & ~ZHA_FLAG_TAIL_ONLY) return ZHA_ERR_UNSUPPORTED;
+    if (c->flags & ~(ZHA_FLAG_TAIL_ONLY | ZHA_FLAG_TCGEN05)) return ZHA_ERR_UNSUPPORTED;
     // int32 token and leaf indices; fixed-point mass sums need <= 2^23 candidates
     if (c->max_len > (1 << 30) || c->max_len / c->chunk > (1 << 23)) return ZHA_ERR_UNSUPPORTED;
     if (c->attn_splits < 0 || c->attn_splits > 4096) return ZHA_ERR_INVALID_ARG;
@@ -272,6 +272,18 @@ zha_status zha_topp_select(const float *scores, const int32_t *counts, int32_t n
     if (stride > (1 << 23)) return ZHA_ERR_UNSUPPORTED;
     return cuda_status(zha::launch_topp_select(scores, counts, n_sets, stride, p, kept, dev_status,
                                                static_cast<cudaStream_t>(stream)));
+}
+
+zha_status zha_p_schedule(float p, int32_t levels, int32_t schedule, float *p_levels) {
+    if (!p_levels || !(p > 0.f) || levels < 1 || levels > ZHA_MAX_LEVELS) return ZHA_ERR_INVALID_ARG;
+    if (schedule != ZHA_P_FIXED && schedule != ZHA_P_DEPTH_ROOT) return ZHA_ERR_INVALID_ARG;
+    float v = p;
+    if (p >= 1.f)
+        v = 1.f;
+    else if (schedule == ZHA_P_DEPTH_ROOT)
+        v = static_cast<float>(pow(static_cast<double>(p), 1.0 / levels));
+    for (int l = 0; l < levels; ++l) p_levels[l] = v;
+    return ZHA_OK;
 }
 
 }  // extern "C"

@@ -174,6 +174,12 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
 cudaError_t launch_decode_write(const Geo &g, void *K, void *V, int32_t *lens, const void *k_new,
                                 const void *v_new, int32_t *status, cudaStream_t st);
 Geo make_geo_for(const zha_config *c);
+bool score_tc_supported(const Geo &g);
+cudaError_t launch_score_tc(const Geo &g, const void *mu_level, const float *bias, const void *q,
+                            const int32_t *lens, int level, int32_t *cand, uint32_t *cmask, float *scores,
+                            int32_t *count, uint32_t *maxkey, uint32_t *minkey, const int32_t *plist_up,
+                            const uint32_t *pmask_up, const int32_t *pcount_up, int32_t *status,
+                            cudaStream_t st);
 cudaError_t launch_topp_select(const float *scores, const int32_t *counts, int n_sets,
                                int64_t stride, float p, uint8_t *kept, int32_t *status,
                                cudaStream_t st);

@@ -758,7 +758,12 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
         const int64_t capv = g.capv[level];
         {
             ProfScope ps(score_names[level], st);
-            if (g.dtype == ZHA_BF16) {
+            if (g.dtype == ZHA_BF16 && (g.flags & ZHA_FLAG_TCGEN05) && score_tc_supported(g)) {
+                e = launch_score_tc(g, tb + g.mu_off[level], reinterpret_cast<const float *>(tb + g.bias_off[level]),
+                                    q, lens, level, lw.cand, lw.cmask, lw.scores, lw.count, lw.maxkey, lw.minkey,
+                                    up.plist, up.pmask, up.pcount, status, st);
+                if (e != cudaSuccess) return e;
+            } else if (g.dtype == ZHA_BF16) {
                 const auto *mu = reinterpret_cast<const __nv_bfloat16 *>(tb + g.mu_off[level]);
                 const auto *bias = reinterpret_cast<const float *>(tb + g.bias_off[level]);
                 const auto *qq = static_cast<const __nv_bfloat16 *>(q);

@@ -47,6 +47,7 @@ class Workload:
     seed: int
     diffuse_nodes: int = 0
     refs_mode: str = "random"
+    p_schedule: str = "fixed"   # "fixed": p per level; "root": p^(1/L) per level
 
     @property
     def group(self) -> int:
@@ -62,12 +63,18 @@ WIDE_32K = Workload("wide N=32768 c=256 L=1", 1, 32, 4, 128, 32768, 256, 1, 16, 
 DEEP_256K = Workload("deep N=262144 c=4 L=6 B=4", 4, 32, 4, 128, 262144, 4, 6, 16, 0.95, 256, "bf16", 2,
                      diffuse_nodes=32)
 DEEP_1M = Workload("deep N=1048576 c=4 L=6", 1, 32, 4, 128, 1048576, 4, 6, 16, 0.95, 256, "bf16", 3)
+# The geometry of the pages' latency model (MarkTechPost, "How fast is ZHA" and the
+# explainer's tab 4): one reference per tree, chunks of 8, p = 0.75, batch 1.
+# Four levels give 4,096 tokens per top node, as in the deep tree.
+SPEED_256K = Workload("speed-model N=262144 c=8 L=4 R=1 p=0.75", 1, 32, 4, 128, 262144, 8, 4, 1, 0.75, 64,
+                      "bf16", 5)
 
 
 def sweep_workload(N: int, tree: str) -> Workload:
-    """Context-sweep workload (batch 1, 32/4 heads, d 128) with the deep or wide tree."""
-    c, L = (4, 6) if tree == "deep" else (256, 1)
-    return Workload(f"sweep-{tree} N={N}", 1, 32, 4, 128, N, c, L, 16, 0.95, 64, "bf16", 4)
+    """Context-sweep workload (batch 1, 32/4 heads, d 128) with the deep, wide or
+    speed-model (R=1, c=8, L=4, p=0.75) tree."""
+    c, L, R, p = {"deep": (4, 6, 16, 0.95), "wide": (256, 1, 16, 0.95), "speed": (8, 4, 1, 0.75)}[tree]
+    return Workload(f"sweep-{tree} N={N}", 1, 32, 4, 128, N, c, L, R, p, 64, "bf16", 4)
 
 
 @dataclass

@@ -17,6 +17,8 @@ LIB_PATH = os.path.join(_HERE, "libzha.so")
 
 ZHA_BF16, ZHA_F32 = 0, 1
 ZHA_FLAG_TAIL_ONLY = 1
+ZHA_FLAG_TCGEN05 = 2
+ZHA_P_FIXED, ZHA_P_DEPTH_ROOT = 0, 1
 ZHA_MAX_LEVELS = 8
 STATUS_NAMES = {0: "ZHA_OK", 1: "ZHA_ERR_INVALID_ARG", 2: "ZHA_ERR_UNSUPPORTED",
                 3: "ZHA_ERR_CAPACITY", 4: "ZHA_ERR_CUDA", 5: "ZHA_ERR_TIMEOUT"}
@@ -76,6 +78,7 @@ def _load():
         "zha_decode": ([CP, P, P, P, P, P, P, P, P, P, SP, P, P, P, P], i32),
         "zha_dense_decode": ([CP, P, P, P, P, P, P, P, P], i32),
         "zha_topp_select": ([P, P, i32, i64, f32, P, P, P], i32),
+        "zha_p_schedule": ([f32, i32, i32, ctypes.POINTER(f32)], i32),
         "zha_launch_count": ([], ctypes.c_uint64),
         "zha_profile_enable": ([i32], i32),
         "zha_profile_read": ([ctypes.c_char_p, i32, ctypes.POINTER(ctypes.c_double),
@@ -149,6 +152,14 @@ def _plevels(cfg: Config, p):
         p = [float(p)] * cfg.levels
     arr = (ctypes.c_float * cfg.levels)(*[float(x) for x in p])
     return arr
+
+
+def p_schedule(p: float, levels: int, schedule=ZHA_P_FIXED) -> list[float]:
+    """Per-level fractions (index l-1 is level l) from libzha's schedule rule."""
+    schedule = {"fixed": ZHA_P_FIXED, "root": ZHA_P_DEPTH_ROOT}.get(schedule, schedule)
+    out = (ctypes.c_float * max(int(levels), 1))()
+    check(_lib.zha_p_schedule(float(p), int(levels), int(schedule), out), "zha_p_schedule")
+    return [float(x) for x in out[:levels]]
 
 
 def _sel(sel) -> Selection:
