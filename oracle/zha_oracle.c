@@ -61,6 +61,7 @@
 #define ORC_STORE_F64 0
 #define ORC_STORE_F32 1
 #define ORC_STORE_BF16 2
+#define ORC_STORE_MXFP8 3
 
 /* Round-to-nearest-even to the storage format the summaries are kept in,
  * so that parents are built from the same stored children a GPU build
@@ -81,6 +82,78 @@ static double store_round(double x, int storage)
 }
 
 double orc_round_storage(double x, int storage) { return store_round(x, storage); }
+
+/*
+ * Low-precision summaries (the MarkTechPost article's TL;DR box says an FP4
+ * router variant was also tried, and gives no format; the reading taken
+ * here, at 8 bits): mu of every plane is kept in
+ * blocks of 32 consecutive coordinates, each block as one power-of-two scale
+ * 2^e times 32 FP8 E4M3 values, the block layout of the OCP Microscaling (MX)
+ * specification v1.0. E4M3 as defined there: 1 sign, 4 exponent bits with
+ * bias 7, 3 mantissa bits; normal magnitudes 2^-6 .. 448, subnormals are
+ * multiples of 2^-9. Rounding to nearest, ties to even. The block's e is the
+ * smallest integer with max|x| <= 448 * 2^e, so that no element saturates
+ * (a choice made here; the MX text allows saturation instead).
+ */
+static double e4m3_round(double x)
+{
+    if (x == 0.0 || !isfinite(x))
+        return x;
+    double a = fabs(x), r;
+    if (a < ldexp(1.0, -6)) {
+        r = ldexp(nearbyint(ldexp(a, 9)), -9);   /* subnormal grid 2^-9 */
+    } else {
+        int e;
+        double m = frexp(a, &e);                 /* a = m 2^e, m in [0.5, 1) */
+        r = ldexp(nearbyint(ldexp(m, 4)), e - 4); /* 4 significant bits */
+    }
+    if (r > 448.0)
+        r = 448.0;
+    return x < 0 ? -r : r;
+}
+
+double orc_e4m3_round(double x) { return e4m3_round(x); }
+
+/* Exponent e of one block's scale 2^e; 0 for an all-zero block. */
+static int mx_block_exponent(const double *x, int n)
+{
+    double amax = 0.0;
+    for (int k = 0; k < n; ++k)
+        if (fabs(x[k]) > amax)
+            amax = fabs(x[k]);
+    if (amax == 0.0)
+        return 0;
+    int k;
+    double f = frexp(amax, &k);      /* amax = f 2^k; 448 = 0.875 2^9 */
+    int e = (f <= 0.875) ? k - 9 : k - 8;
+    if (e < -126) e = -126;
+    if (e > 127) e = 127;
+    return e;
+}
+
+/* Round a plane (d coordinates, d a multiple of 32) to its MX-FP8 value in place;
+ * exps (optional, d/32 entries) receives the block exponents. */
+void orc_mx_round(double *x, int d, int *exps)
+{
+    for (int b0 = 0; b0 < d; b0 += 32) {
+        int e = mx_block_exponent(x + b0, 32);
+        for (int k = b0; k < b0 + 32; ++k)
+            x[k] = ldexp(e4m3_round(ldexp(x[k], -e)), e);
+        if (exps)
+            exps[b0 / 32] = e;
+    }
+}
+
+/* Store one plane's mu in the summary format. */
+static void store_plane(double *m, int d, int storage)
+{
+    if (storage == ORC_STORE_MXFP8) {
+        orc_mx_round(m, d, NULL);
+        return;
+    }
+    for (int k = 0; k < d; ++k)
+        m[k] = store_round(m[k], storage);
+}
 
 int orc_num_threads(void)
 {
@@ -181,8 +254,7 @@ void orc_tree_update(const double *K, int64_t old_N, int64_t new_N, int d,
             double *m = mu[0] + (j * R + r) * d;
             double *bb = b[0] + j * R + r;
             plane_one_ref(c, d, xp, NULL, refs + (int64_t)r * d, s, m, bb);
-            for (int k = 0; k < d; ++k)
-                m[k] = store_round(m[k], storage);
+            store_plane(m, d, storage);
             *bb = store_round(*bb, storage == ORC_STORE_F64 ? ORC_STORE_F64 : ORC_STORE_F32);
         }
         if (xp != x)
@@ -212,8 +284,7 @@ void orc_tree_update(const double *K, int64_t old_N, int64_t new_N, int d,
                 double *m = mu[l - 1] + (p * R + r) * d;
                 double *bb = b[l - 1] + p * R + r;
                 plane_one_ref(nch, d, xp, ap, refs + (int64_t)r * d, s, m, bb);
-                for (int k = 0; k < d; ++k)
-                    m[k] = store_round(m[k], storage);
+                store_plane(m, d, storage);
                 *bb = store_round(*bb, storage == ORC_STORE_F64 ? ORC_STORE_F64 : ORC_STORE_F32);
             }
             if (xp != x)

@@ -28,8 +28,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "zha_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libzha_oracle.so")
 
-STORE_F64, STORE_F32, STORE_BF16 = 0, 1, 2
-_STORAGE = {"f64": STORE_F64, "f32": STORE_F32, "bf16": STORE_BF16}
+STORE_F64, STORE_F32, STORE_BF16, STORE_MXFP8 = 0, 1, 2, 3
+_STORAGE = {"f64": STORE_F64, "f32": STORE_F32, "bf16": STORE_BF16, "mxfp8": STORE_MXFP8}
 
 
 def build_library(force: bool = False) -> str:
@@ -53,6 +53,9 @@ def lib():
         i64, i32, f64 = ctypes.c_int64, ctypes.c_int, ctypes.c_double
         L.orc_round_storage.argtypes = [f64, i32]
         L.orc_round_storage.restype = f64
+        L.orc_e4m3_round.argtypes = [f64]
+        L.orc_e4m3_round.restype = f64
+        L.orc_mx_round.argtypes = [P, i32, P]
         L.orc_num_threads.restype = i32
         L.orc_level_nodes.argtypes = [i64, i32, i32]
         L.orc_level_nodes.restype = i64
@@ -87,6 +90,24 @@ def default_scale(d: int) -> float:
 
 def round_storage(x: float, storage: str) -> float:
     return lib().orc_round_storage(float(x), _STORAGE[storage])
+
+
+def e4m3_round(x: float) -> float:
+    """Nearest FP8 E4M3 value (ties to even, saturating at 448)."""
+    return lib().orc_e4m3_round(float(x))
+
+
+def mx_round(x: np.ndarray):
+    """MX-FP8 value of planes x [..., d] (blocks of 32 coordinates) -> (values, block exponents)."""
+    x = np.array(x, dtype=np.float64, order="C", copy=True)
+    d = x.shape[-1]
+    flat = x.reshape(-1, d)
+    exps = np.zeros((flat.shape[0], d // 32), dtype=np.int32)
+    for i in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[i])
+        lib().orc_mx_round(_ptr(row), d, exps[i].ctypes.data)
+        flat[i] = row
+    return flat.reshape(x.shape), exps.reshape(x.shape[:-1] + (d // 32,))
 
 
 def level_nodes(N: int, c: int, level: int) -> int:

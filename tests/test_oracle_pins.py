@@ -419,3 +419,88 @@ def test_depth_root_schedule_restores_coverage(orc, p):
     root = orc.route(t, q, sched).kept[0][0].sum() / n1
     assert fixed == pytest.approx(p ** L, abs=0.02)
     assert root == pytest.approx(p, abs=0.02)
+
+
+# ------------------------------------------------------- low-precision summaries
+
+
+def _e4m3_grid():
+    """Every finite non-negative E4M3 value, from its bit fields (bias 7)."""
+    vals = [m * 2.0 ** -9 for m in range(8)]                       # subnormals
+    vals += [(1 + m / 8) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8) if not (e == 15 and m == 7)]
+    return np.array(sorted(vals))
+
+
+def test_e4m3_rounding_matches_torch_float8(orc):
+    grid = _e4m3_grid()
+    assert grid[-1] == 448.0 and grid[1] == 2.0 ** -9 and len(grid) == 127
+    mids = (grid[:-1] + grid[1:]) / 2                              # exact ties
+    g = rng(90)
+    rnd = (g.uniform(-1, 1, size=20000) * 2.0 ** g.integers(-12, 9, size=20000)).astype(np.float32)
+    rnd = rnd[np.abs(rnd) <= 448]
+    x = np.concatenate([grid, -grid, mids, -mids, rnd.astype(np.float64)])
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = np.array([orc.e4m3_round(v) for v in x])
+    assert np.array_equal(mine, ref)
+    # ties go to the even mantissa: the midpoint above 1 (= 1 + 1/16) rounds down to 1
+    assert orc.e4m3_round(1.0 + 1 / 16) == 1.0 and orc.e4m3_round(1.0 + 3 / 16) == 1.25
+    assert orc.e4m3_round(1000.0) == 448.0 and orc.e4m3_round(-1000.0) == -448.0
+
+
+def test_mx_block_scale_closed_form(orc):
+    g = rng(91)
+    x = g.normal(size=(64, 128)) * 10.0 ** g.integers(-4, 4, size=(64, 1))
+    x[3, 32:64] = 0.0                                             # an all-zero block
+    v, e = orc.mx_round(x)
+    blocks = x.reshape(64, 4, 32)
+    amax = np.abs(blocks).max(axis=2)
+    live = amax > 0
+    scale = 2.0 ** e
+    # the smallest power of two that brings the block's maximum within 448
+    assert np.all(amax[live] <= 448 * scale[live]) and np.all(amax[live] > 224 * scale[live])
+    assert np.all(v.reshape(64, 4, 32)[~live] == 0)
+    # each element is the nearest E4M3 multiple of its block's scale
+    vb, sb = v.reshape(64, 4, 32), scale[:, :, None]
+    q = vb / sb
+    grid = _e4m3_grid()
+    assert np.all(np.isin(np.abs(q), grid))
+    err = np.abs(vb - blocks)
+    ulp = np.where(np.abs(blocks) / sb < 2.0 ** -6, 2.0 ** -9, 2.0 ** (np.floor(np.log2(np.maximum(np.abs(blocks) / sb, 1e-300))) - 3))
+    assert np.all(err <= 0.5 * ulp * sb * (1 + 1e-12))
+    # power-of-two equivariance and idempotence
+    v2, e2 = orc.mx_round(x * 8.0)
+    assert np.array_equal(v2, v * 8.0) and np.array_equal(e2[live], e[live] + 3)
+    v3, _ = orc.mx_round(v)
+    assert np.array_equal(v3, v)
+
+
+def test_mxfp8_storage_tree_builds_from_rounded_children(orc):
+    N, d, c, L = 512, 64, 4, 3
+    K = _keys(92, N, d, c)
+    refs = rng(93).normal(size=(4, d)) / math.sqrt(d)
+    s = 1 / math.sqrt(d)
+    t = orc.build_tree(K, refs, N, c, L, s, storage="mxfp8")
+    ref = orc.build_tree(K, refs, N, c, L, s)
+    for level in range(L):
+        m = t.mu[level][: t.n(level + 1)]
+        again, _ = orc.mx_round(m)
+        assert np.array_equal(again, m)                            # stored values are MX-FP8
+        # rounding error, relative to the block's largest coordinate: half an E4M3
+        # step (2^-4) per level, a parent inheriting its children's errors
+        r = ref.mu[level][: t.n(level + 1)]
+        bmax = np.abs(r).reshape(r.shape[:-1] + (d // 32, 32)).max(axis=-1, keepdims=True)
+        err = np.abs(m - r).reshape(bmax.shape[:-1] + (32,)) / bmax
+        assert err.max() <= (level + 1) * 2.0 ** -4
+        b = t.b[level][: t.n(level + 1)]
+        assert np.array_equal(b.astype(np.float32).astype(np.float64), b)   # bias kept in fp32
+    # estimates stay close to the exact tree's (the router's purpose)
+    q = rng(94).normal(size=d)
+    for level in range(L):
+        for n in range(t.n(level + 1)):
+            e_mx = orc.estimate(q, t.mu[level][n], t.b[level][n], s)
+            e_64 = orc.estimate(q, ref.mu[level][n], ref.b[level][n], s)
+            # |max_r a_r - max_r b_r| <= max_r |a_r - b_r| (triangle inequality per plane)
+            dmu = np.abs(t.mu[level][n] - ref.mu[level][n])
+            bound = np.max(s * dmu @ np.abs(q) + np.abs(t.b[level][n] - ref.b[level][n]))
+            assert abs(e_mx - e_64) <= bound + 1e-12
+            assert abs(e_mx - e_64) < 0.1
