@@ -42,6 +42,8 @@ def parse():
                     choices=["deep256k", "deep1m", "wide32k", "tiny", "small", "medium", "speed256k"])
     ap.add_argument("--refs", default="random", choices=["random", "aligned"])
     ap.add_argument("--p", type=float, default=None)
+    ap.add_argument("--summary", default="native", choices=["native", "mxfp8"],
+                    help="summary storage: mu in the KV dtype, or MX-FP8 (E4M3 blocks of 32 + scales)")
     ap.add_argument("--p-schedule", default="fixed", choices=["fixed", "root"],
                     help="per-level p: fixed p, or p^(1/L) at every level")
     ap.add_argument("--no-e2e", action="store_true")
@@ -73,7 +75,7 @@ def workload(args):
                                       context=65536, needles=64, diffuse_nodes=8),
          # one sequence of the 256K deep workload (a quarter of its bytes)
          "medium": dataclasses.replace(I.DEEP_256K, name="deep N=262144 c=4 L=6 B=1", batch=1)}[args.workload]
-    w = dataclasses.replace(w, refs_mode=args.refs, p_schedule=args.p_schedule)
+    w = dataclasses.replace(w, refs_mode=args.refs, p_schedule=args.p_schedule, summary=args.summary)
     if args.p is not None:
         w = dataclasses.replace(w, p=args.p)
     return w
@@ -216,7 +218,8 @@ def oracle_sample(w, inp, steps: int, warmup: int = 0):
     V = inp.V[0, 0, :N].to("cpu", torch.float64).numpy()
     refs = inp.refs[0].to("cpu", torch.float64).numpy()
     t0 = time.perf_counter()
-    tree = orc.build_tree(K, refs, N, w.chunk, w.levels, s, storage="bf16" if w.dtype == "bf16" else "f32")
+    storage = "mxfp8" if w.summary == "mxfp8" else ("bf16" if w.dtype == "bf16" else "f32")
+    tree = orc.build_tree(K, refs, N, w.chunk, w.levels, s, storage=storage)
     build_s = time.perf_counter() - t0
     q = inp.q[0, :G].to("cpu", torch.float64).numpy()
     rng = np.random.default_rng(0)
@@ -262,7 +265,7 @@ def oracle_p(orc, w):
 def config_of(w):
     return {"workload": w.name, "batch": w.batch, "context": w.context, "n_q_heads": w.n_q_heads,
             "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "chunk": w.chunk, "levels": w.levels,
-            "n_refs": w.n_refs, "p": w.p, "p_schedule": w.p_schedule, "refs": w.refs_mode,
+            "n_refs": w.n_refs, "p": w.p, "p_schedule": w.p_schedule, "summary": w.summary, "refs": w.refs_mode,
             "needles_per_seq": w.needles,
             "l2": "flushed (256 MiB write) before every timed step, outside the timed region"}
 
@@ -284,7 +287,7 @@ def zha_arm(args, w, world, rank, local):
     cap = w.context + n_total + 8
     inp = make_inputs(w, device="cuda", capacity=cap)
     cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs, w.dtype,
-                     cap, flags=zha.ZHA_FLAG_TCGEN05 if args.scorer == "tcgen05" else 0)
+                     cap, flags=zha.ZHA_FLAG_TCGEN05 if args.scorer == "tcgen05" else 0, summary=w.summary)
     buf = zha.Buffers(cfg)
     K, V, refs, lens = inp.K, inp.V, inp.refs, inp.lens
     k_new, v_new, qs = decode_stream(w, n_total, device="cuda")
@@ -355,7 +358,7 @@ def zha_arm(args, w, world, rank, local):
 
     # bytes the step must move (algorithmic), from the routed counts of each step
     es = 2 if w.dtype == "bf16" else 4
-    node_bytes = w.n_refs * w.head_dim * es + w.n_refs * 4          # summary keys + plane offsets
+    node_bytes = summary_node_bytes(w)                              # summary keys + plane offsets
     cand_bytes = node_bytes + 8 + w.group * 4                       # + index, head mask, G scores
     tok_bytes = 2 * w.head_dim * es                                 # K + V row
     h = hist_a.double().cpu()
@@ -553,9 +556,17 @@ def _timed_dense(zha, cfg, buf, q, K, V, lens, out, flush, n, warmup):
     return sum(a.elapsed_time(b) for a, b in ev) / n
 
 
+def summary_node_bytes(w):
+    """Bytes of one node record: mu (KV dtype, or E4M3 + one scale byte per 32) and fp32 offsets."""
+    if w.summary == "mxfp8":
+        return w.n_refs * w.head_dim + w.n_refs * (w.head_dim // 32) + w.n_refs * 4
+    es = 2 if w.dtype == "bf16" else 4
+    return w.n_refs * w.head_dim * es + w.n_refs * 4
+
+
 def _bytes(w, cand, tokens):
     es = 2 if w.dtype == "bf16" else 4
-    cand_bytes = w.n_refs * w.head_dim * es + w.n_refs * 4 + 8 + w.group * 4
+    cand_bytes = summary_node_bytes(w) + 8 + w.group * 4
     return cand * cand_bytes + tokens * 2 * w.head_dim * es + w.batch * w.n_kv_heads * 2 * w.group * w.head_dim * es
 
 
@@ -574,12 +585,13 @@ def sweep_mode(args):
     for tree in args.sweep_trees.split(","):
         for refs_mode in ("random", "aligned"):
             for N in Ns:
-                w = dataclasses.replace(sweep_workload(N, tree), refs_mode=refs_mode, p_schedule=args.p_schedule)
+                w = dataclasses.replace(sweep_workload(N, tree), refs_mode=refs_mode, p_schedule=args.p_schedule,
+                                        summary=args.summary)
                 n, W = args.steps, args.warmup
                 cap = N + n + W + 8
                 inp = make_inputs(w, device="cuda", capacity=cap)
                 cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs,
-                                 w.dtype, cap)
+                                 w.dtype, cap, summary=w.summary)
                 buf = zha.Buffers(cfg)
                 zha.tree_build(cfg, buf.tree, inp.K, inp.refs, inp.lens, buf.status)
                 k_new, v_new, qs = decode_stream(w, n + W, device="cuda")
@@ -590,7 +602,7 @@ def sweep_mode(args):
                 dense_ms = _timed_dense(zha, cfg, buf, qs[0], inp.K, inp.V, inp.lens, out, flush, n, W)
                 us = ms / n * 1e3
                 touched = _bytes(w, cand, toks)
-                print(json.dumps({"mode": "sweep", "tree": tree, "refs": refs_mode, "context": N, "p": w.p,
+                print(json.dumps({"mode": "sweep", "tree": tree, "refs": refs_mode, "context": N, "p": w.p, "summary": w.summary,
                                   "p_schedule": w.p_schedule,
                                   "zha_us_per_step": us, "dense_us_per_step": dense_ms * 1e3,
                                   "speedup_vs_dense": dense_ms * 1e3 / us,
@@ -618,7 +630,8 @@ def incremental_mode(args, w):
     N = w.context
     cap = N + len(ps) * (n + W) + 8
     inp = make_inputs(w, device="cuda", capacity=cap)
-    cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs, w.dtype, cap)
+    cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs, w.dtype, cap,
+                     summary=w.summary)
     buf = zha.Buffers(cfg)
     lens = torch.zeros_like(inp.lens)
     block = 4096

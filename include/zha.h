@@ -87,6 +87,21 @@ enum {
 
 #define ZHA_MAX_LEVELS 8
 
+/* cfg->summary: how the tree keeps each plane's mu (the bias is always fp32).
+ *   ZHA_SUMMARY_NATIVE  mu in the KV dtype.
+ *   ZHA_SUMMARY_MXFP8   low-precision router summaries (the MarkTechPost
+ *       article's TL;DR box mentions an FP4 router variant without a format;
+ *       this library's reading, at 8 bits): mu in blocks of 32 consecutive
+ *       coordinates, each block one power-of-two scale 2^e (a biased exponent
+ *       byte e + 127) times 32 FP8 E4M3 values, the block layout of the OCP
+ *       Microscaling (MX) specification v1.0; e is the smallest exponent with
+ *       max|x| <= 448 * 2^e, elements round to nearest even. A node record
+ *       shrinks from R*d*2 + 4R bytes to R*d + R*d/32 + 4R. Parents are built
+ *       from the stored (rounded) children. Requires dtype ZHA_BF16. Queries
+ *       are rounded to fp16 for scoring against these summaries (exact for
+ *       |q_k| in [2^-14, 65504]; below, an absolute error under 2^-25). */
+enum { ZHA_SUMMARY_NATIVE = 0, ZHA_SUMMARY_MXFP8 = 1 };
+
 typedef struct zha_config {
     int32_t batch;       /* B */
     int32_t n_q_heads;   /* Hq */
@@ -100,7 +115,8 @@ typedef struct zha_config {
     float scale;         /* s; <= 0 selects 1/sqrt(head_dim) */
     int32_t flags;       /* ZHA_FLAG_* */
     int32_t attn_splits; /* split-K CTAs per (sequence, KV head); 0 = auto */
-    int32_t reserved[3];
+    int32_t summary;     /* ZHA_SUMMARY_NATIVE or ZHA_SUMMARY_MXFP8 */
+    int32_t reserved[2]; /* zero */
 } zha_config;
 
 /*
@@ -147,12 +163,19 @@ ZHA_API int64_t zha_level_nodes(const zha_config *cfg, int64_t n_tokens, int32_t
 
 /* Bytes of the tree buffer for cfg->max_len tokens per sequence, and the
  * byte offsets of level l's arrays inside it:
- *   mu   [batch][n_kv_heads][cap_l][n_refs][head_dim]  dtype (summary keys)
+ *   mu   [batch][n_kv_heads][cap_l][n_refs][head_dim]  dtype (summary keys),
+ *        or FP8 E4M3 bytes with ZHA_SUMMARY_MXFP8
  *   bias [batch][n_kv_heads][cap_l][n_refs]            float (plane offsets)
  * A node's plane r evaluates to s*q.mu_r + bias_r. */
 ZHA_API size_t zha_tree_bytes(const zha_config *cfg);
 ZHA_API zha_status zha_tree_level_offsets(const zha_config *cfg, int32_t level, size_t *mu_off,
                                   size_t *bias_off);
+
+/* ZHA_SUMMARY_MXFP8 only: byte offset of level l's block scales,
+ *   scale [batch][n_kv_heads][cap_l][n_refs][head_dim / 32]  uint8 = e + 127,
+ * mu_r[k] = e4m3(mu byte k) * 2^(scale[k / 32] - 127). ZHA_ERR_INVALID_ARG
+ * for the native format. */
+ZHA_API zha_status zha_tree_level_scales(const zha_config *cfg, int32_t level, size_t *scale_off);
 
 /* Bytes of scratch every call below may use (routing state + split-K partials). */
 ZHA_API size_t zha_workspace_bytes(const zha_config *cfg);

@@ -228,6 +228,29 @@ void orc_direct_planes(const double *K, int64_t t0, int64_t t1, int d,
 }
 
 /*
+ * R2 for one parent from given children: cmu [nch][R][d] and cb [nch][R]
+ * (for instance the children a GPU stored), with the result stored as
+ * `storage` would keep it. mu: [R][d], b: [R].
+ */
+void orc_parent_planes(const double *cmu, const double *cb, int64_t nch, int d,
+                       const double *refs, int R, double s, int storage, double *mu, double *b)
+{
+    const double **x = (const double **)malloc((size_t)nch * sizeof(double *));
+    double *a = (double *)malloc((size_t)nch * sizeof(double));
+    for (int r = 0; r < R; ++r) {
+        for (int64_t i = 0; i < nch; ++i) {
+            x[i] = cmu + (i * R + r) * d;
+            a[i] = cb[i * R + r];
+        }
+        plane_one_ref(nch, d, x, a, refs + (int64_t)r * d, s, mu + (int64_t)r * d, b + r);
+        store_plane(mu + (int64_t)r * d, d, storage);
+        b[r] = store_round(b[r], storage == ORC_STORE_F64 ? ORC_STORE_F64 : ORC_STORE_F32);
+    }
+    free(a);
+    free(x);
+}
+
+/*
  * Build or extend the tree of ONE (sequence, KV head) from old_N to new_N
  * tokens. mu[l-1]: [n_l][R][d], b[l-1]: [n_l][R] for the caller's capacity.
  * Nodes that a longer cache adds or changes are (R3) the new leaf chunks and,

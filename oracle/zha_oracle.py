@@ -56,6 +56,7 @@ def lib():
         L.orc_e4m3_round.argtypes = [f64]
         L.orc_e4m3_round.restype = f64
         L.orc_mx_round.argtypes = [P, i32, P]
+        L.orc_parent_planes.argtypes = [P, P, i64, i32, P, i32, f64, i32, P, P]
         L.orc_num_threads.restype = i32
         L.orc_level_nodes.argtypes = [i64, i32, i32]
         L.orc_level_nodes.restype = i64
@@ -173,6 +174,17 @@ def direct_planes(K: np.ndarray, t0: int, t1: int, refs: np.ndarray, s: float):
     mu = np.zeros((R, d))
     b = np.zeros(R)
     lib().orc_direct_planes(_ptr(K), int(t0), int(t1), d, _ptr(refs), R, float(s), _ptr(mu), _ptr(b))
+    return mu, b
+
+
+def parent_planes(child_mu: np.ndarray, child_b: np.ndarray, refs: np.ndarray, s: float,
+                  storage: str = "f64"):
+    """Planes of one parent from given children (child_mu [n, R, d], child_b [n, R])."""
+    cm, cb, refs = _f64(child_mu), _f64(child_b), _f64(refs)
+    n, R, d = cm.shape
+    mu = np.zeros((R, d))
+    b = np.zeros(R)
+    lib().orc_parent_planes(_ptr(cm), _ptr(cb), n, d, _ptr(refs), R, float(s), _STORAGE[storage], _ptr(mu), _ptr(b))
     return mu, b
 
 

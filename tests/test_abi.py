@@ -110,3 +110,23 @@ def test_p_schedule_host_rule(zha, orc):
     for args in ((0.0, 3, 1), (float("nan"), 3, 1), (0.9, 0, 1), (0.9, 9, 1), (0.9, 3, 7)):
         assert L.zha_p_schedule(ctypes.c_float(args[0]), args[1], args[2], out) == 1
     assert L.zha_p_schedule(ctypes.c_float(0.9), 3, 1, None) == 1
+
+
+def test_mx_summary_config_and_layout(zha):
+    """MX-FP8 summaries need bf16 KV; their records take R*d + R*d/32 + 4R bytes
+    (2,176 at R=16, d=128) instead of R*2d + 4R (4,160), and the block scales
+    have their own offset, which the native format refuses."""
+    with pytest.raises(zha.ZhaError):
+        zha.config(1, 2, 1, 64, 4, 3, 16, "f32", 4096, summary="mxfp8")
+    with pytest.raises(zha.ZhaError):
+        zha.config(1, 2, 1, 64, 4, 3, 16, "bf16", 4096, summary=7)
+    mx = zha.config(1, 8, 1, 128, 4, 1, 16, "bf16", 4096, summary="mxfp8")
+    nat = zha.config(1, 8, 1, 128, 4, 1, 16, "bf16", 4096)
+    n1 = zha.level_nodes(mx, 4096, 1)
+    mu_off, b_off = zha.tree_level_offsets(mx, 1)
+    off = ctypes.c_size_t()
+    assert zha.lib().zha_tree_level_scales(ctypes.byref(mx), 1, ctypes.byref(off)) == 0
+    assert mu_off == 0 and off.value >= n1 * 16 * 128 and b_off >= off.value + n1 * 16 * 4
+    assert zha.tree_bytes(mx) == pytest.approx(n1 * 2176, rel=0.01)
+    assert zha.tree_bytes(nat) == pytest.approx(n1 * 4160, rel=0.01)
+    assert zha.lib().zha_tree_level_scales(ctypes.byref(nat), 1, ctypes.byref(off)) == 1

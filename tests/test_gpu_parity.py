@@ -23,6 +23,10 @@ def zha():
 
 CASES = T.small_workloads()
 IDS = [w.name for w in CASES]
+# plane counts below 16 (several candidates share one MMA tile)
+PACK_CASES = [Workload("R2 d64 c=4 L=3", 1, 16, 2, 64, 2047, 4, 3, 2, 0.9, 8, "bf16", 14),
+              Workload("R4 G16 c=8 L=3", 1, 32, 2, 128, 3001, 8, 3, 4, 0.9, 8, "bf16", 15),
+              Workload("R8 B=2 c=4 L=4", 2, 8, 1, 128, 2500, 4, 4, 8, 0.95, 8, "bf16", 16)]
 
 
 def _lens_for(w):
@@ -92,6 +96,15 @@ def _score_sets(seed, n_sets, stride):
     scores[3, 1::2] = scores[3, 0::2][: scores[3, 1::2].shape[0]]
     scores[4, :] = 0.25
     scores[5, : stride // 2] = -1.5
+    # a crossing among many exactly equal scores below a distinct maximum (more
+    # equal members than the value-bucket path holds: the radix path decides)
+    scores[6, :] = -3.0 + torch.rand(stride, generator=g) * 0.5
+    scores[6, ::2] = 1.0
+    scores[6, 0] = 2.0
+    counts[6] = stride
+    # a crossing inside a dense cluster of close but distinct scores
+    scores[7, :] = 0.5 + torch.arange(stride, dtype=torch.float32) * 1e-6
+    counts[7] = stride
     return scores, counts
 
 
@@ -122,7 +135,7 @@ def test_topp_select_matches_oracle(zha, p, stride):
 # ------------------------------------------------------------------ routing
 
 
-@pytest.mark.parametrize("w", CASES, ids=IDS)
+@pytest.mark.parametrize("w", CASES + PACK_CASES, ids=IDS + [w.name for w in PACK_CASES])
 def test_route_matches_oracle(zha, w):
     cfg, inp, dev, buf = T.build_case(zha, w, lens=_lens_for(w))
     zha.tree_build(cfg, buf.tree, dev.K, dev.refs, dev.lens, buf.status)

@@ -493,6 +493,12 @@ def test_mxfp8_storage_tree_builds_from_rounded_children(orc):
         assert err.max() <= (level + 1) * 2.0 ** -4
         b = t.b[level][: t.n(level + 1)]
         assert np.array_equal(b.astype(np.float32).astype(np.float64), b)   # bias kept in fp32
+    # the parent rule on given children reproduces the tree's parents
+    for level in range(1, L):
+        for node in range(t.n(level + 1)):
+            c0, c1 = node * c, min(node * c + c, t.n(level))
+            pm, pb = orc.parent_planes(t.mu[level - 1][c0:c1], t.b[level - 1][c0:c1], refs, s, "mxfp8")
+            assert np.array_equal(pm, t.mu[level][node]) and np.array_equal(pb, t.b[level][node])
     # estimates stay close to the exact tree's (the router's purpose)
     q = rng(94).normal(size=d)
     for level in range(L):

@@ -27,12 +27,29 @@ def np64(t: torch.Tensor) -> np.ndarray:
 
 
 def storage(w: Workload) -> str:
+    if w.summary == "mxfp8":
+        return "mxfp8"
     return "bf16" if w.dtype == "bf16" else "f32"
+
+
+def mx_decode(mu8: torch.Tensor, scales: torch.Tensor) -> np.ndarray:
+    """Values of MX-FP8 planes read back from the device: E4M3 bytes [..., d]
+    times 2^(scale byte - 127) per 32 coordinates, in float64."""
+    v = mu8.contiguous().view(torch.float8_e4m3fn).to(torch.float64)
+    sc = torch.exp2(scales.to(torch.float64) - 127.0).repeat_interleave(32, dim=-1)
+    return (v * sc).cpu().numpy()
+
+
+def mx_workloads():
+    """The bf16 parity cases with MX-FP8 summaries."""
+    import dataclasses
+    return [dataclasses.replace(w, name=w.name + " mxfp8", summary="mxfp8")
+            for w in small_workloads() if w.dtype == "bf16"]
 
 
 def make_cfg(zha, w: Workload, cap: int, flags: int = 0, splits: int = 0):
     return zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs,
-                      w.dtype, cap, flags=flags, attn_splits=splits)
+                      w.dtype, cap, flags=flags, attn_splits=splits, summary=w.summary)
 
 
 def to_device(inp, device="cuda"):

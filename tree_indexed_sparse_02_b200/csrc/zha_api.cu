@@ -29,6 +29,8 @@ zha_status check_config(const zha_config *c) {
     if (c->max_len > (1 << 30) || c->max_len / c->chunk > (1 << 23)) return ZHA_ERR_UNSUPPORTED;
     if (c->attn_splits < 0 || c->attn_splits > 4096) return ZHA_ERR_INVALID_ARG;
     if (!(c->scale == c->scale)) return ZHA_ERR_INVALID_ARG;
+    if (c->summary != ZHA_SUMMARY_NATIVE && c->summary != ZHA_SUMMARY_MXFP8) return ZHA_ERR_UNSUPPORTED;
+    if (c->summary == ZHA_SUMMARY_MXFP8 && c->dtype != ZHA_BF16) return ZHA_ERR_UNSUPPORTED;
     return ZHA_OK;
 }
 
@@ -44,15 +46,21 @@ Geo make_geo(const zha_config *c) {
     g.R = c->n_refs;
     g.dtype = c->dtype;
     g.flags = c->flags;
+    g.summary = c->summary;
     g.max_len = c->max_len;
     g.s = c->scale > 0.f ? c->scale : 1.f / sqrtf((float)c->head_dim);
     const size_t groups = (size_t)g.B * g.Hkv;
-    const size_t es = g.esize();
+    const size_t es = g.mu_esize();
     size_t off = 0;
     for (int l = 1; l <= g.L; ++l) {
         g.cap[l] = zha::level_nodes(g.max_len, g.c, l);
         g.mu_off[l] = off;
         off = align256(off + groups * g.cap[l] * g.R * g.d * es);
+        g.sc_off[l] = 0;
+        if (g.mx()) {
+            g.sc_off[l] = off;
+            off = align256(off + groups * g.cap[l] * g.R * (g.d / 32));
+        }
         g.bias_off[l] = off;
         off = align256(off + groups * g.cap[l] * g.R * sizeof(float));
     }
@@ -152,6 +160,15 @@ zha_status zha_tree_level_offsets(const zha_config *cfg, int32_t level, size_t *
     Geo g = make_geo(cfg);
     *mu_off = g.mu_off[level];
     *bias_off = g.bias_off[level];
+    return ZHA_OK;
+}
+
+zha_status zha_tree_level_scales(const zha_config *cfg, int32_t level, size_t *scale_off) {
+    zha_status s = check_config(cfg);
+    if (s != ZHA_OK) return s;
+    if (!scale_off || level < 1 || level > cfg->levels || cfg->summary != ZHA_SUMMARY_MXFP8)
+        return ZHA_ERR_INVALID_ARG;
+    *scale_off = make_geo(cfg).sc_off[level];
     return ZHA_OK;
 }
 

@@ -4,6 +4,8 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -25,12 +27,14 @@ __host__ __device__ inline int64_t level_nodes(int64_t n, int c, int level) {
 
 struct Geo {
     int B, Hq, Hkv, G, d, c, L, R, dtype, flags, splits;
+    int summary;                        // ZHA_SUMMARY_*
     int64_t max_len;
     float s;
     int64_t cap[kMaxLevels + 1];        // nodes per level at max_len (index = level)
     int64_t capv[kMaxLevels + 1];       // candidate slots per level: cap + c (padding children)
     size_t mu_off[kMaxLevels + 1];      // tree buffer offsets
     size_t bias_off[kMaxLevels + 1];
+    size_t sc_off[kMaxLevels + 1];      // MX-FP8 block scales (0 for the native format)
     size_t tree_bytes;
     // workspace
     size_t ws_cand[kMaxLevels + 1], ws_cmask[kMaxLevels + 1], ws_scores[kMaxLevels + 1],
@@ -43,6 +47,8 @@ struct Geo {
     size_t ws_bytes;
     __host__ __device__ int groups() const { return B * Hkv; }
     __host__ __device__ int esize() const { return dtype == ZHA_BF16 ? 2 : 4; }
+    __host__ __device__ bool mx() const { return summary == ZHA_SUMMARY_MXFP8; }
+    __host__ __device__ int mu_esize() const { return mx() ? 1 : esize(); }
 };
 
 // ----------------------------------------------------------------- device helpers

@@ -287,6 +287,357 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
     }
 }
 
+// bf16 scoring for R = 2^RL < 16 planes per node: the 16 rows of an MMA tile
+// are (candidate, plane) pairs, 16/R candidates per tile, so no row is idle.
+// Lane (gq, t) holds rows gq and gq + 8, i.e. planes of candidates gq >> RL
+// and (gq + 8) >> RL; a candidate's estimate is the max over its R rows,
+// reduced across the lanes that share it. Same coordinate permutation and
+// outputs as score_mma_kernel.
+template <int D, int NT, int RL, int U>
+__global__ void __launch_bounds__(kScoreWarps * 32)
+score_pack_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_bfloat16 *q,
+                  const int32_t *lens, LevelWs lw, LevelWs up, int level) {
+    constexpr int KP = D / 32;
+    constexpr int R = 1 << RL;
+    constexpr int CPT = 16 / R;          // candidates per tile
+    const int grp = blockIdx.y;
+    const int b = grp / g.Hkv, kvh = grp % g.Hkv;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gq = lane >> 2, t = lane & 3;
+    const int64_t cap = g.cap[level], capv = g.capv[level];
+    const CandSource src = cand_source(g, up, level, grp, group_len(g, lens, grp));
+    const int n = (int)cand_count(g, up, level, grp, src.n_here);
+    if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
+    const uint32_t all = all_heads(g.G);
+
+    uint32_t bq[NT][KP][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int h = nt * 8 + gq;
+#pragma unroll
+        for (int kp = 0; kp < KP; ++kp) {
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (h < g.G) w = ldg16(q + ((int64_t)b * g.Hq + kvh * g.G + h) * D + kp * 32 + t * 8);
+            bq[nt][kp][0] = w.x; bq[nt][kp][1] = w.y; bq[nt][kp][2] = w.z; bq[nt][kp][3] = w.w;
+        }
+    }
+    float runmax[NT][2], runmin[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        runmax[nt][0] = runmax[nt][1] = -INFINITY;
+        runmin[nt][0] = runmin[nt][1] = INFINITY;
+    }
+    const float s = g.s;
+    const int pa = gq & (R - 1), pb = (gq + 8) & (R - 1);   // planes of rows gq, gq + 8
+    const int ca = gq >> RL, cb = (gq + 8) >> RL;           // their candidates in the tile
+    const int stride = gridDim.x * kScoreWarps * U * CPT;
+    for (int i0 = (blockIdx.x * kScoreWarps + warp) * U * CPT; i0 < n; i0 += stride) {
+        int na[U], nb[U];
+        uint32_t ma[U], mb[U];
+        uint4 ra[U][KP], rb[U][KP];
+        float ba[U], bb[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int ia = i0 + u * CPT + ca, ib = i0 + u * CPT + cb;
+            na[u] = nb[u] = 0;
+            ma[u] = mb[u] = 0u;
+            if (ia < n) src.at(ia, na[u], ma[u], all);
+            if (ib < n) src.at(ib, nb[u], mb[u], all);
+            const __nv_bfloat16 *rowa = mu + ((grp * cap + na[u]) * (int64_t)R + pa) * D;
+            const __nv_bfloat16 *rowb = mu + ((grp * cap + nb[u]) * (int64_t)R + pb) * D;
+#pragma unroll
+            for (int kp = 0; kp < KP; ++kp) {
+                ra[u][kp] = ma[u] ? ldg16(rowa + kp * 32 + t * 8) : make_uint4(0, 0, 0, 0);
+                rb[u][kp] = mb[u] ? ldg16(rowb + kp * 32 + t * 8) : make_uint4(0, 0, 0, 0);
+            }
+            ba[u] = ma[u] ? __ldg(bias + (grp * cap + na[u]) * (int64_t)R + pa) : -INFINITY;
+            bb[u] = mb[u] ? __ldg(bias + (grp * cap + nb[u]) * (int64_t)R + pb) : -INFINITY;
+            // candidate bookkeeping: one lane per candidate of the tile
+            if (t == 0 && pa == 0 && ia < n) {
+                lw.cand[grp * capv + ia] = na[u];
+                lw.cmask[grp * capv + ia] = ma[u];
+            }
+            if (t == 0 && pb == 0 && ib < n) {
+                lw.cand[grp * capv + ib] = nb[u];
+                lw.cmask[grp * capv + ib] = mb[u];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (i0 + u * CPT >= n) break;
+            float acc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+            for (int kp = 0; kp < KP; ++kp) {
+                const uint4 &xa = ra[u][kp], &xb = rb[u][kp];
+                const uint32_t a0[4] = {xa.x, xb.x, xa.y, xb.y};
+                const uint32_t a1[4] = {xa.z, xb.z, xa.w, xb.w};
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma_bf16_16816(acc[nt], a0, bq[nt][kp][0], bq[nt][kp][1]);
+                    mma_bf16_16816(acc[nt], a1, bq[nt][kp][2], bq[nt][kp][3]);
+                }
+            }
+            float ea[NT][2], eb[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float va = fmaf(s, acc[nt][j], ba[u]);
+                    float vb = fmaf(s, acc[nt][2 + j], bb[u]);
+#pragma unroll
+                    for (int o = 4; o < 4 * R; o <<= 1) {       // max over the candidate's R rows
+                        va = fmaxf(va, __shfl_xor_sync(0xffffffffu, va, o));
+                        vb = fmaxf(vb, __shfl_xor_sync(0xffffffffu, vb, o));
+                    }
+                    ea[nt][j] = va;
+                    eb[nt][j] = vb;
+                }
+            if (pa == 0) {   // pb == 0 as well: 8 is a multiple of R
+                const int ia = i0 + u * CPT + ca, ib = i0 + u * CPT + cb;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int h = nt * 8 + 2 * t + j;
+                        if (h >= g.G) continue;
+                        if (ia < n) {
+                            const float e = ma[u] ? ea[nt][j] : -INFINITY;
+                            lw.scores[(grp * g.G + h) * capv + ia] = e;
+                            if ((ma[u] >> h) & 1u) {
+                                runmax[nt][j] = fmaxf(runmax[nt][j], e);
+                                runmin[nt][j] = fminf(runmin[nt][j], e);
+                            }
+                        }
+                        if (ib < n) {
+                            const float e = mb[u] ? eb[nt][j] : -INFINITY;
+                            lw.scores[(grp * g.G + h) * capv + ib] = e;
+                            if ((mb[u] >> h) & 1u) {
+                                runmax[nt][j] = fmaxf(runmax[nt][j], e);
+                                runmin[nt][j] = fminf(runmin[nt][j], e);
+                            }
+                        }
+                    }
+            }
+        }
+    }
+    // per-head max/min over the lanes that saw each head (columns 2t, 2t + 1)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            float mx = runmax[nt][j], mn = runmin[nt][j];
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            }
+            const int h = nt * 8 + 2 * t + j;
+            if (gq == 0 && h < g.G && mx > -INFINITY) {
+                atomicMax(&lw.maxkey[(int64_t)grp * g.G + h], ordered_key(mx));
+                atomicMin(&lw.minkey[(int64_t)grp * g.G + h], ordered_key(mn));
+            }
+        }
+}
+
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                              uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// two E4M3 bytes (low 16 bits of w) -> two fp16 (exact: E4M3 is a subset of fp16)
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t w) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// eight bf16 -> eight fp16 (four packed pairs), round to nearest
+__device__ __forceinline__ void bf16x8_f16x8(const uint4 &w, uint32_t (&o)[4]) {
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&in[j]));
+        const __half2 h = __float22half2_rn(f);
+        o[j] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+}
+
+// Scoring against MX-FP8 summaries (E4M3 bytes, one power-of-two scale per 32
+// coordinates of a plane). Same warp layout as score_mma_kernel: A = planes,
+// B = query heads, mma.sync m16n8k16 in fp16 (E4M3 converts to fp16 exactly;
+// the queries are rounded to fp16 once). Each lane reads 8 contiguous bytes of
+// a row per 32-coordinate block, so the two MMAs of a block see one scale per
+// row: they accumulate into a temporary that is scaled into the plane sums.
+template <int D, int MT, int NT, int U>
+__global__ void __launch_bounds__(kScoreWarps * 32)
+score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias, const __nv_bfloat16 *q,
+                 const int32_t *lens, LevelWs lw, LevelWs up, int level) {
+    constexpr int KP = D / 32;          // blocks per plane
+    const int grp = blockIdx.y;
+    const int b = grp / g.Hkv, kvh = grp % g.Hkv;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gq = lane >> 2, t = lane & 3;
+    const int64_t cap = g.cap[level], capv = g.capv[level];
+    const CandSource src = cand_source(g, up, level, grp, group_len(g, lens, grp));
+    const int n = (int)cand_count(g, up, level, grp, src.n_here);
+    if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
+    const uint32_t all = all_heads(g.G);
+
+    uint32_t bq[NT][KP][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int h = nt * 8 + gq;
+#pragma unroll
+        for (int kp = 0; kp < KP; ++kp) {
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (h < g.G) w = ldg16(q + ((int64_t)b * g.Hq + kvh * g.G + h) * D + kp * 32 + t * 8);
+            bf16x8_f16x8(w, bq[nt][kp]);
+        }
+    }
+    float runmax[NT][2], runmin[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        runmax[nt][0] = runmax[nt][1] = -INFINITY;
+        runmin[nt][0] = runmin[nt][1] = INFINITY;
+    }
+
+    const float s = g.s;
+    const int stride = gridDim.x * kScoreWarps * U;
+    for (int i0 = (blockIdx.x * kScoreWarps + warp) * U; i0 < n; i0 += stride) {
+        int node[U];
+        uint32_t hm[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u;
+            node[u] = 0;
+            hm[u] = 0u;
+            if (i < n) {
+                src.at(i, node[u], hm[u], all);
+                if (lane == 0) {
+                    lw.cand[grp * capv + i] = node[u];
+                    lw.cmask[grp * capv + i] = hm[u];
+                }
+            }
+        }
+        // all loads of the U candidates first: E4M3 rows, block scales, biases
+        uint2 ra[U][MT][KP], rb[U][MT][KP];
+        uint32_t sa[U][MT], sb[U][MT];
+        float ba[U][MT], bb[U][MT];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t rec = (grp * cap + node[u]) * (int64_t)g.R;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int r0 = mt * 16 + gq, r1 = r0 + 8;
+                const bool v0 = hm[u] && r0 < g.R, v1 = hm[u] && r1 < g.R;
+#pragma unroll
+                for (int kp = 0; kp < KP; ++kp) {
+                    ra[u][mt][kp] = v0 ? __ldg(reinterpret_cast<const uint2 *>(mu + (rec + r0) * D + kp * 32 + t * 8))
+                                       : make_uint2(0, 0);
+                    rb[u][mt][kp] = v1 ? __ldg(reinterpret_cast<const uint2 *>(mu + (rec + r1) * D + kp * 32 + t * 8))
+                                       : make_uint2(0, 0);
+                }
+                if constexpr (KP == 4) {
+                    sa[u][mt] = v0 ? __ldg(reinterpret_cast<const uint32_t *>(scl + (rec + r0) * KP)) : 0u;
+                    sb[u][mt] = v1 ? __ldg(reinterpret_cast<const uint32_t *>(scl + (rec + r1) * KP)) : 0u;
+                } else {
+                    sa[u][mt] = v0 ? __ldg(reinterpret_cast<const uint16_t *>(scl + (rec + r0) * KP)) : 0u;
+                    sb[u][mt] = v1 ? __ldg(reinterpret_cast<const uint16_t *>(scl + (rec + r1) * KP)) : 0u;
+                }
+                ba[u][mt] = v0 ? __ldg(bias + rec + r0) : -INFINITY;
+                bb[u][mt] = v1 ? __ldg(bias + rec + r1) : -INFINITY;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u;
+            if (i >= n) break;
+            if (hm[u] == 0u) {
+                if (lane < g.G) lw.scores[(grp * g.G + lane) * capv + i] = -INFINITY;
+                continue;
+            }
+            float e[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) e[nt][0] = e[nt][1] = -INFINITY;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                float acc[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+                for (int kp = 0; kp < KP; ++kp) {
+                    const uint2 &xa = ra[u][mt][kp], &xb = rb[u][mt][kp];
+                    const uint32_t a0[4] = {e4m3x2_f16x2(xa.x), e4m3x2_f16x2(xb.x), e4m3x2_f16x2(xa.x >> 16),
+                                            e4m3x2_f16x2(xb.x >> 16)};
+                    const uint32_t a1[4] = {e4m3x2_f16x2(xa.y), e4m3x2_f16x2(xb.y), e4m3x2_f16x2(xa.y >> 16),
+                                            e4m3x2_f16x2(xb.y >> 16)};
+                    // 2^(byte - 127) of this block for rows r0 and r1
+                    const float s0 = __uint_as_float(((sa[u][mt] >> (8 * kp)) & 0xffu) << 23);
+                    const float s1 = __uint_as_float(((sb[u][mt] >> (8 * kp)) & 0xffu) << 23);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_f16_16816(tmp, a0, bq[nt][kp][0], bq[nt][kp][1]);
+                        mma_f16_16816(tmp, a1, bq[nt][kp][2], bq[nt][kp][3]);
+                        acc[nt][0] = fmaf(s0, tmp[0], acc[nt][0]);
+                        acc[nt][1] = fmaf(s0, tmp[1], acc[nt][1]);
+                        acc[nt][2] = fmaf(s1, tmp[2], acc[nt][2]);
+                        acc[nt][3] = fmaf(s1, tmp[3], acc[nt][3]);
+                    }
+                }
+                const float b0 = ba[u][mt], b1 = bb[u][mt];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    e[nt][0] = fmaxf(e[nt][0], fmaxf(fmaf(s, acc[nt][0], b0), fmaf(s, acc[nt][2], b1)));
+                    e[nt][1] = fmaxf(e[nt][1], fmaxf(fmaf(s, acc[nt][1], b0), fmaf(s, acc[nt][3], b1)));
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float v = e[nt][j];
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                    e[nt][j] = v;
+                }
+            if (gq == 0) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int h = nt * 8 + 2 * t + j;
+                        if (h < g.G) {
+                            lw.scores[(grp * g.G + h) * capv + i] = e[nt][j];
+                            if ((hm[u] >> h) & 1u) {
+                                runmax[nt][j] = fmaxf(runmax[nt][j], e[nt][j]);
+                                runmin[nt][j] = fminf(runmin[nt][j], e[nt][j]);
+                            }
+                        }
+                    }
+            }
+        }
+    }
+    if (gq == 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int h = nt * 8 + 2 * t + j;
+                if (h < g.G && runmax[nt][j] > -INFINITY) {
+                    atomicMax(&lw.maxkey[(int64_t)grp * g.G + h], ordered_key(runmax[nt][j]));
+                    atomicMin(&lw.minkey[(int64_t)grp * g.G + h], ordered_key(runmin[nt][j]));
+                }
+            }
+    }
+}
+
 // fp32 scoring on CUDA cores: one block per candidate per iteration, one
 // thread per (plane, head) dot product.
 template <int D>
@@ -403,12 +754,16 @@ __device__ __forceinline__ V block_exclusive_scan(V v, V *red, V *total) {
     return before + x - v;
 }
 
+// masses below e^-23 of the maximum round to 0 in 2^-31 fixed point
+constexpr float kMassRange = 23.f;
+
 struct SelShared {
     uint32_t hist_lo[kBuckets];
     uint32_t hist_hi[kBuckets];
     unsigned long long red[kSelThreads / 32];
     int32_t ties[kMaxTies];
     int32_t sorted_ties[kMaxTies];
+    uint32_t tkey[kMaxTies];
     unsigned long long above, target;
     uint32_t digit, kmax, kmin;
     int ntie;
@@ -468,6 +823,112 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
         return (int)block_sum<unsigned long long>((unsigned long long)kept, sh.red);
     }
     const float m = key_to_float(kmax);
+    // Common case, two passes: a histogram of the masses over the score's
+    // distance below the max, in kBuckets equal steps of at most kMassRange
+    // nats (monotone in the score, so the buckets are contiguous in the
+    // (score desc) order), finds the bucket where the running mass crosses
+    // p; the members of that bucket are then ordered exactly by (score desc,
+    // index asc) in shared memory. If that bucket holds more than kMaxTies
+    // members (near-equal scores), the radix search below decides instead.
+    {
+        const float span = m - key_to_float(kmin);
+        const float W = (float)kBuckets / fminf(span, kMassRange);
+        if (kmax != kmin && W < 1e30f) {
+            auto bucket = [&](float e) -> int {
+                const float x = (m - e) * W;
+                return x < (float)(kBuckets - 1) ? (int)x : kBuckets - 1;
+            };
+            for (int i = tid; i < kBuckets; i += blockDim.x) sh.hist_lo[i] = sh.hist_hi[i] = 0u;
+            if (tid == 0) {
+                sh.above = 0ull;
+                sh.ntie = 0;
+            }
+            __syncthreads();
+            auto add_block = [&](uint32_t mb, const float (&e)[8]) {
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                    if ((mb >> v) & 1u) hist_add(sh.hist_lo, sh.hist_hi, bucket(e[v]), fixed_mass(e[v], m));
+            };
+            for (int64_t blk = tid; blk < nblk; blk += 2 * step) {
+                float e0[8], e1[8];
+                const uint32_t m0 = load8(blk, e0);
+                const uint32_t m1 = blk + step < nblk ? load8(blk + step, e1) : 0u;
+                add_block(m0, e0);
+                add_block(m1, e1);
+            }
+            __syncthreads();
+            constexpr int per = kBuckets / kSelThreads;
+            unsigned long long mine = 0ull;
+#pragma unroll
+            for (int j = 0; j < per; ++j)
+                mine += ((unsigned long long)sh.hist_hi[tid * per + j] << 32) | sh.hist_lo[tid * per + j];
+            unsigned long long z;
+            const unsigned long long excl = block_exclusive_scan<unsigned long long>(mine, sh.red, &z);
+            const unsigned long long target = (unsigned long long)ceil((double)p * (double)z);
+            unsigned long long run = excl;
+#pragma unroll
+            for (int j = 0; j < per; ++j) {
+                const int bk = tid * per + j;
+                const unsigned long long hgt = ((unsigned long long)sh.hist_hi[bk] << 32) | sh.hist_lo[bk];
+                if (hgt && run < target && run + hgt >= target) {
+                    sh.digit = (uint32_t)bk;
+                    sh.above = run;
+                }
+                run += hgt;
+            }
+            __syncthreads();
+            const int bstar = (int)sh.digit;
+            const unsigned long long above = sh.above;
+            for (int64_t blk = tid; blk < nblk; blk += step) {
+                float e[8];
+                const uint32_t mb = load8(blk, e);
+                uint32_t kb = 0u;
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    if (!((mb >> v) & 1u)) continue;
+                    const int bk = bucket(e[v]);
+                    if (bk < bstar) {
+                        kb |= 1u << v;
+                    } else if (bk == bstar) {
+                        const int slot = atomicAdd(&sh.ntie, 1);
+                        if (slot < kMaxTies) {
+                            sh.ties[slot] = (int32_t)((blk << 3) + v);
+                            sh.tkey[slot] = ordered_key(e[v]);
+                        }
+                    }
+                }
+                store8(blk, kb);
+                kept += __popc(kb);
+            }
+            __syncthreads();
+            const int nl = sh.ntie;
+            if (nl <= kMaxTies) {
+                for (int j = tid; j < nl; j += blockDim.x) {
+                    const uint32_t kj = sh.tkey[j];
+                    const int32_t ij = sh.ties[j];
+                    int rank = 0;
+                    for (int w = 0; w < nl; ++w) {
+                        const uint32_t kw = sh.tkey[w];
+                        rank += (kw > kj) || (kw == kj && sh.ties[w] < ij);
+                    }
+                    sh.sorted_ties[rank] = j;
+                }
+                __syncthreads();
+                if (tid == 0) {
+                    unsigned long long cum = above;
+                    for (int r = 0; r < nl && cum < target; ++r) {
+                        const int j = sh.sorted_ties[r];
+                        add_kept(sh.ties[j]);
+                        ++kept;
+                        cum += fixed_mass(key_to_float(sh.tkey[j]), m);
+                    }
+                }
+                return (int)block_sum<unsigned long long>((unsigned long long)kept, sh.red);
+            }
+            kept = 0;   // too many near-equal scores: the radix search rewrites every block
+            __syncthreads();
+        }
+    }
     // u = kmax - key: 0 for the best candidate, growing as the score falls.
     const uint32_t span = kmax - kmin;
     int hi = span ? 32 - __clz(span) : 0;  // bits of u that can be non-zero
@@ -758,11 +1219,55 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
         const int64_t capv = g.capv[level];
         {
             ProfScope ps(score_names[level], st);
-            if (g.dtype == ZHA_BF16 && (g.flags & ZHA_FLAG_TCGEN05) && score_tc_supported(g)) {
+            if (g.mx()) {
+                const auto *mu = reinterpret_cast<const uint8_t *>(tb + g.mu_off[level]);
+                const auto *scl = reinterpret_cast<const uint8_t *>(tb + g.sc_off[level]);
+                const auto *bias = reinterpret_cast<const float *>(tb + g.bias_off[level]);
+                const auto *qq = static_cast<const __nv_bfloat16 *>(q);
+                const int64_t want = (capv + kScoreWarps - 1) / kScoreWarps;
+                const int per_group = (int)max64(1, min64(want, (148 * 8 + groups - 1) / groups));
+                dim3 grid(per_group, groups);
+                const int mt = g.R > 16 ? 2 : 1, nt = g.G > 8 ? 2 : 1;
+#define ZHA_SCORE_MX(D, MT, NT, U) \
+    score_mx8_kernel<D, MT, NT, U><<<grid, kScoreWarps * 32, 0, st>>>(g, mu, scl, bias, qq, lens, lw, up, level)
+                if (g.d == 128) {
+                    if (mt == 1 && nt == 1) ZHA_SCORE_MX(128, 1, 1, 4);
+                    else if (mt == 1) ZHA_SCORE_MX(128, 1, 2, 2);
+                    else if (nt == 1) ZHA_SCORE_MX(128, 2, 1, 2);
+                    else ZHA_SCORE_MX(128, 2, 2, 2);
+                } else {
+                    if (mt == 1 && nt == 1) ZHA_SCORE_MX(64, 1, 1, 4);
+                    else if (mt == 1) ZHA_SCORE_MX(64, 1, 2, 4);
+                    else if (nt == 1) ZHA_SCORE_MX(64, 2, 1, 2);
+                    else ZHA_SCORE_MX(64, 2, 2, 2);
+                }
+#undef ZHA_SCORE_MX
+            } else if (g.dtype == ZHA_BF16 && (g.flags & ZHA_FLAG_TCGEN05) && score_tc_supported(g)) {
                 e = launch_score_tc(g, tb + g.mu_off[level], reinterpret_cast<const float *>(tb + g.bias_off[level]),
                                     q, lens, level, lw.cand, lw.cmask, lw.scores, lw.count, lw.maxkey, lw.minkey,
                                     up.plist, up.pmask, up.pcount, status, st);
                 if (e != cudaSuccess) return e;
+            } else if (g.dtype == ZHA_BF16 && g.R < 16 && (g.R & (g.R - 1)) == 0) {
+                const auto *mu = reinterpret_cast<const __nv_bfloat16 *>(tb + g.mu_off[level]);
+                const auto *bias = reinterpret_cast<const float *>(tb + g.bias_off[level]);
+                const auto *qq = static_cast<const __nv_bfloat16 *>(q);
+                const int cpt = 16 / g.R;
+                const int64_t want = (capv + kScoreWarps * cpt - 1) / (kScoreWarps * cpt);
+                const int per_group = (int)max64(1, min64(want, (148 * 8 + groups - 1) / groups));
+                dim3 grid(per_group, groups);
+                const int rl = __builtin_ctz(g.R);
+#define ZHA_SCORE_PACK(D, NT, RL) \
+    score_pack_kernel<D, NT, RL, 2><<<grid, kScoreWarps * 32, 0, st>>>(g, mu, bias, qq, lens, lw, up, level)
+#define ZHA_SCORE_PACK_R(D, NT) \
+    do { if (rl == 0) ZHA_SCORE_PACK(D, NT, 0); else if (rl == 1) ZHA_SCORE_PACK(D, NT, 1); \
+         else if (rl == 2) ZHA_SCORE_PACK(D, NT, 2); else ZHA_SCORE_PACK(D, NT, 3); } while (0)
+                if (g.d == 128) {
+                    if (g.G > 8) ZHA_SCORE_PACK_R(128, 2); else ZHA_SCORE_PACK_R(128, 1);
+                } else {
+                    if (g.G > 8) ZHA_SCORE_PACK_R(64, 2); else ZHA_SCORE_PACK_R(64, 1);
+                }
+#undef ZHA_SCORE_PACK_R
+#undef ZHA_SCORE_PACK
             } else if (g.dtype == ZHA_BF16) {
                 const auto *mu = reinterpret_cast<const __nv_bfloat16 *>(tb + g.mu_off[level]);
                 const auto *bias = reinterpret_cast<const float *>(tb + g.bias_off[level]);

@@ -479,7 +479,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }  // namespace
 
 bool score_tc_supported(const Geo &g) {
-    return g.dtype == ZHA_BF16 && g.d == 128 && g.R == 16 && g.G <= 16 && g.groups() <= kMaxGroups &&
+    return g.dtype == ZHA_BF16 && !g.mx() && g.d == 128 && g.R == 16 && g.G <= 16 && g.groups() <= kMaxGroups &&
            encode_fn() != nullptr;
 }
 

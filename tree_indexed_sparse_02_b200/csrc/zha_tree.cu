@@ -24,17 +24,50 @@ namespace {
 
 constexpr int kLevelWarps = 8;
 
+// Points of one plane computation, d coordinates each, lane owning EPL of them.
 template <typename T, int EPL>
-__device__ __forceinline__ void warp_plane(const T *x0, int64_t xstride, const float *a0,
-                                           int64_t astride, int npts, const float (&rv)[EPL],
-                                           float s, T *mu_out, float *b_out, int lane) {
+struct RawPoints {        // keys of a leaf chunk, or children kept in the KV dtype
+    const T *x0;
+    int64_t stride;
+    __device__ __forceinline__ void load(int i, int lane, float (&x)[EPL]) const {
+        load_vec<EPL>(x0 + (int64_t)i * stride + lane * EPL, x);
+    }
+};
+
+// 2^(byte - 127) for a biased scale exponent byte in 1..254
+__device__ __forceinline__ float mx_scale(uint8_t byte) { return __uint_as_float((uint32_t)byte << 23); }
+
+template <int EPL>
+struct Mx8Points {        // children kept as MX-FP8 (E4M3 bytes + one scale per 32)
+    const uint8_t *x0;
+    const uint8_t *s0;
+    int64_t stride, sstride;
+    __device__ __forceinline__ void load(int i, int lane, float (&x)[EPL]) const {
+        const float sc = mx_scale(s0[(int64_t)i * sstride + (lane * EPL) / 32]);
+        const uint8_t *p = x0 + (int64_t)i * stride + lane * EPL;
+#pragma unroll
+        for (int e = 0; e < EPL; e += 2) {
+            const __nv_fp8x2_storage_t two = *reinterpret_cast<const __nv_fp8x2_storage_t *>(p + e);
+            const __half2 h = __half2(__nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3));
+            const float2 f = __half22float2(h);
+            x[e] = f.x * sc;
+            x[e + 1] = f.y * sc;
+        }
+    }
+};
+
+// mu_out/b_out of one plane from its points (online single pass; see top).
+template <class P, int EPL>
+__device__ __forceinline__ void warp_plane(const P &pts, const float *a0, int64_t astride, int npts,
+                                           const float (&rv)[EPL], float s, float (&acc)[EPL],
+                                           float &b_out) {
     float m = -INFINITY, sum = 0.f, wl = 0.f;
-    float acc[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+    const int lane = threadIdx.x & 31;
     for (int i = 0; i < npts; ++i) {
         float x[EPL];
-        load_vec<EPL>(x0 + (int64_t)i * xstride + lane * EPL, x);
+        pts.load(i, lane, x);
         float part = 0.f;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) part = fmaf(rv[e], x[e], part);
@@ -58,37 +91,83 @@ __device__ __forceinline__ void warp_plane(const T *x0, int64_t xstride, const f
     const float inv = 1.f / sum;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) acc[e] *= inv;
-    store_vec<EPL>(mu_out + lane * EPL, acc);
-    if (lane == 0) *b_out = (m + logf(sum)) - wl * inv;
+    b_out = (m + logf(sum)) - wl * inv;
+}
+
+// MX-FP8 store of one plane: the lanes sharing a 32-coordinate block agree on
+// its scale exponent e (smallest with max|x| <= 448 * 2^e) and round x / 2^e
+// to E4M3, nearest even.
+template <int EPL>
+__device__ __forceinline__ void mx_store(uint8_t *mu_out, uint8_t *sc_out, const float (&v)[EPL], int lane) {
+    constexpr int kLanesPerBlock = 32 / EPL;
+    float a = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) a = fmaxf(a, fabsf(v[e]));
+#pragma unroll
+    for (int o = 1; o < kLanesPerBlock; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    int ex = 0;
+    if (a > 0.f) {
+        int k;
+        const float f = frexpf(a, &k);                 // a = f 2^k, 448 = 0.875 2^9
+        ex = (f <= 0.875f) ? k - 9 : k - 8;
+        ex = ex < -126 ? -126 : (ex > 127 ? 127 : ex);
+    }
+    uint32_t packed = 0;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+        const __nv_fp8_storage_t q = __nv_cvt_float_to_fp8(scalbnf(v[e], -ex), __NV_SATFINITE, __NV_E4M3);
+        packed |= (uint32_t)q << (8 * e);
+    }
+    if constexpr (EPL == 4)
+        *reinterpret_cast<uint32_t *>(mu_out + lane * 4) = packed;
+    else
+        *reinterpret_cast<uint16_t *>(mu_out + lane * 2) = (uint16_t)packed;
+    if (lane % kLanesPerBlock == 0) sc_out[lane / kLanesPerBlock] = (uint8_t)(ex + 127);
 }
 
 struct TreePtrs {
     void *mu[kMaxLevels + 1];
+    uint8_t *sc[kMaxLevels + 1];
     float *bias[kMaxLevels + 1];
 };
 
-// Plane r of node `node` at `level` of group `grp`.
-template <typename T, int EPL>
+// Plane r of node `node` at `level` of group `grp`; MX selects the summary format.
+template <typename T, int EPL, bool MX>
 __device__ __forceinline__ void node_plane(const Geo &g, const TreePtrs &tp, const T *K,
                                            const T *refs, int grp, int level, int64_t node,
                                            int64_t n_below, int r, int lane) {
     const int kvh = grp % g.Hkv;
     float rv[EPL];
     load_vec<EPL>(refs + ((int64_t)kvh * g.R + r) * g.d + lane * EPL, rv);
-    T *mu = reinterpret_cast<T *>(tp.mu[level]) + ((grp * g.cap[level] + node) * g.R + r) * g.d;
-    float *bias = tp.bias[level] + (grp * g.cap[level] + node) * g.R + r;
+    const int64_t rec = (grp * g.cap[level] + node) * g.R + r;      // plane record index
+    float *bias = tp.bias[level] + rec;
+    float acc[EPL];
+    float bval;
     if (level == 1) {
-        const T *x0 = K + ((int64_t)grp * g.max_len + node * g.c) * g.d;
-        warp_plane<T, EPL>(x0, g.d, nullptr, 0, g.c, rv, g.s, mu, bias, lane);
+        const RawPoints<T, EPL> pts{K + ((int64_t)grp * g.max_len + node * g.c) * g.d, g.d};
+        warp_plane(pts, nullptr, 0, g.c, rv, g.s, acc, bval);
     } else {
         const int64_t c0 = node * g.c;
         const int64_t c1 = min(c0 + g.c, n_below);
-        const T *x0 = reinterpret_cast<const T *>(tp.mu[level - 1]) +
-                      ((grp * g.cap[level - 1] + c0) * g.R + r) * g.d;
-        const float *a0 = tp.bias[level - 1] + (grp * g.cap[level - 1] + c0) * g.R + r;
-        warp_plane<T, EPL>(x0, (int64_t)g.R * g.d, a0, g.R, (int)(c1 - c0), rv, g.s, mu, bias,
-                           lane);
+        const int64_t crec = (grp * g.cap[level - 1] + c0) * g.R + r;
+        const float *a0 = tp.bias[level - 1] + crec;
+        if constexpr (MX) {
+            const Mx8Points<EPL> pts{static_cast<const uint8_t *>(tp.mu[level - 1]) + crec * g.d,
+                                     tp.sc[level - 1] + crec * (g.d / 32), (int64_t)g.R * g.d,
+                                     (int64_t)g.R * (g.d / 32)};
+            warp_plane(pts, a0, g.R, (int)(c1 - c0), rv, g.s, acc, bval);
+        } else {
+            const RawPoints<T, EPL> pts{static_cast<const T *>(tp.mu[level - 1]) + crec * g.d,
+                                        (int64_t)g.R * g.d};
+            warp_plane(pts, a0, g.R, (int)(c1 - c0), rv, g.s, acc, bval);
+        }
     }
+    if constexpr (MX)
+        mx_store<EPL>(static_cast<uint8_t *>(tp.mu[level]) + rec * g.d, tp.sc[level] + rec * (g.d / 32), acc,
+                      lane);
+    else
+        store_vec<EPL>(static_cast<T *>(tp.mu[level]) + rec * g.d + lane * EPL, acc);
+    if (lane == 0) *bias = bval;
 }
 
 // Tokens before/after the update of sequence b; false if nothing changes.
@@ -104,7 +183,7 @@ __device__ __forceinline__ bool update_range(const Geo &g, const int32_t *lens, 
 }
 
 // One level, many nodes: grid.x covers node slots x references, grid.y groups.
-template <typename T, int EPL>
+template <typename T, int EPL, bool MX>
 __global__ void __launch_bounds__(kLevelWarps * 32)
 tree_level_kernel(Geo g, TreePtrs tp, const T *K, const T *refs, const int32_t *lens, int level,
                   int n_new, int64_t slots, int32_t *status) {
@@ -121,13 +200,13 @@ tree_level_kernel(Geo g, TreePtrs tp, const T *K, const T *refs, const int32_t *
     const int r = (int)(item % g.R);
     if (node >= level_nodes(n_now, g.c, level)) return;
     const int64_t n_below = level > 1 ? level_nodes(n_now, g.c, level - 1) : 0;
-    node_plane<T, EPL>(g, tp, K, refs, grp, level, node, n_below, r, lane);
+    node_plane<T, EPL, MX>(g, tp, K, refs, grp, level, node, n_below, r, lane);
 }
 
 // Few new tokens (a decode step): one block per group walks every level,
 // warp r computing plane r of each changed node; levels are separated by a
 // block barrier, which also makes the children's global writes visible.
-template <typename T, int EPL>
+template <typename T, int EPL, bool MX>
 __global__ void tree_path_kernel(Geo g, TreePtrs tp, const T *K, const T *refs,
                                  const int32_t *lens, int n_new, int32_t *status) {
     const int grp = blockIdx.x;
@@ -144,19 +223,19 @@ __global__ void tree_path_kernel(Geo g, TreePtrs tp, const T *K, const T *refs,
         const int64_t n_below = level > 1 ? level_nodes(n_now, g.c, level - 1) : 0;
         const int64_t items = (hi - lo) * g.R;
         for (int64_t it = warp; it < items; it += blockDim.x >> 5)
-            node_plane<T, EPL>(g, tp, K, refs, grp, level, lo + it / g.R, n_below,
-                               (int)(it % g.R), lane);
+            node_plane<T, EPL, MX>(g, tp, K, refs, grp, level, lo + it / g.R, n_below,
+                                   (int)(it % g.R), lane);
         __syncthreads();
     }
 }
 
-template <typename T, int EPL>
+template <typename T, int EPL, bool MX>
 cudaError_t tree_update_t(const Geo &g, const TreePtrs &tp, const T *K, const T *refs,
                           const int32_t *lens, int n_new, int32_t *status, cudaStream_t st) {
     if (n_new >= 0 && n_new <= g.c) {
         const int warps = g.R < 4 ? 4 : g.R;
         ProfScope ps("tree_path", st);
-        tree_path_kernel<T, EPL><<<g.groups(), warps * 32, 0, st>>>(g, tp, K, refs, lens, n_new,
+        tree_path_kernel<T, EPL, MX><<<g.groups(), warps * 32, 0, st>>>(g, tp, K, refs, lens, n_new,
                                                                     status);
         return cudaGetLastError();
     }
@@ -172,7 +251,7 @@ cudaError_t tree_update_t(const Geo &g, const TreePtrs &tp, const T *K, const T 
                                           "tree_level[l4]", "tree_level[l5]", "tree_level[l6]",
                                           "tree_level[l7]", "tree_level[l8]"};
             ProfScope ps(names[level], st);
-            tree_level_kernel<T, EPL><<<grid, kLevelWarps * 32, 0, st>>>(g, tp, K, refs, lens, level,
+            tree_level_kernel<T, EPL, MX><<<grid, kLevelWarps * 32, 0, st>>>(g, tp, K, refs, lens, level,
                                                                          n_new, bound, status);
         }
         cudaError_t e = cudaGetLastError();
@@ -189,17 +268,21 @@ cudaError_t launch_tree_update(const Geo &g, void *tree, const void *K, const vo
     for (int l = 1; l <= g.L; ++l) {
         tp.mu[l] = static_cast<char *>(tree) + g.mu_off[l];
         tp.bias[l] = reinterpret_cast<float *>(static_cast<char *>(tree) + g.bias_off[l]);
+        tp.sc[l] = g.mx() ? reinterpret_cast<uint8_t *>(static_cast<char *>(tree) + g.sc_off[l]) : nullptr;
     }
     if (g.dtype == ZHA_BF16) {
         auto k = static_cast<const __nv_bfloat16 *>(K);
         auto r = static_cast<const __nv_bfloat16 *>(refs);
-        return g.d == 128 ? tree_update_t<__nv_bfloat16, 4>(g, tp, k, r, lens, n_new, status, st)
-                          : tree_update_t<__nv_bfloat16, 2>(g, tp, k, r, lens, n_new, status, st);
+        if (g.mx())
+            return g.d == 128 ? tree_update_t<__nv_bfloat16, 4, true>(g, tp, k, r, lens, n_new, status, st)
+                              : tree_update_t<__nv_bfloat16, 2, true>(g, tp, k, r, lens, n_new, status, st);
+        return g.d == 128 ? tree_update_t<__nv_bfloat16, 4, false>(g, tp, k, r, lens, n_new, status, st)
+                          : tree_update_t<__nv_bfloat16, 2, false>(g, tp, k, r, lens, n_new, status, st);
     }
     auto k = static_cast<const float *>(K);
     auto r = static_cast<const float *>(refs);
-    return g.d == 128 ? tree_update_t<float, 4>(g, tp, k, r, lens, n_new, status, st)
-                      : tree_update_t<float, 2>(g, tp, k, r, lens, n_new, status, st);
+    return g.d == 128 ? tree_update_t<float, 4, false>(g, tp, k, r, lens, n_new, status, st)
+                      : tree_update_t<float, 2, false>(g, tp, k, r, lens, n_new, status, st);
 }
 
 // Decode step prologue: write the new token of every (sequence, KV head) at

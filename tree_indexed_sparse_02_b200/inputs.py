@@ -48,6 +48,7 @@ class Workload:
     diffuse_nodes: int = 0
     refs_mode: str = "random"
     p_schedule: str = "fixed"   # "fixed": p per level; "root": p^(1/L) per level
+    summary: str = "native"     # "native": mu in the KV dtype; "mxfp8": E4M3 blocks of 32 + scales
 
     @property
     def group(self) -> int:

@@ -19,6 +19,7 @@ ZHA_BF16, ZHA_F32 = 0, 1
 ZHA_FLAG_TAIL_ONLY = 1
 ZHA_FLAG_TCGEN05 = 2
 ZHA_P_FIXED, ZHA_P_DEPTH_ROOT = 0, 1
+ZHA_SUMMARY_NATIVE, ZHA_SUMMARY_MXFP8 = 0, 1
 ZHA_MAX_LEVELS = 8
 STATUS_NAMES = {0: "ZHA_OK", 1: "ZHA_ERR_INVALID_ARG", 2: "ZHA_ERR_UNSUPPORTED",
                 3: "ZHA_ERR_CAPACITY", 4: "ZHA_ERR_CUDA", 5: "ZHA_ERR_TIMEOUT"}
@@ -35,7 +36,7 @@ class Config(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("chunk", ctypes.c_int32), ("levels", ctypes.c_int32),
                 ("n_refs", ctypes.c_int32), ("dtype", ctypes.c_int32), ("max_len", ctypes.c_int64),
                 ("scale", ctypes.c_float), ("flags", ctypes.c_int32), ("attn_splits", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 3)]
+                ("summary", ctypes.c_int32), ("reserved", ctypes.c_int32 * 2)]
 
     @property
     def group(self) -> int:
@@ -69,6 +70,7 @@ def _load():
         "zha_level_nodes": ([CP, i64, i32], i64),
         "zha_tree_bytes": ([CP], sz),
         "zha_tree_level_offsets": ([CP, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)], i32),
+        "zha_tree_level_scales": ([CP, i32, ctypes.POINTER(sz)], i32),
         "zha_workspace_bytes": ([CP], sz),
         "zha_workspace_level_view": ([CP, i32, ctypes.POINTER(LevelView)], i32),
         "zha_tree_build": ([CP, P, P, P, P, P, P], i32),
@@ -99,10 +101,11 @@ def lib():
 
 
 def config(batch, n_q_heads, n_kv_heads, head_dim, chunk, levels, n_refs, dtype="bf16", max_len=4096,
-           scale=0.0, flags=0, attn_splits=0) -> Config:
+           scale=0.0, flags=0, attn_splits=0, summary="native") -> Config:
     dt = {"bf16": ZHA_BF16, "f32": ZHA_F32}.get(dtype, dtype)
+    sm = {"native": ZHA_SUMMARY_NATIVE, "mxfp8": ZHA_SUMMARY_MXFP8}.get(summary, summary)
     c = Config(batch, n_q_heads, n_kv_heads, head_dim, chunk, levels, n_refs, dt, max_len, scale, flags,
-               attn_splits)
+               attn_splits, sm)
     check(_lib.zha_check_config(ctypes.byref(c)), "zha_check_config")
     return c
 
@@ -290,16 +293,31 @@ class Buffers:
 
     # views of the tree buffer (for inspection and tests)
     def tree_level(self, level: int):
+        """(mu, bias) views of one level; with MX-FP8 summaries mu is the E4M3
+        byte array and tree_level_scales() gives the block scales."""
         cfg = self.cfg
         mu_off, b_off = tree_level_offsets(cfg, level)
         cap = level_nodes(cfg, cfg.max_len, level)
-        es = 2 if cfg.dtype == ZHA_BF16 else 4
+        shape = (cfg.batch, cfg.n_kv_heads, cap, cfg.n_refs, cfg.head_dim)
         n_mu = cfg.batch * cfg.n_kv_heads * cap * cfg.n_refs * cfg.head_dim
-        mu = self.tree[mu_off:mu_off + n_mu * es].view(cfg.torch_dtype).view(
-            cfg.batch, cfg.n_kv_heads, cap, cfg.n_refs, cfg.head_dim)
+        if cfg.summary == ZHA_SUMMARY_MXFP8:
+            mu = self.tree[mu_off:mu_off + n_mu].view(*shape)
+        else:
+            es = 2 if cfg.dtype == ZHA_BF16 else 4
+            mu = self.tree[mu_off:mu_off + n_mu * es].view(cfg.torch_dtype).view(*shape)
         n_b = cfg.batch * cfg.n_kv_heads * cap * cfg.n_refs
         bias = self.tree[b_off:b_off + n_b * 4].view(torch.float32).view(cfg.batch, cfg.n_kv_heads, cap, cfg.n_refs)
         return mu, bias
+
+    def tree_level_scales(self, level: int):
+        """Block-scale bytes [B, Hkv, cap, R, d/32] of an MX-FP8 level (2^(byte-127))."""
+        cfg = self.cfg
+        off = ctypes.c_size_t()
+        check(_lib.zha_tree_level_scales(ctypes.byref(cfg), level, ctypes.byref(off)), "zha_tree_level_scales")
+        cap = level_nodes(cfg, cfg.max_len, level)
+        n = cfg.batch * cfg.n_kv_heads * cap * cfg.n_refs * (cfg.head_dim // 32)
+        return self.tree[off.value:off.value + n].view(cfg.batch, cfg.n_kv_heads, cap, cfg.n_refs,
+                                                        cfg.head_dim // 32)
 
     def level_state(self, level: int):
         """Routing state of one level from the last route/decode call."""
