@@ -290,3 +290,46 @@ def decode_group(tree: Tree, q: np.ndarray, K: np.ndarray, V: np.ndarray, p, tai
         masks[h] = token_set(N, tree.c, kept_leaf, tail_only)
         outs[h] = attend(q[h], K, V, N, tree.s, masks[h])
     return outs, r, masks
+
+
+# ----------------------------------------------------------- multi-query blocks
+#
+# T consecutive query positions of one sequence at once (a multi-query decode
+# or a chunked-prefill block). The pages describe routing for one decoding
+# query ("How does top-p routing pick tokens"); the reading taken for a block:
+# every query routes over the tree of the N0 tokens cached before the block,
+# and query t attends {0} U its kept leaf chunks U [c*floor(N0/c), N0 + t],
+# i.e. the cached tail after the tree's last complete chunk and the block's
+# own tokens up to its position (causal).
+
+
+def block_token_set(N0: int, t: int, c: int, kept_leaf: np.ndarray) -> np.ndarray:
+    """Tokens query t of a block attends -> bool[N0 + t + 1]."""
+    n = N0 + t + 1
+    m = np.zeros(n, dtype=bool)
+    m[0] = True
+    for j in np.nonzero(np.asarray(kept_leaf, dtype=bool))[0]:
+        m[j * c:(j + 1) * c] = True
+    m[c * (N0 // c):n] = True
+    return m
+
+
+def decode_block_group(tree: Tree, q: np.ndarray, K: np.ndarray, V: np.ndarray, p):
+    """One group's block: q [T, G, d], K/V hold at least tree.N + T tokens.
+
+    Returns (out [T, G, d], route over the T*G rows (row t*G + h), token masks
+    per row [T*G] of bool arrays)."""
+    q = _f64(q)
+    T, G, d = q.shape
+    N0 = tree.N
+    r = route(tree, q.reshape(T * G, d), p)
+    out = np.zeros((T, G, d))
+    masks = []
+    for t in range(T):
+        for h in range(G):
+            row = t * G + h
+            kept_leaf = r.kept[0][row] if tree.n(1) > 0 else np.zeros(0, dtype=bool)
+            m = block_token_set(N0, t, tree.c, kept_leaf)
+            masks.append(m)
+            out[t, h] = attend(q[t, h], K, V, N0 + t + 1, tree.s, m)
+    return out, r, masks

@@ -510,3 +510,63 @@ def test_mxfp8_storage_tree_builds_from_rounded_children(orc):
             bound = np.max(s * dmu @ np.abs(q) + np.abs(t.b[level][n] - ref.b[level][n]))
             assert abs(e_mx - e_64) <= bound + 1e-12
             assert abs(e_mx - e_64) < 0.1
+
+
+# ------------------------------------------------------------ multi-query blocks
+
+
+def test_block_p1_rows_equal_causal_dense(orc):
+    """p = 1: every row of a block attends its whole causal prefix [0, N0 + t]."""
+    N0, T, d, c, L, R, G = 517, 5, 16, 4, 3, 4, 2
+    K, V, refs, _ = _group(100, N0 + T, d, c, L, R, G)
+    q = rng(101).normal(size=(T, G, d))
+    t = orc.build_tree(K, refs, N0, c, L)
+    out, r, masks = orc.decode_block_group(t, q, K, V, 1.0)
+    for tt in range(T):
+        n = N0 + tt + 1
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[tt])[None, :, None, :], torch.from_numpy(K[:n])[None, None].expand(1, G, n, d),
+            torch.from_numpy(V[:n])[None, None].expand(1, G, n, d), scale=t.s)[0, :, 0]
+        assert np.allclose(out[tt], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_block_single_query_equals_decode_when_no_chunk_completes(orc):
+    """T = 1 and N0 + 1 not a multiple of c: the tree before and after the token
+    is the same, and the block's token rule is the decode rule."""
+    d, c, L, R, G = 16, 4, 3, 4, 3
+    for N0 in (401, 402, 1000, 4):
+        K, V, refs, _ = _group(102 + N0, N0 + 1, d, c, L, R, G)
+        q = rng(103).normal(size=(1, G, d))
+        t = orc.build_tree(K, refs, N0, c, L)
+        for p in (0.6, 0.95):
+            ob, rb, mb = orc.decode_block_group(t, q, K, V, p)
+            t1 = orc.build_tree(K, refs, N0 + 1, c, L)
+            od, rd, md = orc.decode_group(t1, q[0], K, V, p)
+            assert np.array_equal(np.stack(mb), md)
+            assert np.allclose(ob[0], od, rtol=1e-12, atol=1e-12)
+
+
+def test_block_rows_are_causal(orc):
+    """A row's output does not depend on the block's later tokens; its token set
+    is the sink, its kept leaves and [c*floor(N0/c), N0 + t]."""
+    N0, T, d, c, L, R, G = 389, 6, 16, 8, 2, 4, 2
+    K, V, refs, _ = _group(104, N0 + T, d, c, L, R, G)
+    q = rng(105).normal(size=(T, G, d))
+    t = orc.build_tree(K, refs, N0, c, L)
+    out, r, masks = orc.decode_block_group(t, q, K, V, 0.8)
+    K2, V2 = K.copy(), V.copy()
+    K2[N0 + 2:] += 5.0
+    V2[N0 + 2:] -= 3.0
+    out2, _, _ = orc.decode_block_group(t, q, K2, V2, 0.8)
+    assert np.array_equal(out[:2], out2[:2]) and not np.allclose(out[2:], out2[2:])
+    for tt in range(T):
+        for h in range(G):
+            m = masks[tt * G + h]
+            assert m.shape == (N0 + tt + 1,) and m[0] and m[c * (N0 // c):].all()
+            kept = np.nonzero(r.kept[0][tt * G + h])[0]
+            want = np.zeros_like(m)
+            want[0] = True
+            for j in kept:
+                want[j * c:(j + 1) * c] = True
+            want[c * (N0 // c):] = True
+            assert np.array_equal(m, want)
