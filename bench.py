@@ -59,6 +59,8 @@ def parse():
                     help="context sweep vs dense (deep and wide trees, random and aligned references)")
     ap.add_argument("--sweep-n", default="8192,32768,65536,131072,524288,2097152,4194304")
     ap.add_argument("--sweep-trees", default="deep,wide", help="comma list of deep, wide, speed")
+    ap.add_argument("--block", default=None,
+                    help="comma list of query positions per call: time zha_decode_block at each")
     ap.add_argument("--incremental", action="store_true",
                     help="build the tree by 4,096-token appends, then decode at p = 0.9, 0.95, 0.99")
     return ap.parse_args()
@@ -670,6 +672,69 @@ def incremental_mode(args, w):
     print(json.dumps(res), flush=True)
 
 
+def block_mode(args, w):
+    """Multi-query blocks: zha_decode_block with T query positions per sequence
+    (every summary and KV read shared by the T * G query rows of a group),
+    against T single-query zha_decode steps on the same cache; one JSON line per T."""
+    import torch
+
+    from tree_indexed_sparse_02_b200 import zha
+    from tree_indexed_sparse_02_b200.inputs import decode_stream, make_inputs
+    Ts = [int(x) for x in args.block.split(",")]
+    n, W = args.steps, args.warmup
+    N = w.context
+    steps_tokens = (n + W) * max(Ts)
+    cap = N + len(Ts) * 2 * steps_tokens + 8
+    inp = make_inputs(w, device="cuda", capacity=cap)
+    cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs, w.dtype, cap,
+                     summary=w.summary, queries=max(Ts))
+    buf = zha.Buffers(cfg)
+    zha.tree_build(cfg, buf.tree, inp.K, inp.refs, inp.lens, buf.status)
+    p = zha.p_schedule(w.p, w.levels, w.p_schedule)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    # queries and new tokens from the workload's decode stream (aligned mode: near the references)
+    k_s, v_s, q_s = decode_stream(w, max(Ts), device="cuda")
+
+    def timed(call, reps):
+        for _ in range(W):
+            call()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for j in range(reps):
+            flush.fill_(float(j))
+            ev[j][0].record(stream)
+            call()
+            ev[j][1].record(stream)
+        torch.cuda.synchronize()
+        buf.check_status("block steps")
+        return sum(a.elapsed_time(b) for a, b in ev) / reps
+
+    for T in Ts:
+        q = q_s[:T].transpose(0, 1).contiguous()          # [B, T, Hq, d]
+        kn = k_s[:T].transpose(0, 1).contiguous()
+        vn = v_s[:T].transpose(0, 1).contiguous()
+        out = torch.empty_like(q)
+        call = lambda: zha.decode_block(cfg, T, buf.tree, inp.K, inp.V, inp.refs, inp.lens, q, kn, vn, p,  # noqa: E731
+                                        buf.sel, out, buf.workspace, buf.status)
+        blk_ms = timed(call, n)
+        zha.profile_enable(True)
+        call()
+        torch.cuda.synchronize()
+        zha.profile_enable(False)
+        kern = {k: round(v[0] * 1e3, 1) for k, v in zha.profile_read().items()}
+        q1, k1, v1 = q[:, 0].contiguous(), kn[:, 0].contiguous(), vn[:, 0].contiguous()
+        o1 = torch.empty_like(q1)
+        one_ms = timed(lambda: zha.decode(cfg, buf.tree, inp.K, inp.V, inp.refs, inp.lens, q1, k1, v1, p, buf.sel,
+                                          o1, buf.workspace, buf.status), n)
+        print(json.dumps({"mode": "block", "workload": w.name, "refs": w.refs_mode, "summary": w.summary,
+                          "queries_per_call": T, "us_per_call": blk_ms * 1e3,
+                          "tokens_per_s": w.batch * T / (blk_ms / 1e3),
+                          "single_query_us_per_step": one_ms * 1e3,
+                          "single_query_tokens_per_s": w.batch / (one_ms / 1e3),
+                          "speedup_vs_single_query": (one_ms * T) / blk_ms, "kernels_us": kern,
+                          "l2": "flushed (256 MiB write) before every timed call"}), flush=True)
+
+
 def main():
     args = parse()
     w = workload(args)
@@ -682,6 +747,9 @@ def main():
         return
     if args.incremental:
         incremental_mode(args, w)
+        return
+    if args.block:
+        block_mode(args, w)
         return
     res = zha_arm(args, w, world, rank, local)
     if rank == 0:

@@ -97,9 +97,10 @@ enum {
  *       Microscaling (MX) specification v1.0; e is the smallest exponent with
  *       max|x| <= 448 * 2^e, elements round to nearest even. A node record
  *       shrinks from R*d*2 + 4R bytes to R*d + R*d/32 + 4R. Parents are built
- *       from the stored (rounded) children. Requires dtype ZHA_BF16. Queries
- *       are rounded to fp16 for scoring against these summaries (exact for
- *       |q_k| in [2^-14, 65504]; below, an absolute error under 2^-25). */
+ *       from the stored (rounded) children. Requires dtype ZHA_BF16. Scoring
+ *       against these summaries runs on E4M3 tensor-core MMAs: each query
+ *       head is held as 2^e (hi + lo/16) with hi, lo E4M3 and one power-of-two
+ *       scale per head (about 8 significant bits, as bf16). */
 enum { ZHA_SUMMARY_NATIVE = 0, ZHA_SUMMARY_MXFP8 = 1 };
 
 typedef struct zha_config {
@@ -116,7 +117,10 @@ typedef struct zha_config {
     int32_t flags;       /* ZHA_FLAG_* */
     int32_t attn_splits; /* split-K CTAs per (sequence, KV head); 0 = auto */
     int32_t summary;     /* ZHA_SUMMARY_NATIVE or ZHA_SUMMARY_MXFP8 */
-    int32_t reserved[2]; /* zero */
+    int32_t queries;     /* most query positions per sequence in one zha_decode_block
+                            call (0 or 1: single-query use only); the workspace is
+                            sized for it; queries * (n_q_heads / n_kv_heads) <= 32 */
+    int32_t reserved;    /* zero */
 } zha_config;
 
 /*
@@ -180,6 +184,10 @@ ZHA_API zha_status zha_tree_level_scales(const zha_config *cfg, int32_t level, s
 /* Bytes of scratch every call below may use (routing state + split-K partials). */
 ZHA_API size_t zha_workspace_bytes(const zha_config *cfg);
 ZHA_API zha_status zha_workspace_level_view(const zha_config *cfg, int32_t level, zha_level_view *v);
+/* The same for the last zha_decode_block call with T query positions (its
+ * scores are [batch][n_kv_heads][T * G][cap], row t * G + head). */
+ZHA_API zha_status zha_workspace_level_view_block(const zha_config *cfg, int32_t T, int32_t level,
+                                                  zha_level_view *v);
 
 /*
  * zha_tree_build -- summarise the first lens[b] tokens of every sequence
@@ -243,6 +251,33 @@ ZHA_API zha_status zha_decode(const zha_config *cfg, void *tree, void *K, void *
                       int32_t *lens, const void *q, const void *k_new, const void *v_new,
                       const float *p_levels, const zha_selection *sel, void *out,
                       void *workspace, int32_t *dev_status, void *stream);
+
+/*
+ * zha_decode_block -- T consecutive query positions of every sequence in one
+ * call: a multi-query decode or chunked-prefill block. The pages describe
+ * routing for one decoding query (section "How does top-p routing pick
+ * tokens"); this entry point applies it to T queries that share every
+ * summary and KV read. Reading taken here: with N0 = lens[b] tokens cached,
+ *   1. the block's keys/values k_new, v_new [batch][T][n_kv_heads][head_dim]
+ *      are written at positions N0 .. N0+T-1 and lens[b] becomes N0 + T;
+ *   2. every query row (t, head) routes as in zha_route over the tree of the
+ *      first N0 tokens (the tree before the block; p_levels as in zha_route);
+ *   3. row t attends exactly over {0} U its kept leaf chunks U
+ *      [c*floor(N0/c), N0 + t]: the cached tail after the last complete
+ *      chunk and the block's tokens up to its own position (causal);
+ *   4. the tree is extended by the T new tokens (as zha_tree_append).
+ * q and out are [batch][T][n_q_heads][head_dim]. In *sel, a group's head
+ * mask bit r is query row r = t * (n_q_heads / n_kv_heads) + head, and
+ * level_kept is [batch][n_kv_heads][T][n_q_heads / n_kv_heads][levels].
+ * Requires 1 <= T <= max(1, cfg->queries); ZHA_FLAG_TCGEN05 is ignored.
+ * With T = 1 the token set equals zha_decode's; the routing differs from it
+ * only when the new token completes a chunk (zha_decode routes over the
+ * extended tree).
+ */
+ZHA_API zha_status zha_decode_block(const zha_config *cfg, int32_t T, void *tree, void *K, void *V,
+                                    const void *refs, int32_t *lens, const void *q, const void *k_new,
+                                    const void *v_new, const float *p_levels, const zha_selection *sel,
+                                    void *out, void *workspace, int32_t *dev_status, void *stream);
 
 /*
  * zha_dense_decode -- the comparison kernel: exact softmax attention of every

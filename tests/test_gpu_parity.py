@@ -329,7 +329,7 @@ def test_p1_routes_all_and_equals_dense(zha):
 # ------------------------------------------------------------------- decode
 
 
-@pytest.mark.parametrize("w", [CASES[0], CASES[1], CASES[3]], ids=[IDS[0], IDS[1], IDS[3]])
+@pytest.mark.parametrize("w", CASES[:4], ids=IDS[:4])
 def test_decode_steps_match_oracle(zha, w):
     """zha_decode appends, routes and attends; the oracle repeats each step."""
     steps = 9

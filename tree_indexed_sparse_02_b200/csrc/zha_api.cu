@@ -31,15 +31,23 @@ zha_status check_config(const zha_config *c) {
     if (!(c->scale == c->scale)) return ZHA_ERR_INVALID_ARG;
     if (c->summary != ZHA_SUMMARY_NATIVE && c->summary != ZHA_SUMMARY_MXFP8) return ZHA_ERR_UNSUPPORTED;
     if (c->summary == ZHA_SUMMARY_MXFP8 && c->dtype != ZHA_BF16) return ZHA_ERR_UNSUPPORTED;
+    if (c->queries < 0) return ZHA_ERR_INVALID_ARG;
+    if ((c->queries > 1 ? c->queries : 1) * (c->n_q_heads / c->n_kv_heads) > 32) return ZHA_ERR_UNSUPPORTED;
     return ZHA_OK;
 }
 
-Geo make_geo(const zha_config *c) {
+// Geometry of one call; T query positions per sequence (zha_decode_block),
+// 1 for every other entry point. Workspace offsets depend on T; each call
+// lays out its own, inside zha_workspace_bytes (sized for the largest T).
+Geo make_geo(const zha_config *c, int T = 1) {
     Geo g{};
     g.B = c->batch;
     g.Hq = c->n_q_heads;
     g.Hkv = c->n_kv_heads;
-    g.G = c->n_q_heads / c->n_kv_heads;
+    g.Gq = c->n_q_heads / c->n_kv_heads;
+    g.T = T;
+    g.G = T * g.Gq;
+    g.lag = 0;
     g.d = c->head_dim;
     g.c = c->chunk;
     g.L = c->levels;
@@ -174,14 +182,20 @@ zha_status zha_tree_level_scales(const zha_config *cfg, int32_t level, size_t *s
 
 size_t zha_workspace_bytes(const zha_config *cfg) {
     if (check_config(cfg) != ZHA_OK) return 0;
-    return make_geo(cfg).ws_bytes;
+    return make_geo(cfg, cfg->queries > 1 ? cfg->queries : 1).ws_bytes;
 }
 
 zha_status zha_workspace_level_view(const zha_config *cfg, int32_t level, zha_level_view *v) {
+    return zha_workspace_level_view_block(cfg, 1, level, v);
+}
+
+zha_status zha_workspace_level_view_block(const zha_config *cfg, int32_t T, int32_t level,
+                                          zha_level_view *v) {
     zha_status s = check_config(cfg);
     if (s != ZHA_OK) return s;
     if (level < 1 || level > cfg->levels || !v) return ZHA_ERR_INVALID_ARG;
-    Geo g = make_geo(cfg);
+    if (T < 1 || T > (cfg->queries > 1 ? cfg->queries : 1)) return ZHA_ERR_INVALID_ARG;
+    Geo g = make_geo(cfg, T);
     v->cap = g.capv[level];
     v->cand_idx = g.ws_cand[level];
     v->cand_mask = g.ws_cmask[level];
@@ -277,6 +291,36 @@ zha_status zha_decode(const zha_config *cfg, void *tree, void *K, void *V, const
         e = zha::launch_route(g, tree, q, lens, p_levels, *sel, workspace, dev_status, st);
     if (e == cudaSuccess)
         e = zha::launch_attention(g, q, K, V, lens, sel, out, workspace, dev_status, st);
+    return cuda_status(e);
+}
+
+zha_status zha_decode_block(const zha_config *cfg, int32_t T, void *tree, void *K, void *V,
+                            const void *refs, int32_t *lens, const void *q, const void *k_new,
+                            const void *v_new, const float *p_levels, const zha_selection *sel,
+                            void *out, void *workspace, int32_t *dev_status, void *stream) {
+    zha_status s = check_config(cfg);
+    if (s != ZHA_OK) return s;
+    if (T < 1 || T > (cfg->queries > 1 ? cfg->queries : 1)) return ZHA_ERR_INVALID_ARG;
+    if ((s = check_p(cfg, p_levels)) != ZHA_OK) return s;
+    if ((s = check_sel(sel)) != ZHA_OK) return s;
+    if (!tree || !K || !V || !refs || !lens || !q || !k_new || !v_new || !out || !workspace ||
+        !aligned16(tree) || !aligned16(K) || !aligned16(V) || !aligned16(q) || !aligned16(out) ||
+        !aligned16(workspace) || !aligned16(refs))
+        return ZHA_ERR_INVALID_ARG;
+    Geo g = make_geo(cfg, T);
+    g.flags &= ~ZHA_FLAG_TCGEN05;
+    g.block = 1;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // tokens in; route over the tree before the block (lens - T); attend; extend the tree
+    cudaError_t e = zha::launch_decode_write(g, K, V, lens, k_new, v_new, dev_status, st);
+    if (e == cudaSuccess) {
+        Geo gr = g;
+        gr.lag = T;
+        e = zha::launch_route(gr, tree, q, lens, p_levels, *sel, workspace, dev_status, st);
+    }
+    if (e == cudaSuccess)
+        e = zha::launch_attention(g, q, K, V, lens, sel, out, workspace, dev_status, st);
+    if (e == cudaSuccess) e = zha::launch_tree_update(g, tree, K, refs, lens, T, dev_status, st);
     return cuda_status(e);
 }
 

@@ -37,9 +37,19 @@ struct TokenPlan {
     int b_start, b_len;    // current-chunk span
     int nv;                // stream length
     int lc;                // log2(c)
+    int blk_start;         // zha_decode_block: first block position (INT_MAX otherwise)
+    int gq;                // query heads per position: row r is position r / gq of the block
     uint32_t all;
     const int32_t *leaf;
     const uint32_t *hmask;
+
+    // rows that see position pos of the always-attended spans: all of them,
+    // except for a block token, which the block's earlier positions do not see
+    __device__ __forceinline__ uint32_t span_mask(int pos) const {
+        if (pos < blk_start) return all;
+        const int k = (pos - blk_start) * gq;
+        return k >= 32 ? 0u : (all & ~((1u << k) - 1u));
+    }
 
     // Split form of at(): fetch() issues the selection loads, finish() uses them.
     __device__ __forceinline__ void fetch(int v, int &lf, uint32_t &hm) const {
@@ -58,7 +68,7 @@ struct TokenPlan {
                 return;
             }
             pos = (lf << lc) | (v & ((1 << lc) - 1));
-            mask = hm | ((pos == 0 || pos >= cur_start) ? all : 0u);
+            mask = hm | ((pos == 0 || pos >= cur_start) ? span_mask(pos) : 0u);
             return;
         }
         at(v, pos, mask, status);
@@ -75,7 +85,7 @@ struct TokenPlan {
                 return;
             }
             pos = (lf << lc) | (v & ((1 << lc) - 1));
-            mask = __ldg(&hmask[e]) | ((pos == 0 || pos >= cur_start) ? all : 0u);
+            mask = __ldg(&hmask[e]) | ((pos == 0 || pos >= cur_start) ? span_mask(pos) : 0u);
             return;
         }
         v -= sel_tokens;
@@ -87,7 +97,7 @@ struct TokenPlan {
         v -= a_len;
         if (v < b_len) {
             pos = b_start + v;
-            mask = all;
+            mask = span_mask(pos);
             return;
         }
         pos = 0;
@@ -109,6 +119,8 @@ __device__ __forceinline__ TokenPlan make_plan(const Geo &g, const int32_t *lens
     tp.lc = __ffs(g.c) - 1;
     tp.all = g.G >= 32 ? 0xffffffffu : ((1u << g.G) - 1u);
     tp.n1 = N >> tp.lc;
+    tp.blk_start = 0x7fffffff;
+    tp.gq = g.Gq;
     if (dense || N == 0) {
         tp.b_start = 0;
         tp.b_len = N;
@@ -116,7 +128,20 @@ __device__ __forceinline__ TokenPlan make_plan(const Geo &g, const int32_t *lens
         tp.nv = N;
         return tp;
     }
-    tp.cur_start = (int)current_chunk_start(N, g.c, g.flags);
+    if (g.block) {
+        // the tree holds the first N - T tokens; the rest is the cached tail
+        // after its last complete chunk plus the block, attended causally
+        int n_tree = N - g.T;
+        if (n_tree < 0) {
+            set_status(status, ZHA_ERR_INVALID_ARG);
+            n_tree = 0;
+        }
+        tp.blk_start = n_tree;
+        tp.n1 = n_tree >> tp.lc;
+        tp.cur_start = tp.n1 << tp.lc;
+    } else {
+        tp.cur_start = (int)current_chunk_start(N, g.c, g.flags);
+    }
     int ns = sel->count[grp];
     if (ns < 0 || ns > g.cap[1]) {
         set_status(status, ZHA_ERR_INVALID_ARG);
@@ -202,6 +227,7 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
 
     const int grp = blockIdx.y, split = blockIdx.x, S = gridDim.x;
+    const int rbase = blockIdx.z * 16;     // this CTA's 16 query rows of the group
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gq = lane >> 2, t = lane & 3;
@@ -209,12 +235,12 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     const __nv_bfloat16 *Kg = K + (int64_t)grp * g.max_len * D;
     const __nv_bfloat16 *Vg = V + (int64_t)grp * g.max_len * D;
 
-    // Q as the A operand: rows gq and gq+8 are heads of this group (rows >= G are zero)
+    // Q as the A operand: rows gq and gq+8 are query rows of this group (rows >= G are zero)
     uint32_t qf[D / 16][4];
-    const int h0 = gq, h1 = gq + 8;
+    const int h0 = rbase + gq, h1 = rbase + gq + 8;
     {
-        const uint32_t *q0 = reinterpret_cast<const uint32_t *>(q + ((int64_t)b * g.Hq + kvh * g.G + h0) * D);
-        const uint32_t *q1 = reinterpret_cast<const uint32_t *>(q + ((int64_t)b * g.Hq + kvh * g.G + h1) * D);
+        const uint32_t *q0 = reinterpret_cast<const uint32_t *>(q + g.qrow(b, kvh, h0 < g.G ? h0 : 0) * D);
+        const uint32_t *q1 = reinterpret_cast<const uint32_t *>(q + g.qrow(b, kvh, h1 < g.G ? h1 : 0) * D);
 #pragma unroll
         for (int st = 0; st < D / 16; ++st) {
             qf[st][0] = h0 < g.G ? q0[st * 8 + t] : 0u;
@@ -392,8 +418,9 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
         sm_o[(warp * 16 + gq + 8) * OS + 8 * j + 2 * t + 1] = o[j][3];
     }
     __syncthreads();
-    const int64_t pbase = ((int64_t)grp * S + split) * g.G;
-    for (int i = threadIdx.x; i < g.G * D; i += blockDim.x) {
+    const int64_t pbase = ((int64_t)grp * S + split) * g.G + rbase;
+    const int rows = min(16, g.G - rbase);
+    for (int i = threadIdx.x; i < rows * D; i += blockDim.x) {
         const int h = i / D, dim = i % D;
         float M = -INFINITY;
 #pragma unroll
@@ -427,12 +454,13 @@ attn_simt_kernel(Geo g, const T *q, const T *K, const T *V, const int32_t *lens,
     __shared__ float sm_m[kAttnWarps][16], sm_l[kAttnWarps][16];
     __shared__ float sm_o[kAttnWarps][16][D];
     const int grp = blockIdx.y, split = blockIdx.x, S = gridDim.x;
+    const int rbase = blockIdx.z * 16;     // this CTA's 16 query rows of the group
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int G = g.G;
+    const int G = min(16, g.G - rbase);
     const TokenPlan tp = make_plan(g, lens, grp, &sel, dense != 0, status);
     for (int i = threadIdx.x; i < G * D; i += blockDim.x)
-        qs[i / D][i % D] = to_f32(q[((int64_t)b * g.Hq + kvh * G + i / D) * D + i % D]);
+        qs[i / D][i % D] = to_f32(q[g.qrow(b, kvh, rbase + i / D) * D + i % D]);
     __syncthreads();
     const T *Kg = K + (int64_t)grp * g.max_len * D;
     const T *Vg = V + (int64_t)grp * g.max_len * D;
@@ -466,7 +494,7 @@ attn_simt_kernel(Geo g, const T *q, const T *K, const T *V, const int32_t *lens,
 #pragma unroll
         for (int h = 0; h < 16; ++h) {
             if (h >= G) continue;
-            const float x = ((mask >> h) & 1u) ? sc[h] * sl2 : -INFINITY;
+            const float x = ((mask >> (rbase + h)) & 1u) ? sc[h] * sl2 : -INFINITY;
             const float mx = warp_max(x);
             const float m_new = fmaxf(m_run[h], mx);
             const float corr = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - m_new);
@@ -502,7 +530,7 @@ attn_simt_kernel(Geo g, const T *q, const T *K, const T *V, const int32_t *lens,
 #pragma unroll
             for (int e = 0; e < DL; ++e) sm_o[warp][h][lane + 32 * e] = o[h][e];
     __syncthreads();
-    const int64_t pbase = ((int64_t)grp * S + split) * G;
+    const int64_t pbase = ((int64_t)grp * S + split) * g.G + rbase;
     for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
         const int h = i / D, dim = i % D;
         float M = -INFINITY;
@@ -527,23 +555,49 @@ attn_simt_kernel(Geo g, const T *q, const T *K, const T *V, const int32_t *lens,
 template <typename T>
 __global__ void attn_merge_kernel(Geo g, int S, const float *part_ml, const float *part_o,
                                   T *out) {
+    // One block per (group, head): the splits' weights 2^(m_s - M) are formed
+    // in parallel (shared memory), then each thread sums one output coordinate
+    // over the splits with independent loads in flight.
+    extern __shared__ float wsplit[];                 // [S]
+    __shared__ float red[32];
     const int grp = blockIdx.x / g.G, h = blockIdx.x % g.G;
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int D = g.d;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int64_t base = (int64_t)grp * S;
+    float mx = -INFINITY;
+    for (int s = threadIdx.x; s < S; s += blockDim.x) mx = fmaxf(mx, part_ml[((base + s) * g.G + h) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
     float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, part_ml[(((int64_t)grp * S + s) * g.G + h) * 2]);
+    for (int w = 0; w < nw; ++w) M = fmaxf(M, red[w]);
+    __syncthreads();
+    float ls = 0.f;
+    for (int s = threadIdx.x; s < S; s += blockDim.x) {
+        const int64_t idx = (base + s) * g.G + h;
+        const float ms = part_ml[idx * 2];
+        const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+        wsplit[s] = f;
+        ls += f == 0.f ? 0.f : part_ml[idx * 2 + 1] * f;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    if (lane == 0) red[warp] = ls;
+    __syncthreads();
+    float L = 0.f;
+    for (int w = 0; w < nw; ++w) L += red[w];
     for (int dim = threadIdx.x; dim < D; dim += blockDim.x) {
-        float L = 0.f, acc = 0.f;
-        if (M != -INFINITY)
+        float acc = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll 8
             for (int s = 0; s < S; ++s) {
-                const int64_t idx = ((int64_t)grp * S + s) * g.G + h;
-                const float ms = part_ml[idx * 2];
-                if (ms == -INFINITY) continue;
-                const float f = exp2f(ms - M);
-                L += part_ml[idx * 2 + 1] * f;
-                acc += part_o[idx * D + dim] * f;
+                const float f = wsplit[s];
+                if (f != 0.f) acc = fmaf(part_o[((base + s) * g.G + h) * D + dim], f, acc);
             }
-        out[((int64_t)b * g.Hq + kvh * g.G + h) * D + dim] = from_f32<T>(L > 0.f ? acc / L : 0.f);
+        }
+        out[g.qrow(b, kvh, h) * D + dim] = from_f32<T>(L > 0.f ? acc / L : 0.f);
     }
 }
 
@@ -558,7 +612,7 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
     const int dense = sel == nullptr;
     zha_selection sv{};
     if (sel) sv = *sel;
-    dim3 grid(S, g.groups());
+    dim3 grid(S, g.groups(), (g.G + 15) / 16);
     const char *attn_name = dense ? "attn_dense" : "attn_sparse";
     if (g.dtype == ZHA_BF16) {
         auto qq = static_cast<const __nv_bfloat16 *>(q);
@@ -587,7 +641,8 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         ProfScope pm("attn_merge", st);
-        attn_merge_kernel<__nv_bfloat16><<<g.groups() * g.G, g.d, 0, st>>>(g, S, part_ml, part_o, static_cast<__nv_bfloat16 *>(out));
+        attn_merge_kernel<__nv_bfloat16><<<g.groups() * g.G, g.d, S * sizeof(float), st>>>(
+            g, S, part_ml, part_o, static_cast<__nv_bfloat16 *>(out));
     } else {
         auto qq = static_cast<const float *>(q);
         auto kk = static_cast<const float *>(K);
@@ -602,7 +657,8 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         ProfScope pm("attn_merge", st);
-        attn_merge_kernel<float><<<g.groups() * g.G, g.d, 0, st>>>(g, S, part_ml, part_o, static_cast<float *>(out));
+        attn_merge_kernel<float><<<g.groups() * g.G, g.d, S * sizeof(float), st>>>(
+            g, S, part_ml, part_o, static_cast<float *>(out));
     }
     return cudaGetLastError();
 }

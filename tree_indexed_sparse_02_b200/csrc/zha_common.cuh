@@ -26,7 +26,12 @@ __host__ __device__ inline int64_t level_nodes(int64_t n, int c, int level) {
 }
 
 struct Geo {
+    // G is the number of query rows a group routes and attends: T query
+    // positions x Gq query heads (T = 1 outside zha_decode_block)
     int B, Hq, Hkv, G, d, c, L, R, dtype, flags, splits;
+    int T, Gq;
+    int lag;                            // block tokens the tree does not hold yet (route reads lens - lag)
+    int block;                          // zha_decode_block: causal current span, tree before the block
     int summary;                        // ZHA_SUMMARY_*
     int64_t max_len;
     float s;
@@ -46,6 +51,12 @@ struct Geo {
     size_t ws_part_ml, ws_part_o;       // split-K partials
     size_t ws_bytes;
     __host__ __device__ int groups() const { return B * Hkv; }
+    // row r of group (b, kvh) -> index of its query vector in q [B][T][Hq][d]
+    // (and of its output in out, same layout); rows are ordered (t, head)
+    __host__ __device__ int64_t qrow(int b, int kvh, int r) const {
+        const int t = r / Gq;
+        return ((int64_t)b * T + t) * Hq + kvh * Gq + (r - t * Gq);
+    }
     __host__ __device__ int esize() const { return dtype == ZHA_BF16 ? 2 : 4; }
     __host__ __device__ bool mx() const { return summary == ZHA_SUMMARY_MXFP8; }
     __host__ __device__ int mu_esize() const { return mx() ? 1 : esize(); }

@@ -84,8 +84,9 @@ struct CandSource {
     }
 };
 
+// tokens the tree of group grp holds (a block call routes over the tree before its block)
 __device__ __forceinline__ int64_t group_len(const Geo &g, const int32_t *lens, int grp) {
-    const int64_t N = lens[grp / g.Hkv];
+    const int64_t N = (int64_t)lens[grp / g.Hkv] - g.lag;
     return (N < 0 || N > g.max_len) ? 0 : N;
 }
 
@@ -95,7 +96,7 @@ __global__ void route_init_kernel(Geo g, uint32_t *maxkey, uint32_t *minkey, uin
                                   const int32_t *lens, int32_t *status) {
     const int grp = blockIdx.x;
     if (threadIdx.x == 0) {
-        const int64_t N = lens[grp / g.Hkv];
+        const int64_t N = (int64_t)lens[grp / g.Hkv] - g.lag;
         if (N < 0 || N > g.max_len) set_status(status, ZHA_ERR_CAPACITY);
     }
     for (int i = threadIdx.x; i < g.L * g.G; i += blockDim.x) {
@@ -162,7 +163,7 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
 #pragma unroll
         for (int kp = 0; kp < KP; ++kp) {
             uint4 w = make_uint4(0, 0, 0, 0);
-            if (h < g.G) w = ldg16(q + ((int64_t)b * g.Hq + kvh * g.G + h) * D + kp * 32 + t * 8);
+            if (h < g.G) w = ldg16(q + g.qrow(b, kvh, h) * D + kp * 32 + t * 8);
             bq[nt][kp][0] = w.x; bq[nt][kp][1] = w.y; bq[nt][kp][2] = w.z; bq[nt][kp][3] = w.w;
         }
     }
@@ -317,7 +318,7 @@ score_pack_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_
 #pragma unroll
         for (int kp = 0; kp < KP; ++kp) {
             uint4 w = make_uint4(0, 0, 0, 0);
-            if (h < g.G) w = ldg16(q + ((int64_t)b * g.Hq + kvh * g.G + h) * D + kp * 32 + t * 8);
+            if (h < g.G) w = ldg16(q + g.qrow(b, kvh, h) * D + kp * 32 + t * 8);
             bq[nt][kp][0] = w.x; bq[nt][kp][1] = w.y; bq[nt][kp][2] = w.z; bq[nt][kp][3] = w.w;
         }
     }
@@ -441,38 +442,33 @@ score_pack_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_
         }
 }
 
-__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4],
-                                              uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// two E4M3 bytes (low 16 bits of w) -> two fp16 (exact: E4M3 is a subset of fp16)
-__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t w) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xffffu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+__device__ __forceinline__ uint32_t e4m3_rn(float x) {
+    return (uint32_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
 }
 
-// eight bf16 -> eight fp16 (four packed pairs), round to nearest
-__device__ __forceinline__ void bf16x8_f16x8(const uint4 &w, uint32_t (&o)[4]) {
-    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&in[j]));
-        const __half2 h = __float22half2_rn(f);
-        o[j] = *reinterpret_cast<const uint32_t *>(&h);
-    }
+__device__ __forceinline__ float e4m3_value(uint32_t byte) {
+    return __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)byte, __NV_E4M3)));
 }
 
 // Scoring against MX-FP8 summaries (E4M3 bytes, one power-of-two scale per 32
-// coordinates of a plane). Same warp layout as score_mma_kernel: A = planes,
-// B = query heads, mma.sync m16n8k16 in fp16 (E4M3 converts to fp16 exactly;
-// the queries are rounded to fp16 once). Each lane reads 8 contiguous bytes of
-// a row per 32-coordinate block, so the two MMAs of a block see one scale per
-// row: they accumulate into a temporary that is scaled into the plane sums.
+// coordinates of a plane) with E4M3 tensor-core MMAs, so the summaries are
+// never converted: mma.sync m16n8k32 (A = planes, B = query heads, one MMA
+// per 32-coordinate block). Each query head is held as two E4M3 terms with
+// one power-of-two scale per head: q ~ 2^e (hi + lo / 16), hi the nearest
+// E4M3 of q / 2^e (e the smallest with max|q| <= 448 * 2^e), lo that of the
+// remainder times 16 -- about 8 significant bits, the precision of bf16.
+// Each lane reads 8 contiguous bytes of a row per block, so an MMA sees one
+// plane scale per row; the block's two MMAs (hi, lo) are combined and scaled
+// into the plane sums, and the head scale is applied once at the end.
 template <int D, int MT, int NT, int U>
 __global__ void __launch_bounds__(kScoreWarps * 32)
 score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias, const __nv_bfloat16 *q,
@@ -488,16 +484,55 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
     if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
     const uint32_t all = all_heads(g.G);
 
-    uint32_t bq[NT][KP][4];
+    // B fragments: head nt*8 + gq, block kp, bytes [32 kp + 8 t, +8) as two words,
+    // for the hi and lo terms; hscale[nt][j]: 2^e of the head in C column 2t + j
+    uint32_t bhi[NT][KP][2], blo[NT][KP][2];
+    float hscale[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         const int h = nt * 8 + gq;
+        float v[KP][8];
+        float amax = 0.f;
 #pragma unroll
         for (int kp = 0; kp < KP; ++kp) {
             uint4 w = make_uint4(0, 0, 0, 0);
-            if (h < g.G) w = ldg16(q + ((int64_t)b * g.Hq + kvh * g.G + h) * D + kp * 32 + t * 8);
-            bf16x8_f16x8(w, bq[nt][kp]);
+            if (h < g.G) w = ldg16(q + g.qrow(b, kvh, h) * D + kp * 32 + t * 8);
+            const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&in[j]));
+                v[kp][2 * j] = f.x;
+                v[kp][2 * j + 1] = f.y;
+                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
         }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        int ex = 0;
+        if (amax > 0.f) {
+            int k;
+            const float f = frexpf(amax, &k);          // amax = f 2^k, 448 = 0.875 2^9
+            ex = (f <= 0.875f) ? k - 9 : k - 8;
+        }
+#pragma unroll
+        for (int kp = 0; kp < KP; ++kp)
+#pragma unroll
+            for (int w2 = 0; w2 < 2; ++w2) {
+                uint32_t hi = 0u, lo = 0u;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x = scalbnf(v[kp][4 * w2 + e], -ex);
+                    const uint32_t bh = e4m3_rn(x);
+                    const uint32_t bl = e4m3_rn((x - e4m3_value(bh)) * 16.f);
+                    hi |= bh << (8 * e);
+                    lo |= bl << (8 * e);
+                }
+                bhi[nt][kp][w2] = hi;
+                blo[nt][kp][w2] = lo;
+            }
+        const float myscale = scalbnf(1.f, ex);
+        hscale[nt][0] = __shfl_sync(0xffffffffu, myscale, (2 * t) * 4);
+        hscale[nt][1] = __shfl_sync(0xffffffffu, myscale, (2 * t + 1) * 4);
     }
     float runmax[NT][2], runmin[NT][2];
 #pragma unroll
@@ -572,29 +607,26 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
 #pragma unroll
                 for (int kp = 0; kp < KP; ++kp) {
                     const uint2 &xa = ra[u][mt][kp], &xb = rb[u][mt][kp];
-                    const uint32_t a0[4] = {e4m3x2_f16x2(xa.x), e4m3x2_f16x2(xb.x), e4m3x2_f16x2(xa.x >> 16),
-                                            e4m3x2_f16x2(xb.x >> 16)};
-                    const uint32_t a1[4] = {e4m3x2_f16x2(xa.y), e4m3x2_f16x2(xb.y), e4m3x2_f16x2(xa.y >> 16),
-                                            e4m3x2_f16x2(xb.y >> 16)};
                     // 2^(byte - 127) of this block for rows r0 and r1
                     const float s0 = __uint_as_float(((sa[u][mt] >> (8 * kp)) & 0xffu) << 23);
                     const float s1 = __uint_as_float(((sb[u][mt] >> (8 * kp)) & 0xffu) << 23);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_f16_16816(tmp, a0, bq[nt][kp][0], bq[nt][kp][1]);
-                        mma_f16_16816(tmp, a1, bq[nt][kp][2], bq[nt][kp][3]);
-                        acc[nt][0] = fmaf(s0, tmp[0], acc[nt][0]);
-                        acc[nt][1] = fmaf(s0, tmp[1], acc[nt][1]);
-                        acc[nt][2] = fmaf(s1, tmp[2], acc[nt][2]);
-                        acc[nt][3] = fmaf(s1, tmp[3], acc[nt][3]);
+                        float th[4] = {0.f, 0.f, 0.f, 0.f}, tl[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_e4m3_16832(th, xa.x, xb.x, xa.y, xb.y, bhi[nt][kp][0], bhi[nt][kp][1]);
+                        mma_e4m3_16832(tl, xa.x, xb.x, xa.y, xb.y, blo[nt][kp][0], blo[nt][kp][1]);
+                        acc[nt][0] = fmaf(s0, fmaf(tl[0], 0.0625f, th[0]), acc[nt][0]);
+                        acc[nt][1] = fmaf(s0, fmaf(tl[1], 0.0625f, th[1]), acc[nt][1]);
+                        acc[nt][2] = fmaf(s1, fmaf(tl[2], 0.0625f, th[2]), acc[nt][2]);
+                        acc[nt][3] = fmaf(s1, fmaf(tl[3], 0.0625f, th[3]), acc[nt][3]);
                     }
                 }
                 const float b0 = ba[u][mt], b1 = bb[u][mt];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    e[nt][0] = fmaxf(e[nt][0], fmaxf(fmaf(s, acc[nt][0], b0), fmaf(s, acc[nt][2], b1)));
-                    e[nt][1] = fmaxf(e[nt][1], fmaxf(fmaf(s, acc[nt][1], b0), fmaf(s, acc[nt][3], b1)));
+                    const float c0 = s * hscale[nt][0], c1 = s * hscale[nt][1];
+                    e[nt][0] = fmaxf(e[nt][0], fmaxf(fmaf(c0, acc[nt][0], b0), fmaf(c0, acc[nt][2], b1)));
+                    e[nt][1] = fmaxf(e[nt][1], fmaxf(fmaf(c1, acc[nt][1], b0), fmaf(c1, acc[nt][3], b1)));
                 }
             }
 #pragma unroll
@@ -643,8 +675,8 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
 template <int D>
 __global__ void score_f32_kernel(Geo g, const float *mu, const float *bias, const float *q,
                                  const int32_t *lens, LevelWs lw, LevelWs up, int level) {
-    __shared__ float qs[16][D];
-    __shared__ float es[32][16];
+    __shared__ float qs[32][D];
+    __shared__ float es[32][32];
     const int grp = blockIdx.y;
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int64_t cap = g.cap[level], capv = g.capv[level];
@@ -653,7 +685,7 @@ __global__ void score_f32_kernel(Geo g, const float *mu, const float *bias, cons
     if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
     const uint32_t all = all_heads(g.G);
     for (int i = threadIdx.x; i < g.G * D; i += blockDim.x)
-        qs[i / D][i % D] = q[((int64_t)b * g.Hq + kvh * g.G + i / D) * D + i % D];
+        qs[i / D][i % D] = q[g.qrow(b, kvh, i / D) * D + i % D];
     float runmax = -INFINITY, runmin = INFINITY;
     __syncthreads();
     for (int i = blockIdx.x; i < n; i += gridDim.x) {
@@ -1134,7 +1166,7 @@ select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t 
         [&](int64_t i) { mybits[i >> 3] |= (uint8_t)(1u << (i & 7)); });
     if (level_kept && threadIdx.x == 0) {
         const int b = grp / g.Hkv, kvh = grp % g.Hkv;
-        level_kept[((int64_t)b * g.Hq + kvh * g.G + h) * g.L + (level - 1)] = nk;
+        level_kept[((int64_t)grp * g.G + h) * g.L + (level - 1)] = nk;
     }
     // the last of the group's G CTAs joins the heads' bitmaps and compacts
     __threadfence();
@@ -1227,20 +1259,18 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                 const int64_t want = (capv + kScoreWarps - 1) / kScoreWarps;
                 const int per_group = (int)max64(1, min64(want, (148 * 8 + groups - 1) / groups));
                 dim3 grid(per_group, groups);
-                const int mt = g.R > 16 ? 2 : 1, nt = g.G > 8 ? 2 : 1;
+                const int mt = g.R > 16 ? 2 : 1, nt = g.G > 16 ? 4 : (g.G > 8 ? 2 : 1);
 #define ZHA_SCORE_MX(D, MT, NT, U) \
     score_mx8_kernel<D, MT, NT, U><<<grid, kScoreWarps * 32, 0, st>>>(g, mu, scl, bias, qq, lens, lw, up, level)
+#define ZHA_SCORE_MX_N(D, MT, U1) \
+    do { if (nt == 1) ZHA_SCORE_MX(D, MT, 1, U1); else if (nt == 2) ZHA_SCORE_MX(D, MT, 2, 2); \
+         else ZHA_SCORE_MX(D, MT, 4, 1); } while (0)
                 if (g.d == 128) {
-                    if (mt == 1 && nt == 1) ZHA_SCORE_MX(128, 1, 1, 4);
-                    else if (mt == 1) ZHA_SCORE_MX(128, 1, 2, 2);
-                    else if (nt == 1) ZHA_SCORE_MX(128, 2, 1, 2);
-                    else ZHA_SCORE_MX(128, 2, 2, 2);
+                    if (mt == 1) ZHA_SCORE_MX_N(128, 1, 4); else ZHA_SCORE_MX_N(128, 2, 2);
                 } else {
-                    if (mt == 1 && nt == 1) ZHA_SCORE_MX(64, 1, 1, 4);
-                    else if (mt == 1) ZHA_SCORE_MX(64, 1, 2, 4);
-                    else if (nt == 1) ZHA_SCORE_MX(64, 2, 1, 2);
-                    else ZHA_SCORE_MX(64, 2, 2, 2);
+                    if (mt == 1) ZHA_SCORE_MX_N(64, 1, 4); else ZHA_SCORE_MX_N(64, 2, 2);
                 }
+#undef ZHA_SCORE_MX_N
 #undef ZHA_SCORE_MX
             } else if (g.dtype == ZHA_BF16 && (g.flags & ZHA_FLAG_TCGEN05) && score_tc_supported(g)) {
                 e = launch_score_tc(g, tb + g.mu_off[level], reinterpret_cast<const float *>(tb + g.bias_off[level]),
@@ -1262,9 +1292,13 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
     do { if (rl == 0) ZHA_SCORE_PACK(D, NT, 0); else if (rl == 1) ZHA_SCORE_PACK(D, NT, 1); \
          else if (rl == 2) ZHA_SCORE_PACK(D, NT, 2); else ZHA_SCORE_PACK(D, NT, 3); } while (0)
                 if (g.d == 128) {
-                    if (g.G > 8) ZHA_SCORE_PACK_R(128, 2); else ZHA_SCORE_PACK_R(128, 1);
+                    if (g.G > 16) ZHA_SCORE_PACK_R(128, 4);
+                    else if (g.G > 8) ZHA_SCORE_PACK_R(128, 2);
+                    else ZHA_SCORE_PACK_R(128, 1);
                 } else {
-                    if (g.G > 8) ZHA_SCORE_PACK_R(64, 2); else ZHA_SCORE_PACK_R(64, 1);
+                    if (g.G > 16) ZHA_SCORE_PACK_R(64, 4);
+                    else if (g.G > 8) ZHA_SCORE_PACK_R(64, 2);
+                    else ZHA_SCORE_PACK_R(64, 1);
                 }
 #undef ZHA_SCORE_PACK_R
 #undef ZHA_SCORE_PACK
@@ -1275,20 +1309,17 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                 const int64_t want = (capv + kScoreWarps - 1) / kScoreWarps;
                 const int per_group = (int)max64(1, min64(want, (148 * 8 + groups - 1) / groups));
                 dim3 grid(per_group, groups);
-                const int mt = g.R > 16 ? 2 : 1, nt = g.G > 8 ? 2 : 1;
+                const int mt = g.R > 16 ? 2 : 1, nt = g.G > 16 ? 4 : (g.G > 8 ? 2 : 1);
 #define ZHA_SCORE(D, MT, NT) \
     score_mma_kernel<D, MT, NT><<<grid, kScoreWarps * 32, 0, st>>>(g, mu, bias, qq, lens, lw, up, level)
+#define ZHA_SCORE_N(D, MT) \
+    do { if (nt == 1) ZHA_SCORE(D, MT, 1); else if (nt == 2) ZHA_SCORE(D, MT, 2); else ZHA_SCORE(D, MT, 4); } while (0)
                 if (g.d == 128) {
-                    if (mt == 1 && nt == 1) ZHA_SCORE(128, 1, 1);
-                    else if (mt == 1) ZHA_SCORE(128, 1, 2);
-                    else if (nt == 1) ZHA_SCORE(128, 2, 1);
-                    else ZHA_SCORE(128, 2, 2);
+                    if (mt == 1) ZHA_SCORE_N(128, 1); else ZHA_SCORE_N(128, 2);
                 } else {
-                    if (mt == 1 && nt == 1) ZHA_SCORE(64, 1, 1);
-                    else if (mt == 1) ZHA_SCORE(64, 1, 2);
-                    else if (nt == 1) ZHA_SCORE(64, 2, 1);
-                    else ZHA_SCORE(64, 2, 2);
+                    if (mt == 1) ZHA_SCORE_N(64, 1); else ZHA_SCORE_N(64, 2);
                 }
+#undef ZHA_SCORE_N
 #undef ZHA_SCORE
             } else {
                 const auto *mu = reinterpret_cast<const float *>(tb + g.mu_off[level]);

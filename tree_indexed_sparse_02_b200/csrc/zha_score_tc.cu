@@ -233,7 +233,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap mu_map, Geo g, TcArgs a) {
         const int b = grp / g.Hkv, kvh = grp % g.Hkv;
         uint4 v = make_uint4(0, 0, 0, 0);
         if (row < g.G)
-            v = *reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * g.Hq + kvh * g.G + row) * 128 + chunk * 8);
+            v = *reinterpret_cast<const uint4 *>(a.q + g.qrow(b, kvh, row) * 128 + chunk * 8);
         const int half = chunk >> 3, c8 = chunk & 7;
         *reinterpret_cast<uint4 *>(smem + kTcStages * kStageBytes + kMetaSlots * kMetaBytes + grp * kQBytes +
                                    half * 2048 + row * 128 +
@@ -479,7 +479,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }  // namespace
 
 bool score_tc_supported(const Geo &g) {
-    return g.dtype == ZHA_BF16 && !g.mx() && g.d == 128 && g.R == 16 && g.G <= 16 && g.groups() <= kMaxGroups &&
+    return g.dtype == ZHA_BF16 && !g.mx() && g.T == 1 && g.lag == 0 && g.d == 128 && g.R == 16 && g.G <= 16 && g.groups() <= kMaxGroups &&
            encode_fn() != nullptr;
 }
 

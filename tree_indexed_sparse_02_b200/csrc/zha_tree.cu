@@ -206,8 +206,10 @@ tree_level_kernel(Geo g, TreePtrs tp, const T *K, const T *refs, const int32_t *
 // Few new tokens (a decode step): one block per group walks every level,
 // warp r computing plane r of each changed node; levels are separated by a
 // block barrier, which also makes the children's global writes visible.
+constexpr int kPathWarps = 16;
+
 template <typename T, int EPL, bool MX>
-__global__ void tree_path_kernel(Geo g, TreePtrs tp, const T *K, const T *refs,
+__global__ void __launch_bounds__(kPathWarps * 32) tree_path_kernel(Geo g, TreePtrs tp, const T *K, const T *refs,
                                  const int32_t *lens, int n_new, int32_t *status) {
     const int grp = blockIdx.x;
     const int b = grp / g.Hkv;
@@ -233,7 +235,8 @@ template <typename T, int EPL, bool MX>
 cudaError_t tree_update_t(const Geo &g, const TreePtrs &tp, const T *K, const T *refs,
                           const int32_t *lens, int n_new, int32_t *status, cudaStream_t st) {
     if (n_new >= 0 && n_new <= g.c) {
-        const int warps = g.R < 4 ? 4 : g.R;
+        // one warp per plane of a node, up to kPathWarps (more planes: a warp takes several)
+        const int warps = g.R < 4 ? 4 : (g.R > kPathWarps ? kPathWarps : g.R);
         ProfScope ps("tree_path", st);
         tree_path_kernel<T, EPL, MX><<<g.groups(), warps * 32, 0, st>>>(g, tp, K, refs, lens, n_new,
                                                                     status);
@@ -285,27 +288,29 @@ cudaError_t launch_tree_update(const Geo &g, void *tree, const void *K, const vo
                       : tree_update_t<float, 2, false>(g, tp, k, r, lens, n_new, status, st);
 }
 
-// Decode step prologue: write the new token of every (sequence, KV head) at
-// position lens[b], then advance lens[b] (one block per sequence, so the
-// increment follows every read of the old length in the block).
+// Decode step prologue: write the g.T new tokens of every (sequence, KV head)
+// (k_new [B][T][Hkv][d]) at positions lens[b] .. lens[b] + T - 1, then advance
+// lens[b] by T (one block per sequence, so the increment follows every read
+// of the old length in the block).
 template <typename T>
 __global__ void decode_write_kernel(Geo g, T *K, T *V, int32_t *lens, const T *k_new,
                                     const T *v_new, int32_t *status) {
     const int b = blockIdx.x;
     const int64_t n = lens[b];
-    const bool ok = n >= 0 && n < g.max_len;
+    const bool ok = n >= 0 && n + g.T <= g.max_len;
     if (ok) {
-        for (int i = threadIdx.x; i < g.Hkv * g.d; i += blockDim.x) {
-            const int kvh = i / g.d, e = i % g.d;
-            const int64_t dst = (((int64_t)b * g.Hkv + kvh) * g.max_len + n) * g.d + e;
-            K[dst] = k_new[((int64_t)b * g.Hkv + kvh) * g.d + e];
-            V[dst] = v_new[((int64_t)b * g.Hkv + kvh) * g.d + e];
+        for (int i = threadIdx.x; i < g.T * g.Hkv * g.d; i += blockDim.x) {
+            const int t = i / (g.Hkv * g.d), kvh = (i / g.d) % g.Hkv, e = i % g.d;
+            const int64_t dst = (((int64_t)b * g.Hkv + kvh) * g.max_len + n + t) * g.d + e;
+            const int64_t src = (((int64_t)b * g.T + t) * g.Hkv + kvh) * g.d + e;
+            K[dst] = k_new[src];
+            V[dst] = v_new[src];
         }
     }
     __syncthreads();
     if (threadIdx.x == 0) {
         if (ok)
-            lens[b] = (int32_t)(n + 1);
+            lens[b] = (int32_t)(n + g.T);
         else
             set_status(status, ZHA_ERR_CAPACITY);
     }

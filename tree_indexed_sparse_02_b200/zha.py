@@ -36,7 +36,7 @@ class Config(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("chunk", ctypes.c_int32), ("levels", ctypes.c_int32),
                 ("n_refs", ctypes.c_int32), ("dtype", ctypes.c_int32), ("max_len", ctypes.c_int64),
                 ("scale", ctypes.c_float), ("flags", ctypes.c_int32), ("attn_splits", ctypes.c_int32),
-                ("summary", ctypes.c_int32), ("reserved", ctypes.c_int32 * 2)]
+                ("summary", ctypes.c_int32), ("queries", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
     @property
     def group(self) -> int:
@@ -73,11 +73,13 @@ def _load():
         "zha_tree_level_scales": ([CP, i32, ctypes.POINTER(sz)], i32),
         "zha_workspace_bytes": ([CP], sz),
         "zha_workspace_level_view": ([CP, i32, ctypes.POINTER(LevelView)], i32),
+        "zha_workspace_level_view_block": ([CP, i32, i32, ctypes.POINTER(LevelView)], i32),
         "zha_tree_build": ([CP, P, P, P, P, P, P], i32),
         "zha_tree_append": ([CP, P, P, P, P, i32, P, P], i32),
         "zha_route": ([CP, P, P, P, P, SP, P, P, P], i32),
         "zha_sparse_attn": ([CP, P, P, P, P, SP, P, P, P, P], i32),
         "zha_decode": ([CP, P, P, P, P, P, P, P, P, P, SP, P, P, P, P], i32),
+        "zha_decode_block": ([CP, i32, P, P, P, P, P, P, P, P, P, SP, P, P, P, P], i32),
         "zha_dense_decode": ([CP, P, P, P, P, P, P, P, P], i32),
         "zha_topp_select": ([P, P, i32, i64, f32, P, P, P], i32),
         "zha_p_schedule": ([f32, i32, i32, ctypes.POINTER(f32)], i32),
@@ -101,11 +103,11 @@ def lib():
 
 
 def config(batch, n_q_heads, n_kv_heads, head_dim, chunk, levels, n_refs, dtype="bf16", max_len=4096,
-           scale=0.0, flags=0, attn_splits=0, summary="native") -> Config:
+           scale=0.0, flags=0, attn_splits=0, summary="native", queries=0) -> Config:
     dt = {"bf16": ZHA_BF16, "f32": ZHA_F32}.get(dtype, dtype)
     sm = {"native": ZHA_SUMMARY_NATIVE, "mxfp8": ZHA_SUMMARY_MXFP8}.get(summary, summary)
     c = Config(batch, n_q_heads, n_kv_heads, head_dim, chunk, levels, n_refs, dt, max_len, scale, flags,
-               attn_splits, sm)
+               attn_splits, sm, queries)
     check(_lib.zha_check_config(ctypes.byref(c)), "zha_check_config")
     return c
 
@@ -144,9 +146,10 @@ def tree_level_offsets(cfg: Config, level: int):
     return mu.value, b.value
 
 
-def workspace_level_view(cfg: Config, level: int) -> LevelView:
+def workspace_level_view(cfg: Config, level: int, T: int = 1) -> LevelView:
     v = LevelView()
-    check(_lib.zha_workspace_level_view(ctypes.byref(cfg), level, ctypes.byref(v)), "zha_workspace_level_view")
+    check(_lib.zha_workspace_level_view_block(ctypes.byref(cfg), int(T), level, ctypes.byref(v)),
+          "zha_workspace_level_view_block")
     return v
 
 
@@ -198,6 +201,15 @@ def decode(cfg, tree, K, V, refs, lens, q, k_new, v_new, p, sel, out, workspace,
     check(_lib.zha_decode(ctypes.byref(cfg), _p(tree), _p(K), _p(V), _p(refs), _p(lens), _p(q), _p(k_new),
                           _p(v_new), _plevels(cfg, p), ctypes.byref(s), _p(out), _p(workspace),
                           _p(dev_status), _stream(stream)), "zha_decode")
+
+
+def decode_block(cfg, T, tree, K, V, refs, lens, q, k_new, v_new, p, sel, out, workspace, dev_status=None,
+                 stream=None):
+    """T query positions per sequence: q, out [B, T, Hq, d]; k_new, v_new [B, T, Hkv, d]."""
+    s = _sel(sel)
+    check(_lib.zha_decode_block(ctypes.byref(cfg), int(T), _p(tree), _p(K), _p(V), _p(refs), _p(lens), _p(q),
+                                _p(k_new), _p(v_new), _plevels(cfg, p), ctypes.byref(s), _p(out),
+                                _p(workspace), _p(dev_status), _stream(stream)), "zha_decode_block")
 
 
 def dense_decode(cfg, q, K, V, lens, out, workspace, dev_status=None, stream=None):
@@ -279,8 +291,9 @@ class Buffers:
             "leaf_idx": torch.zeros((cfg.batch, cfg.n_kv_heads, cap1), dtype=torch.int32, device=device),
             "head_mask": torch.zeros((cfg.batch, cfg.n_kv_heads, cap1), dtype=torch.int32, device=device),
             "count": torch.zeros((cfg.batch, cfg.n_kv_heads), dtype=torch.int32, device=device),
-            "level_kept": (torch.zeros((cfg.batch, cfg.n_q_heads, cfg.levels), dtype=torch.int32, device=device)
-                           if level_kept else None),
+            # [B, Hq, L] for single queries; a block call writes [B, Hkv, T, G, L]
+            "level_kept": (torch.zeros((cfg.batch, cfg.n_q_heads * max(cfg.queries, 1), cfg.levels),
+                                       dtype=torch.int32, device=device) if level_kept else None),
         }
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         del G
@@ -319,13 +332,14 @@ class Buffers:
         return self.tree[off.value:off.value + n].view(cfg.batch, cfg.n_kv_heads, cap, cfg.n_refs,
                                                         cfg.head_dim // 32)
 
-    def level_state(self, level: int):
-        """Routing state of one level from the last route/decode call."""
+    def level_state(self, level: int, T: int = 1):
+        """Routing state of one level from the last route/decode call (T: query
+        positions of the last decode_block call; its rows are t * G + head)."""
         cfg = self.cfg
-        v = workspace_level_view(cfg, level)
+        v = workspace_level_view(cfg, level, T)
         cap = v.cap
         BG = cfg.batch * cfg.n_kv_heads
-        G = cfg.group
+        G = cfg.group * T
         ws = self.workspace
 
         def arr(off, n, dt):
