@@ -74,6 +74,11 @@ Geo make_geo(const zha_config *c, int T = 1) {
     }
     g.tree_bytes = off;
     off = 0;
+    {
+        const size_t rows_max = (size_t)g.Gq * (c->queries > 1 ? c->queries : 1);
+        g.ws_ghist = off;
+        off = align256(off + groups * rows_max * zha::kSelBuckets * 8);
+    }
     for (int l = 1; l <= g.L; ++l) {
         g.capv[l] = (g.cap[l] + g.c + 7) & ~int64_t(7);
         const size_t n = groups * g.capv[l];
@@ -81,7 +86,7 @@ Geo make_geo(const zha_config *c, int T = 1) {
         g.ws_cmask[l] = off;  off = align256(off + n * 4);
         g.ws_kept[l] = off;   off = align256(off + n * 4);
         g.ws_scores[l] = off; off = align256(off + n * g.G * 4);
-        g.ws_keptbits[l] = off; off = align256(off + n * g.G / 8);
+        g.ws_keptbits[l] = off; off = align256(off + groups * g.G * g.bits_stride(l));
         g.ws_count[l] = off;  off = align256(off + groups * 4);
         const size_t k = groups * g.cap[l];
         g.ws_plist[l] = off;  off = align256(off + k * 4);
@@ -94,6 +99,15 @@ Geo make_geo(const zha_config *c, int T = 1) {
     off = align256(off + (size_t)g.L * groups * g.G * 4);
     g.ws_done = off;
     off = align256(off + (size_t)g.L * groups * 4);
+    g.ws_glidx = off;
+    off = align256(off + groups * g.G * zha::kSelList * 4);
+    g.ws_glkey = off;
+    off = align256(off + groups * g.G * zha::kSelList * 4);
+    g.ws_gctr = off;
+    off = align256(off + (size_t)g.L * groups * g.G * 4 * 4);
+    g.ws_lookback = off;
+    for (int l = 1; l <= g.L; ++l) off += groups * ((g.capv[l] + zha::kJoinChunk - 1) / zha::kJoinChunk) * 8;
+    off = align256(off);
     int splits = c->attn_splits;
     if (splits == 0) {
         // one wave of two resident CTAs per SM over all groups, at most one per 64 tokens

@@ -25,6 +25,10 @@ __host__ __device__ inline int64_t level_nodes(int64_t n, int c, int level) {
     return m;
 }
 
+constexpr int kSelBuckets = 4096;       // histogram buckets of the top-p selection
+constexpr int kSelList = 1024;          // crossing-bucket members ordered in shared memory
+constexpr int kJoinChunk = 2048;        // candidates per CTA of the join / compaction
+
 struct Geo {
     // G is the number of query rows a group routes and attends: T query
     // positions x Gq query heads (T = 1 outside zha_decode_block)
@@ -45,12 +49,20 @@ struct Geo {
     size_t ws_cand[kMaxLevels + 1], ws_cmask[kMaxLevels + 1], ws_scores[kMaxLevels + 1],
         ws_kept[kMaxLevels + 1], ws_count[kMaxLevels + 1];     // candidates of a level
     size_t ws_plist[kMaxLevels + 1], ws_pmask[kMaxLevels + 1], ws_pcount[kMaxLevels + 1];  // kept
-    size_t ws_keptbits[kMaxLevels + 1];  // [B*Hkv][G][capv/8] bytes: each head's kept bitmap
+    size_t ws_keptbits[kMaxLevels + 1];  // [B*Hkv][G][bits_stride] bytes: each row's kept bitmap
+    size_t ws_lookback;                 // [L][B*Hkv][join chunks] u64 running counts of the compaction
     size_t ws_maxkey, ws_minkey;        // [L][B*Hkv][G] u32 ordered keys of the scores
     size_t ws_done;                     // [L][B*Hkv] u32 finished select CTAs
     size_t ws_part_ml, ws_part_o;       // split-K partials
+    // selection spread over several CTAs per query row (same offset for every T:
+    // the histograms come first and are left zeroed by every call)
+    size_t ws_ghist;                    // [B*Hkv][rows at cfg.queries][kSelBuckets] u64
+    size_t ws_glidx, ws_glkey;          // [B*Hkv][G][kSelList] crossing-bucket members
+    size_t ws_gctr;                     // [L][B*Hkv][G][4] u32 arrivals, list count, kept count
     size_t ws_bytes;
     __host__ __device__ int groups() const { return B * Hkv; }
+    // bytes of one row's kept bitmap at a level (capv / 8, padded to 16 bytes)
+    __host__ __device__ int64_t bits_stride(int level) const { return ((capv[level] >> 3) + 15) & ~int64_t(15); }
     // row r of group (b, kvh) -> index of its query vector in q [B][T][Hq][d]
     // (and of its output in out, same layout); rows are ordered (t, head)
     __host__ __device__ int64_t qrow(int b, int kvh, int r) const {

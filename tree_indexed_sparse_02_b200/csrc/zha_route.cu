@@ -93,7 +93,8 @@ __device__ __forceinline__ int64_t group_len(const Geo &g, const int32_t *lens, 
 // ----------------------------------------------------------------------- init
 
 __global__ void route_init_kernel(Geo g, uint32_t *maxkey, uint32_t *minkey, uint32_t *done,
-                                  const int32_t *lens, int32_t *status) {
+                                  uint32_t *gctr, unsigned long long *lookback, const int32_t *lens,
+                                  int32_t *status) {
     const int grp = blockIdx.x;
     if (threadIdx.x == 0) {
         const int64_t N = (int64_t)lens[grp / g.Hkv] - g.lag;
@@ -103,8 +104,17 @@ __global__ void route_init_kernel(Geo g, uint32_t *maxkey, uint32_t *minkey, uin
         const int64_t at = ((int64_t)(i / g.G) * g.groups() + grp) * g.G + i % g.G;
         maxkey[at] = 0u;
         minkey[at] = 0xffffffffu;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) gctr[at * 4 + k] = 0u;
     }
     for (int l = threadIdx.x; l < g.L; l += blockDim.x) done[(int64_t)l * g.groups() + grp] = 0u;
+    // the joins' look-back words of this group, every level
+    int64_t off = 0;
+    for (int l = 1; l <= g.L; ++l) {
+        const int64_t chunks = (g.capv[l] + kJoinChunk - 1) / kJoinChunk;
+        for (int64_t i = threadIdx.x; i < chunks; i += blockDim.x) lookback[off + grp * chunks + i] = 0ull;
+        off += (int64_t)g.groups() * chunks;
+    }
 }
 
 // ---------------------------------------------------------------------- score
@@ -462,13 +472,14 @@ __device__ __forceinline__ float e4m3_value(uint32_t byte) {
 // Scoring against MX-FP8 summaries (E4M3 bytes, one power-of-two scale per 32
 // coordinates of a plane) with E4M3 tensor-core MMAs, so the summaries are
 // never converted: mma.sync m16n8k32 (A = planes, B = query heads, one MMA
-// per 32-coordinate block). Each query head is held as two E4M3 terms with
-// one power-of-two scale per head: q ~ 2^e (hi + lo / 16), hi the nearest
-// E4M3 of q / 2^e (e the smallest with max|q| <= 448 * 2^e), lo that of the
-// remainder times 16 -- about 8 significant bits, the precision of bf16.
+// per 32-coordinate block and query term). Each query head is held as two
+// E4M3 terms with one power-of-two scale per head: q ~ 2^e (hi + lo), hi the
+// nearest E4M3 of q / 2^e (e the smallest with max|q| <= 448 * 2^e), lo that
+// of the remainder -- about 8 significant bits, the precision of bf16.
 // Each lane reads 8 contiguous bytes of a row per block, so an MMA sees one
-// plane scale per row; the block's two MMAs (hi, lo) are combined and scaled
-// into the plane sums, and the head scale is applied once at the end.
+// plane scale per row; the block's two MMAs (hi, then lo into the same
+// accumulator) are scaled into the plane sums, and the head scale is applied
+// once at the end.
 template <int D, int MT, int NT, int U>
 __global__ void __launch_bounds__(kScoreWarps * 32)
 score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias, const __nv_bfloat16 *q,
@@ -523,7 +534,7 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
                 for (int e = 0; e < 4; ++e) {
                     const float x = scalbnf(v[kp][4 * w2 + e], -ex);
                     const uint32_t bh = e4m3_rn(x);
-                    const uint32_t bl = e4m3_rn((x - e4m3_value(bh)) * 16.f);
+                    const uint32_t bl = e4m3_rn(x - e4m3_value(bh));
                     hi |= bh << (8 * e);
                     lo |= bl << (8 * e);
                 }
@@ -608,17 +619,17 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
                 for (int kp = 0; kp < KP; ++kp) {
                     const uint2 &xa = ra[u][mt][kp], &xb = rb[u][mt][kp];
                     // 2^(byte - 127) of this block for rows r0 and r1
-                    const float s0 = __uint_as_float(((sa[u][mt] >> (8 * kp)) & 0xffu) << 23);
-                    const float s1 = __uint_as_float(((sb[u][mt] >> (8 * kp)) & 0xffu) << 23);
+                    const float s0 = __uint_as_float(__byte_perm(sa[u][mt], 0u, 0x4440u + kp) << 23);
+                    const float s1 = __uint_as_float(__byte_perm(sb[u][mt], 0u, 0x4440u + kp) << 23);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        float th[4] = {0.f, 0.f, 0.f, 0.f}, tl[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_e4m3_16832(th, xa.x, xb.x, xa.y, xb.y, bhi[nt][kp][0], bhi[nt][kp][1]);
-                        mma_e4m3_16832(tl, xa.x, xb.x, xa.y, xb.y, blo[nt][kp][0], blo[nt][kp][1]);
-                        acc[nt][0] = fmaf(s0, fmaf(tl[0], 0.0625f, th[0]), acc[nt][0]);
-                        acc[nt][1] = fmaf(s0, fmaf(tl[1], 0.0625f, th[1]), acc[nt][1]);
-                        acc[nt][2] = fmaf(s1, fmaf(tl[2], 0.0625f, th[2]), acc[nt][2]);
-                        acc[nt][3] = fmaf(s1, fmaf(tl[3], 0.0625f, th[3]), acc[nt][3]);
+                        float tq[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_e4m3_16832(tq, xa.x, xb.x, xa.y, xb.y, bhi[nt][kp][0], bhi[nt][kp][1]);
+                        mma_e4m3_16832(tq, xa.x, xb.x, xa.y, xb.y, blo[nt][kp][0], blo[nt][kp][1]);
+                        acc[nt][0] = fmaf(s0, tq[0], acc[nt][0]);
+                        acc[nt][1] = fmaf(s0, tq[1], acc[nt][1]);
+                        acc[nt][2] = fmaf(s1, tq[2], acc[nt][2]);
+                        acc[nt][3] = fmaf(s1, tq[3], acc[nt][3]);
                     }
                 }
                 const float b0 = ba[u][mt], b1 = bb[u][mt];
@@ -732,7 +743,8 @@ __global__ void score_f32_kernel(Geo g, const float *mu, const float *bias, cons
 constexpr int kSelThreads = 1024;
 constexpr int kDigitBits = 12;
 constexpr int kBuckets = 1 << kDigitBits;
-constexpr int kMaxTies = 1024;
+constexpr int kMaxTies = kSelList;
+static_assert(kBuckets == kSelBuckets, "select histogram size");
 // masses e^{E - max} in (0, 1] are summed exactly as integers in units of
 // 2^-31 (per-candidate rounding error <= 2^-32)
 constexpr float kMassScale = 2147483648.0f;
@@ -889,16 +901,14 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
                 add_block(m1, e1);
             }
             __syncthreads();
-            constexpr int per = kBuckets / kSelThreads;
+            const int per = kBuckets / (int)blockDim.x;
             unsigned long long mine = 0ull;
-#pragma unroll
             for (int j = 0; j < per; ++j)
                 mine += ((unsigned long long)sh.hist_hi[tid * per + j] << 32) | sh.hist_lo[tid * per + j];
             unsigned long long z;
             const unsigned long long excl = block_exclusive_scan<unsigned long long>(mine, sh.red, &z);
             const unsigned long long target = (unsigned long long)ceil((double)p * (double)z);
             unsigned long long run = excl;
-#pragma unroll
             for (int j = 0; j < per; ++j) {
                 const int bk = tid * per + j;
                 const unsigned long long hgt = ((unsigned long long)sh.hist_hi[bk] << 32) | sh.hist_lo[bk];
@@ -1000,9 +1010,8 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
             first = false;
         }
         // crossing digit: running mass from digit 0 (best) upward first reaches target
-        constexpr int per = kBuckets / kSelThreads;
+        const int per = kBuckets / (int)blockDim.x;
         unsigned long long mine = 0ull;
-#pragma unroll
         for (int j = 0; j < per; ++j)
             mine += ((unsigned long long)sh.hist_hi[tid * per + j] << 32) | sh.hist_lo[tid * per + j];
         unsigned long long tot;
@@ -1010,7 +1019,6 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
         unsigned long long run = sh.above + excl;
         const unsigned long long target = sh.target;
         __syncthreads();
-#pragma unroll
         for (int j = 0; j < per; ++j) {
             const int dgt = tid * per + j;
             const unsigned long long hgt = ((unsigned long long)sh.hist_hi[dgt] << 32) | sh.hist_lo[dgt];
@@ -1085,59 +1093,12 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
     return (int)block_sum<unsigned long long>((unsigned long long)kept, sh.red);
 }
 
-// Joins the G heads' kept bitmaps of a group (bits[h][blk], byte per 8
-// candidates) into per-candidate head masks (written to kept[]) and compacts
-// the candidates some head kept, in order, into (out_idx, out_mask). Returns
-// the number written (every thread). Rows are padded to 8 entries.
-__device__ int64_t join_and_compact(const uint8_t *bits, int64_t bits_stride, int G,
-                                    uint32_t *kept, const int32_t *cand, int64_t n,
-                                    int32_t *out_idx, uint32_t *out_mask, unsigned long long *red) {
-    const int64_t nblk = (n + 7) >> 3;
-    int64_t run = 0;
-    for (int64_t base = 0; base < nblk; base += blockDim.x) {
-        const int64_t blk = base + threadIdx.x;
-        uint32_t km[8];
-#pragma unroll
-        for (int v = 0; v < 8; ++v) km[v] = 0u;
-        if (blk < nblk) {
-            for (int h = 0; h < G; ++h) {
-                const uint32_t b = __ldcg(bits + h * bits_stride + blk);
-#pragma unroll
-                for (int v = 0; v < 8; ++v) km[v] |= ((b >> v) & 1u) << h;
-            }
-            uint4 *kp = reinterpret_cast<uint4 *>(kept + (blk << 3));
-            kp[0] = make_uint4(km[0], km[1], km[2], km[3]);
-            kp[1] = make_uint4(km[4], km[5], km[6], km[7]);
-        }
-        int cnt = 0;
-#pragma unroll
-        for (int v = 0; v < 8; ++v) cnt += km[v] != 0u;
-        unsigned long long tot;
-        int64_t o = run + (int64_t)block_exclusive_scan<unsigned long long>((unsigned long long)cnt, red, &tot);
-        if (cnt) {
-            const int4 c0 = *reinterpret_cast<const int4 *>(cand + (blk << 3));
-            const int4 c1 = *reinterpret_cast<const int4 *>(cand + (blk << 3) + 4);
-            const int32_t cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-                if (km[v]) {
-                    out_idx[o] = cv[v];
-                    out_mask[o] = km[v];
-                    ++o;
-                }
-        }
-        run += (int64_t)tot;
-    }
-    return run;
-}
-
 __global__ void __launch_bounds__(kSelThreads)
-select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t *level_kept,
-              zha_selection sel) {
+select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t *level_kept) {
     __shared__ SelShared sh;
     const int h = blockIdx.x, grp = blockIdx.y;
     const int64_t capv = g.capv[level];
-    const int64_t bstride = capv >> 3;  // bytes of one head's bitmap
+    const int64_t bstride = g.bits_stride(level);  // bytes of one row's bitmap
     const int64_t n = lw.count[grp];
     const uint32_t bit = 1u << h;
     const uint32_t *cmask = lw.cmask + grp * capv;
@@ -1164,31 +1125,386 @@ select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t 
         },
         [&](int64_t blk, uint32_t kb) { mybits[blk] = (uint8_t)kb; },
         [&](int64_t i) { mybits[i >> 3] |= (uint8_t)(1u << (i & 7)); });
-    if (level_kept && threadIdx.x == 0) {
-        const int b = grp / g.Hkv, kvh = grp % g.Hkv;
-        level_kept[((int64_t)grp * g.G + h) * g.L + (level - 1)] = nk;
+    if (level_kept && threadIdx.x == 0) level_kept[((int64_t)grp * g.G + h) * g.L + (level - 1)] = nk;
+}
+
+// ------------------------------------------------- selection over several CTAs per row
+
+constexpr int kSplitThreads = 256;
+constexpr int kSplitMinSlice = 4096;                  // candidates per CTA, at least
+constexpr long long kSpinCycles = 2000000000LL;       // about a second: a wait that long is an error
+
+struct SplitWs {
+    unsigned long long *hist;   // [rows][kSelBuckets], left zeroed
+    int32_t *lidx;              // [rows][kSelList]
+    uint32_t *lkey;
+    uint32_t *ctr;              // [L][rows][4]: arrivals, list count, kept count
+};
+
+// Arrive at a counter shared by the CTAs of one row and wait, bounded, until
+// it reaches target. On timeout the status is set and false returned (the
+// results of the call are then invalid; nothing waits forever).
+__device__ bool row_barrier(uint32_t *ctr, uint32_t target, int32_t *status, int *ok_sh) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ctr, 1u);
+        const long long t0 = clock64();
+        int ok = 1;
+        while (*reinterpret_cast<volatile uint32_t *>(ctr) < target) {
+            if (clock64() - t0 > kSpinCycles) {
+                set_status(status, ZHA_ERR_TIMEOUT);
+                ok = 0;
+                break;
+            }
+            __nanosleep(64);
+        }
+        __threadfence();
+        *ok_sh = ok;
     }
-    // the last of the group's G CTAs joins the heads' bitmaps and compacts
-    __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) sh.last = atomicAdd(&lw.done[grp], 1u) == (uint32_t)(g.G - 1);
+    return *ok_sh != 0;
+}
+
+// The selection of select_kernel with one row's candidates spread over the
+// gridDim.x CTAs of (blockIdx.y = row, blockIdx.z = group): each CTA builds
+// the mass histogram of its slice and adds it to the row's global histogram;
+// after a barrier every CTA finds the same crossing bucket, keeps its slice's
+// members below it and lists the crossing bucket's members; after a second
+// barrier the row's first CTA orders that list and finalises the row. The
+// grid is sized on the host so that all its CTAs can be resident at once,
+// and the row's CTAs are consecutive in launch order.
+__global__ void __launch_bounds__(kSplitThreads, 4)
+select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t *level_kept,
+                    SplitWs sw, int32_t *status) {
+    __shared__ SelShared sh;
+    __shared__ int ok_sh;
+    __shared__ int nk_sh;
+    const int sidx = blockIdx.x, S = gridDim.x, h = blockIdx.y, grp = blockIdx.z;
+    const int tid = threadIdx.x;
+    const int64_t step = blockDim.x;
+    const int64_t capv = g.capv[level];
+    const int64_t bstride = g.bits_stride(level);
+    const int64_t n = lw.count[grp];
+    const int64_t nblk = (n + 7) >> 3;
+    const int64_t blo = nblk * sidx / S, bhi = nblk * (sidx + 1) / S;
+    const int64_t row = (int64_t)grp * g.G + h;
+    const uint32_t bit = 1u << h;
+    const uint32_t *cmask = lw.cmask + grp * capv;
+    const float *sc = lw.scores + row * capv;
+    uint8_t *mybits = keptbits + row * bstride;
+    const uint32_t kmax = lw.maxkey[row], kmin = lw.minkey[row];
+    uint32_t *ctr = sw.ctr + (((int64_t)(level - 1) * g.groups() + grp) * g.G + h) * 4;
+    unsigned long long *gh = sw.hist + row * kBuckets;
+    auto load8 = [&](int64_t blk, float (&e)[8]) -> uint32_t {
+        const int64_t i0 = blk << 3;
+        const float4 e0 = __ldg(reinterpret_cast<const float4 *>(sc + i0));
+        const float4 e1 = __ldg(reinterpret_cast<const float4 *>(sc + i0) + 1);
+        const uint4 m0 = __ldg(reinterpret_cast<const uint4 *>(cmask + i0));
+        const uint4 m1 = __ldg(reinterpret_cast<const uint4 *>(cmask + i0) + 1);
+        e[0] = e0.x; e[1] = e0.y; e[2] = e0.z; e[3] = e0.w;
+        e[4] = e1.x; e[5] = e1.y; e[6] = e1.z; e[7] = e1.w;
+        const uint32_t mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+        uint32_t mb = 0u;
+#pragma unroll
+        for (int v = 0; v < 8; ++v) mb |= ((mm[v] & bit) != 0u && i0 + v < n) ? (1u << v) : 0u;
+        return mb;
+    };
+    auto store8 = [&](int64_t blk, uint32_t kb) { mybits[blk] = (uint8_t)kb; };
+    auto add_kept = [&](int64_t i) { mybits[i >> 3] |= (uint8_t)(1u << (i & 7)); };
+    auto finalise = [&](int nk) {
+        if (level_kept && tid == 0) level_kept[row * g.L + (level - 1)] = nk;
+    };
+
+    const float m = key_to_float(kmax);
+    const float W = (float)kBuckets / fminf(m - key_to_float(kmin), kMassRange);
+    if (kmax == 0u || p >= 1.f) {
+        // no member, or every member kept: each slice stores its membership
+        int kept = 0;
+        for (int64_t blk = blo + tid; blk < bhi; blk += step) {
+            float e[8];
+            const uint32_t mb = kmax ? load8(blk, e) : 0u;
+            store8(blk, mb);
+            kept += __popc(mb);
+        }
+        kept = (int)block_sum<unsigned long long>((unsigned long long)kept, sh.red);
+        if (tid == 0 && kept) atomicAdd(&ctr[2], (uint32_t)kept);
+        if (!row_barrier(&ctr[0], (uint32_t)S, status, &ok_sh)) return;
+        if (sidx == 0) finalise((int)*reinterpret_cast<volatile uint32_t *>(&ctr[2]));
+        return;
+    }
+    if (kmax == kmin || !(W < 1e30f)) {
+        // equal scores (or a range too narrow to bucket): the row on one CTA
+        if (sidx != 0) return;
+        const int nk = topp_core(sh, n, p, kmax, kmin, load8, store8, add_kept);
+        finalise(nk);
+        return;
+    }
+    auto bucket = [&](float e) -> int {
+        const float x = (m - e) * W;
+        return x < (float)(kBuckets - 1) ? (int)x : kBuckets - 1;
+    };
+    // 1. this slice's mass histogram into the row's global histogram
+    for (int i = tid; i < kBuckets; i += blockDim.x) sh.hist_lo[i] = sh.hist_hi[i] = 0u;
     __syncthreads();
-    if (!sh.last) return;
-    __threadfence();
-    const uint8_t *gbits = keptbits + (int64_t)grp * g.G * bstride;
-    uint32_t *kept = lw.kept + grp * capv;
+    auto add_block = [&](uint32_t mb, const float (&e)[8]) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+            if ((mb >> v) & 1u) hist_add(sh.hist_lo, sh.hist_hi, bucket(e[v]), fixed_mass(e[v], m));
+    };
+    for (int64_t blk = blo + tid; blk < bhi; blk += 2 * step) {
+        float e0[8], e1[8];
+        const uint32_t m0 = load8(blk, e0);
+        const uint32_t m1 = blk + step < bhi ? load8(blk + step, e1) : 0u;
+        add_block(m0, e0);
+        add_block(m1, e1);
+    }
+    __syncthreads();
+    for (int i = tid; i < kBuckets; i += blockDim.x) {
+        const unsigned long long v = ((unsigned long long)sh.hist_hi[i] << 32) | sh.hist_lo[i];
+        if (v) atomicAdd(&gh[i], v);
+    }
+    if (!row_barrier(&ctr[0], (uint32_t)S, status, &ok_sh)) return;
+    // 2. the crossing bucket (every CTA of the row computes the same); the row's
+    // histogram comes in with all loads in flight at once
+    constexpr int per = kBuckets / kSplitThreads;
+    unsigned long long hv[per];
+#pragma unroll
+    for (int j = 0; j < per; ++j) hv[j] = __ldcg(&gh[tid * per + j]);
+    unsigned long long mine = 0ull;
+#pragma unroll
+    for (int j = 0; j < per; ++j) mine += hv[j];
+    unsigned long long z;
+    if (tid == 0) {
+        sh.digit = kBuckets - 1;
+        sh.above = 0ull;
+    }
+    const unsigned long long excl = block_exclusive_scan<unsigned long long>(mine, sh.red, &z);
+    const unsigned long long target = (unsigned long long)ceil((double)p * (double)z);
+    unsigned long long run = excl;
+#pragma unroll
+    for (int j = 0; j < per; ++j) {
+        const int bk = tid * per + j;
+        const unsigned long long hgt = hv[j];
+        if (hgt && run < target && run + hgt >= target) {
+            sh.digit = (uint32_t)bk;
+            sh.above = run;
+        }
+        run += hgt;
+    }
+    __syncthreads();
+    const int bstar = (int)sh.digit;
+    const unsigned long long above = sh.above;
+    // 3. keep this slice's members below the crossing bucket; list the bucket's members
+    int kept = 0;
+    for (int64_t blk = blo + tid; blk < bhi; blk += step) {
+        float e[8];
+        const uint32_t mb = load8(blk, e);
+        uint32_t kb = 0u;
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            if (!((mb >> v) & 1u)) continue;
+            const int bk = bucket(e[v]);
+            if (bk < bstar) {
+                kb |= 1u << v;
+            } else if (bk == bstar) {
+                const uint32_t slot = atomicAdd(&ctr[1], 1u);
+                if (slot < (uint32_t)kSelList) {
+                    sw.lidx[row * kSelList + slot] = (int32_t)((blk << 3) + v);
+                    sw.lkey[row * kSelList + slot] = ordered_key(e[v]);
+                }
+            }
+        }
+        store8(blk, kb);
+        kept += __popc(kb);
+    }
+    kept = (int)block_sum<unsigned long long>((unsigned long long)kept, sh.red);
+    if (tid == 0 && kept) atomicAdd(&ctr[2], (uint32_t)kept);
+    if (!row_barrier(&ctr[0], 2u * (uint32_t)S, status, &ok_sh)) return;
+    // 4. every CTA has read the histogram: clear this CTA's share for the next use
+    for (int i = (int)((int64_t)kBuckets * sidx / S) + tid; i < (int)((int64_t)kBuckets * (sidx + 1) / S);
+         i += blockDim.x)
+        gh[i] = 0ull;
+    if (sidx != 0) return;
+    // 5. the row's first CTA: the crossing bucket in (score desc, index asc) order
+    const uint32_t nl = *reinterpret_cast<volatile uint32_t *>(&ctr[1]);
+    if (nl <= (uint32_t)kSelList) {
+        for (uint32_t j = tid; j < nl; j += blockDim.x) {
+            sh.ties[j] = __ldcg(&sw.lidx[row * kSelList + j]);
+            sh.tkey[j] = __ldcg(&sw.lkey[row * kSelList + j]);
+        }
+        __syncthreads();
+        for (uint32_t j = tid; j < nl; j += blockDim.x) {
+            const uint32_t kj = sh.tkey[j];
+            const int32_t ij = sh.ties[j];
+            int rank = 0;
+            for (uint32_t w = 0; w < nl; ++w) {
+                const uint32_t kw = sh.tkey[w];
+                rank += (kw > kj) || (kw == kj && sh.ties[w] < ij);
+            }
+            sh.sorted_ties[rank] = (int)j;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int added = 0;
+            unsigned long long cum = above;
+            for (uint32_t r = 0; r < nl && cum < target; ++r) {
+                const int j = sh.sorted_ties[r];
+                const int64_t i = sh.ties[j];
+                // other CTAs wrote neighbouring bytes: set the bit with a word atomic
+                const uintptr_t a = reinterpret_cast<uintptr_t>(mybits + (i >> 3));
+                atomicOr(reinterpret_cast<uint32_t *>(a & ~uintptr_t(3)), 1u << (((a & 3u) << 3) + (i & 7)));
+                ++added;
+                cum += fixed_mass(key_to_float(sh.tkey[j]), m);
+            }
+            nk_sh = (int)*reinterpret_cast<volatile uint32_t *>(&ctr[2]) + added;
+        }
+        __syncthreads();
+        finalise(nk_sh);
+        return;
+    }
+    // too many members in the crossing bucket (near-equal scores): the row on this CTA
+    const int nk = topp_core(sh, n, p, kmax, kmin, load8, store8, add_kept);
+    finalise(nk);
+}
+
+// ------------------------------------------------------------------ join
+
+constexpr int kJoinThreads = kJoinChunk / 8;       // 8 candidates per thread
+constexpr unsigned long long kLbAggregate = 1ull << 62, kLbInclusive = 2ull << 62;
+constexpr unsigned long long kLbValue = (1ull << 62) - 1;
+
+// The G rows' kept bitmaps of a group joined into per-candidate row masks
+// (written to kept[]), and the candidates some row kept compacted, in order,
+// into the next level's parent list (or, at level 1, the selection). One CTA
+// per chunk of kJoinChunk candidates; the output offset of a chunk is the
+// number kept by the chunks before it, found by looking back over their
+// published counts (each chunk publishes its own count at once and its
+// running total once known; every wait is bounded).
+__global__ void __launch_bounds__(kJoinThreads)
+join_kernel(Geo g, LevelWs lw, const uint8_t *keptbits, int level, zha_selection sel,
+            unsigned long long *lb, int32_t *status) {
+    __shared__ __align__(16) uint8_t sbits[32][kJoinChunk / 8];
+    __shared__ unsigned long long red[kJoinThreads / 32];
+    __shared__ unsigned long long s_excl;
+    const int chunk = blockIdx.x, grp = blockIdx.y;
+    const int tid = threadIdx.x;
+    const int64_t capv = g.capv[level];
+    const int64_t bstride = g.bits_stride(level);
+    const int64_t n = lw.count[grp];
+    const int64_t nchunks = (n + kJoinChunk - 1) / kJoinChunk;
+    if (n <= 0) {
+        if (chunk == 0 && tid == 0) {
+            if (level > 1)
+                lw.pcount[grp] = 0;
+            else
+                sel.count[grp] = 0;
+        }
+        return;
+    }
+    if (chunk >= nchunks) return;
+    unsigned long long *mylb = lb + (int64_t)grp * gridDim.x;
+    const int64_t blk0 = (int64_t)chunk * (kJoinChunk / 8);
+    const int nb = (int)min64(kJoinChunk / 8, ((n + 7) >> 3) - blk0);
+    // 1. the rows' bitmap bytes of this chunk, 16 bytes per load
+    const uint8_t *gbits = keptbits + (int64_t)grp * g.G * bstride + blk0;
+    constexpr int kVec = kJoinChunk / 8 / 16;         // 16-byte words per row and chunk
+    for (int i = tid; i < g.G * kVec; i += blockDim.x) {
+        const int h = i / kVec, j = i % kVec;
+        uint4 w = make_uint4(0, 0, 0, 0);
+        if (j * 16 < nb && blk0 + j * 16 + 16 <= bstride)
+            w = __ldcg(reinterpret_cast<const uint4 *>(gbits + h * bstride) + j);
+        else if (j * 16 < nb) {
+            uint8_t tmp[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) tmp[k] = (blk0 + j * 16 + k < bstride) ? __ldcg(gbits + h * bstride + j * 16 + k) : 0;
+            w = *reinterpret_cast<const uint4 *>(tmp);
+        }
+        *reinterpret_cast<uint4 *>(&sbits[h][j * 16]) = w;
+    }
+    __syncthreads();
+    // 2. row masks of this thread's 8 candidates
+    uint32_t km[8];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) km[v] = 0u;
+    const bool mine = tid < nb;
+    if (mine) {
+        for (int h = 0; h < g.G; ++h) {
+            const uint32_t b = sbits[h][tid];
+#pragma unroll
+            for (int v = 0; v < 8; ++v) km[v] |= ((b >> v) & 1u) << h;
+        }
+        uint4 *kp = reinterpret_cast<uint4 *>(lw.kept + grp * capv + ((blk0 + tid) << 3));
+        kp[0] = make_uint4(km[0], km[1], km[2], km[3]);
+        kp[1] = make_uint4(km[4], km[5], km[6], km[7]);
+    }
+    int cnt = 0;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) cnt += km[v] != 0u;
+    unsigned long long total;
+    const unsigned long long local = block_exclusive_scan<unsigned long long>((unsigned long long)cnt, red, &total);
+    // 3. running total of the chunks before this one
+    if (tid == 0) {
+        unsigned long long excl = 0ull;
+        if (chunk == 0) {
+            __threadfence();
+            atomicExch(&mylb[0], kLbInclusive | total);
+        } else {
+            __threadfence();
+            atomicExch(&mylb[chunk], kLbAggregate | total);
+            const long long t0 = clock64();
+            for (int64_t pc = chunk - 1; pc >= 0;) {
+                const unsigned long long w = *reinterpret_cast<volatile unsigned long long *>(&mylb[pc]);
+                if ((w >> 62) == 0ull) {
+                    if (clock64() - t0 > kSpinCycles) {
+                        set_status(status, ZHA_ERR_TIMEOUT);
+                        break;
+                    }
+                    __nanosleep(32);
+                    continue;
+                }
+                excl += w & kLbValue;
+                if ((w >> 62) == 2ull) break;
+                --pc;
+            }
+            __threadfence();
+            atomicExch(&mylb[chunk], kLbInclusive | (excl + total));
+        }
+        s_excl = excl;
+    }
+    __syncthreads();
+    // 4. the kept candidates, in order
+    const int64_t base = (int64_t)s_excl + (int64_t)local;
+    int32_t *out_idx;
+    uint32_t *out_mask;
     if (level > 1) {
-        const int64_t m = join_and_compact(gbits, bstride, g.G, kept, lw.cand + grp * capv, n,
-                                           lw.plist + grp * g.cap[level], lw.pmask + grp * g.cap[level],
-                                           sh.red);
-        if (threadIdx.x == 0) lw.pcount[grp] = (int32_t)m;
+        out_idx = lw.plist + grp * g.cap[level];
+        out_mask = lw.pmask + grp * g.cap[level];
     } else {
-        const int64_t m = join_and_compact(gbits, bstride, g.G, kept, lw.cand + grp * capv, n,
-                                           sel.leaf_idx + grp * g.cap[1], sel.head_mask + grp * g.cap[1],
-                                           sh.red);
-        if (threadIdx.x == 0) sel.count[grp] = (int32_t)m;
+        out_idx = sel.leaf_idx + grp * g.cap[1];
+        out_mask = sel.head_mask + grp * g.cap[1];
     }
-    if (threadIdx.x == 0) lw.done[grp] = 0u;
+    if (mine && cnt) {
+        const int32_t *cand = lw.cand + grp * capv + ((blk0 + tid) << 3);
+        const int4 c0 = *reinterpret_cast<const int4 *>(cand);
+        const int4 c1 = *reinterpret_cast<const int4 *>(cand + 4);
+        const int32_t cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        int64_t o = base;
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+            if (km[v]) {
+                out_idx[o] = cv[v];
+                out_mask[o] = km[v];
+                ++o;
+            }
+    }
+    if (chunk == nchunks - 1 && tid == 0) {
+        const int32_t m = (int32_t)(s_excl + total);
+        if (level > 1)
+            lw.pcount[grp] = m;
+        else
+            sel.count[grp] = m;
+    }
 }
 
 __global__ void __launch_bounds__(kSelThreads)
@@ -1224,6 +1540,22 @@ select_sets_kernel(const float *scores, const int32_t *counts, int64_t stride, f
         [&](int64_t i) { kp[i] = 1; });
 }
 
+// CTAs of select_split_kernel that fit on the current device at once (0: none known)
+int64_t split_slots() {
+    static int64_t slots[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (slots[dev] == 0) {
+        int sms = 0, per_sm = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_split_kernel, kSplitThreads, 0) !=
+                cudaSuccess)
+            return 0;
+        slots[dev] = (int64_t)sms * per_sm;
+    }
+    return slots[dev];
+}
+
 }  // namespace
 
 cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const int32_t *lens,
@@ -1233,6 +1565,12 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                                         "score[l5]", "score[l6]", "score[l7]", "score[l8]"};
     static const char *select_names[] = {"", "select[l1]", "select[l2]", "select[l3]", "select[l4]",
                                          "select[l5]", "select[l6]", "select[l7]", "select[l8]"};
+    static const char *join_names[] = {"", "join[l1]", "join[l2]", "join[l3]", "join[l4]",
+                                       "join[l5]", "join[l6]", "join[l7]", "join[l8]"};
+    // look-back words of each level's join: [groups][chunks of that level]
+    int64_t lb_off[kMaxLevels + 2] = {};
+    for (int l = 1; l <= g.L; ++l)
+        lb_off[l + 1] = lb_off[l] + (int64_t)g.groups() * ((g.capv[l] + kJoinChunk - 1) / kJoinChunk);
     const int groups = g.groups();
     {
         ProfScope ps("route_init", st);
@@ -1240,7 +1578,9 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
         route_init_kernel<<<groups, 64, 0, st>>>(
             g, reinterpret_cast<uint32_t *>(base + g.ws_maxkey),
             reinterpret_cast<uint32_t *>(base + g.ws_minkey),
-            reinterpret_cast<uint32_t *>(base + g.ws_done), lens, status);
+            reinterpret_cast<uint32_t *>(base + g.ws_done),
+            reinterpret_cast<uint32_t *>(base + g.ws_gctr),
+            reinterpret_cast<unsigned long long *>(base + g.ws_lookback), lens, status);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -1266,9 +1606,9 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
     do { if (nt == 1) ZHA_SCORE_MX(D, MT, 1, U1); else if (nt == 2) ZHA_SCORE_MX(D, MT, 2, 2); \
          else ZHA_SCORE_MX(D, MT, 4, 1); } while (0)
                 if (g.d == 128) {
-                    if (mt == 1) ZHA_SCORE_MX_N(128, 1, 4); else ZHA_SCORE_MX_N(128, 2, 2);
+                    if (mt == 1) ZHA_SCORE_MX_N(128, 1, 2); else ZHA_SCORE_MX_N(128, 2, 2);
                 } else {
-                    if (mt == 1) ZHA_SCORE_MX_N(64, 1, 4); else ZHA_SCORE_MX_N(64, 2, 2);
+                    if (mt == 1) ZHA_SCORE_MX_N(64, 1, 2); else ZHA_SCORE_MX_N(64, 2, 2);
                 }
 #undef ZHA_SCORE_MX_N
 #undef ZHA_SCORE_MX
@@ -1338,8 +1678,32 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
         {
             ProfScope ps(select_names[level], st);
             uint8_t *keptbits = reinterpret_cast<uint8_t *>(static_cast<char *>(ws) + g.ws_keptbits[level]);
-            select_kernel<<<dim3(g.G, groups), kSelThreads, 0, st>>>(g, lw, keptbits, level,
-                                                                     p_levels[level - 1], sel.level_kept, sel);
+            // rows with many candidates: several CTAs per row, as many as can be resident together
+            const int64_t rows = (int64_t)g.G * groups;
+            const int S = (int)min64(capv / kSplitMinSlice, split_slots() / rows);
+            if (S >= 2) {
+                char *base = static_cast<char *>(ws);
+                const SplitWs sw{reinterpret_cast<unsigned long long *>(base + g.ws_ghist),
+                                 reinterpret_cast<int32_t *>(base + g.ws_glidx),
+                                 reinterpret_cast<uint32_t *>(base + g.ws_glkey),
+                                 reinterpret_cast<uint32_t *>(base + g.ws_gctr)};
+                select_split_kernel<<<dim3(S, g.G, groups), kSplitThreads, 0, st>>>(
+                    g, lw, keptbits, level, p_levels[level - 1], sel.level_kept, sw, status);
+            } else {
+                select_kernel<<<dim3(g.G, groups), kSelThreads, 0, st>>>(g, lw, keptbits, level,
+                                                                         p_levels[level - 1], sel.level_kept);
+            }
+        }
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        {
+            ProfScope ps(join_names[level], st);
+            const uint8_t *keptbits = reinterpret_cast<const uint8_t *>(static_cast<char *>(ws) + g.ws_keptbits[level]);
+            const int64_t chunks = (capv + kJoinChunk - 1) / kJoinChunk;
+            unsigned long long *lb = reinterpret_cast<unsigned long long *>(static_cast<char *>(ws) + g.ws_lookback) +
+                                     lb_off[level];
+            join_kernel<<<dim3((unsigned)chunks, groups), kJoinThreads, 0, st>>>(g, lw, keptbits, level, sel, lb,
+                                                                                status);
         }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
