@@ -493,7 +493,7 @@ def traffic_for(kernel: str, alg_bytes_per_launch: float):
         with open(path) as f:
             d = json.load(f)
         ent = d["kernels"][kernel]
-        if ent.get("source_sha") != source_sha():
+        if ent.get("source_sha", d.get("source_sha")) != source_sha():
             return None
         return ent["dram_bytes_per_alg_byte"] * alg_bytes_per_launch
     except Exception:

@@ -177,8 +177,11 @@ ZHA_API zha_status zha_tree_level_offsets(const zha_config *cfg, int32_t level, 
 
 /* ZHA_SUMMARY_MXFP8 only: byte offset of level l's block scales,
  *   scale [batch][n_kv_heads][cap_l][n_refs][head_dim / 32]  uint8 = e + 127,
- * mu_r[k] = e4m3(mu byte k) * 2^(scale[k / 32] - 127). ZHA_ERR_INVALID_ARG
- * for the native format. */
+ * mu_r[k] = e4m3(mu byte o(k)) * 2^(scale[k / 32] - 127), where a plane's
+ * head_dim bytes are stored permuted so that a scoring lane fetches its bytes
+ * of two adjacent blocks with one 16-byte load: with b = k / 32, w = k % 32,
+ *   o(k) = 64 (b / 2) + 16 ((w % 16) / 4) + 8 (b % 2) + 4 (w / 16) + w % 4.
+ * ZHA_ERR_INVALID_ARG for the native format. */
 ZHA_API zha_status zha_tree_level_scales(const zha_config *cfg, int32_t level, size_t *scale_off);
 
 /* Bytes of scratch every call below may use (routing state + split-K partials). */

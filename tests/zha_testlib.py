@@ -32,10 +32,22 @@ def storage(w: Workload) -> str:
     return "bf16" if w.dtype == "bf16" else "f32"
 
 
+def mx_byte_offsets(d: int) -> np.ndarray:
+    """Byte position of each coordinate in a stored MX-FP8 row (the order
+    include/zha.h gives): block b = k // 32, w = k % 32 sits at
+    64 (b // 2) + 16 ((w % 16) // 4) + 8 (b % 2) + 4 (w // 16) + w % 4."""
+    k = np.arange(d)
+    b, w = k // 32, k % 32
+    return 64 * (b // 2) + 16 * ((w % 16) // 4) + 8 * (b % 2) + 4 * (w // 16) + w % 4
+
+
 def mx_decode(mu8: torch.Tensor, scales: torch.Tensor) -> np.ndarray:
     """Values of MX-FP8 planes read back from the device: E4M3 bytes [..., d]
-    times 2^(scale byte - 127) per 32 coordinates, in float64."""
-    v = mu8.contiguous().view(torch.float8_e4m3fn).to(torch.float64)
+    (stored in the permuted order) times 2^(scale byte - 127) per 32
+    coordinates, in float64, in coordinate order."""
+    d = mu8.shape[-1]
+    perm = torch.from_numpy(mx_byte_offsets(d)).to(mu8.device)
+    v = mu8.contiguous()[..., perm].contiguous().view(torch.float8_e4m3fn).to(torch.float64)
     sc = torch.exp2(scales.to(torch.float64) - 127.0).repeat_interleave(32, dim=-1)
     return (v * sc).cpu().numpy()
 

@@ -226,8 +226,11 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
 
-    const int grp = blockIdx.y, split = blockIdx.x, S = gridDim.x;
-    const int rbase = blockIdx.z * 16;     // this CTA's 16 query rows of the group
+    // the 16-row tiles of a (group, split) are adjacent in launch order, so
+    // with more than 16 rows their CTAs stream the same K/V at about the same
+    // time and the second read comes from L2
+    const int grp = blockIdx.z, split = blockIdx.y, S = gridDim.y;
+    const int rbase = blockIdx.x * 16;     // this CTA's 16 query rows of the group
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gq = lane >> 2, t = lane & 3;
@@ -253,29 +256,31 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     const int ntiles = (tp.nv + kTile - 1) / kTile;
     const int t_lo = (int)((int64_t)ntiles * split / S), t_hi = (int)((int64_t)ntiles * (split + 1) / S);
 
-    // Cache positions and head masks of the next tiles, resolved one iteration
-    // ahead of their copies (by threads 0..63, one row each) so that the
-    // lookups' latency overlaps a whole tile of compute.
+    // Each warp owns rows 16 w .. 16 w + 15 of every tile: it looks up their
+    // cache positions and head masks (one iteration ahead of their copies, so
+    // that the lookups' latency overlaps a tile of compute), copies them, and
+    // computes on them, so the pipeline needs no block-wide barrier.
     constexpr int kSlots = kStages + 1;
     __shared__ int spos[kSlots][kTile];
     __shared__ uint32_t smask[kSlots][kTile];
     auto resolve = [&](int tile, int slot) {
-        if (threadIdx.x < kTile) {
-            const int v = tile * kTile + threadIdx.x;
+        if (lane < 16) {
+            const int row = warp * 16 + lane;
+            const int v = tile * kTile + row;
             int pos;
             uint32_t m;
             tp.at(v, pos, m, status);
-            spos[slot][threadIdx.x] = pos;
-            smask[slot][threadIdx.x] = v < tp.nv ? m : 0u;
+            spos[slot][row] = pos;
+            smask[slot][row] = v < tp.nv ? m : 0u;
         }
     };
-    // 16 threads per row of a tile: one 16-byte chunk of K and of V each
+    // the warp's 16 rows, one 16-byte chunk of K and of V per lane and step
     auto issue = [&](int tile, int stage, int slot) {
         const uint32_t kb = sbase + stage * STAGE_B, vb = kb + TILE_B;
 #pragma unroll
-        for (int k = 0; k < kTile * CH / (kAttnWarps * 32); ++k) {
-            const int c = threadIdx.x + k * kAttnWarps * 32;
-            const int row = c / CH, ch = c % CH;
+        for (int k = 0; k < 16 * CH / 32; ++k) {
+            const int c = lane + k * 32;
+            const int row = warp * 16 + c / CH, ch = c % CH;
             const int pos = spos[slot][row];
             const bool valid = tile * kTile + row < tp.nv;
             const uint32_t off = row * ROWB + ((ch ^ (row & 7)) << 4);
@@ -296,7 +301,7 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
 #pragma unroll
     for (int st = 0; st < kStages; ++st)
         if (t_lo + st < t_hi) resolve(t_lo + st, st);
-    __syncthreads();
+    __syncwarp();
 #pragma unroll
     for (int st = 0; st < kStages - 1; ++st) {
         if (t_lo + st < t_hi) issue(t_lo + st, st, st);
@@ -304,7 +309,10 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     }
     for (int it = 0; t_lo + it < t_hi; ++it) {
         cp_async_wait<kStages - 2>();
-        __syncthreads();
+        // contiguous (dense) streams keep the warps in step, so that the CTA's
+        // copies of a tile hit the same DRAM pages together
+        if (dense) __syncthreads();
+        else __syncwarp();
         {
             const int nt = t_lo + it + kStages - 1;
             if (nt < t_hi) issue(nt, (it + kStages - 1) % kStages, (it + kStages - 1) % kSlots);
@@ -453,8 +461,11 @@ attn_simt_kernel(Geo g, const T *q, const T *K, const T *V, const int32_t *lens,
     __shared__ float qs[16][D];
     __shared__ float sm_m[kAttnWarps][16], sm_l[kAttnWarps][16];
     __shared__ float sm_o[kAttnWarps][16][D];
-    const int grp = blockIdx.y, split = blockIdx.x, S = gridDim.x;
-    const int rbase = blockIdx.z * 16;     // this CTA's 16 query rows of the group
+    // the 16-row tiles of a (group, split) are adjacent in launch order, so
+    // with more than 16 rows their CTAs stream the same K/V at about the same
+    // time and the second read comes from L2
+    const int grp = blockIdx.z, split = blockIdx.y, S = gridDim.y;
+    const int rbase = blockIdx.x * 16;     // this CTA's 16 query rows of the group
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int G = min(16, g.G - rbase);
@@ -552,21 +563,24 @@ attn_simt_kernel(Geo g, const T *q, const T *K, const T *V, const int32_t *lens,
 }
 
 // Log-sum-exp merge of the split-K partials: one block per (group, head).
+constexpr int kMergeLanes = 4;     // threads per output coordinate, each summing every 4th split
+
 template <typename T>
 __global__ void attn_merge_kernel(Geo g, int S, const float *part_ml, const float *part_o,
                                   T *out) {
-    // One block per (group, head): the splits' weights 2^(m_s - M) are formed
-    // in parallel (shared memory), then each thread sums one output coordinate
-    // over the splits with independent loads in flight.
-    extern __shared__ float wsplit[];                 // [S]
+    // One block per (group, row), kMergeLanes x head_dim threads: the splits'
+    // weights 2^(m_s - M) are formed in parallel (shared memory), then each
+    // coordinate's weighted sum is split over kMergeLanes threads, with
+    // independent loads in flight, and combined through shared memory.
+    extern __shared__ float wsplit[];                 // [S] weights, then [kMergeLanes][D] partial sums
     __shared__ float red[32];
     const int grp = blockIdx.x / g.G, h = blockIdx.x % g.G;
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int D = g.d;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const int64_t base = (int64_t)grp * S;
     float mx = -INFINITY;
-    for (int s = threadIdx.x; s < S; s += blockDim.x) mx = fmaxf(mx, part_ml[((base + s) * g.G + h) * 2]);
+    for (int s = tid; s < S; s += blockDim.x) mx = fmaxf(mx, part_ml[((base + s) * g.G + h) * 2]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if (lane == 0) red[warp] = mx;
@@ -575,7 +589,7 @@ __global__ void attn_merge_kernel(Geo g, int S, const float *part_ml, const floa
     for (int w = 0; w < nw; ++w) M = fmaxf(M, red[w]);
     __syncthreads();
     float ls = 0.f;
-    for (int s = threadIdx.x; s < S; s += blockDim.x) {
+    for (int s = tid; s < S; s += blockDim.x) {
         const int64_t idx = (base + s) * g.G + h;
         const float ms = part_ml[idx * 2];
         const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
@@ -588,16 +602,23 @@ __global__ void attn_merge_kernel(Geo g, int S, const float *part_ml, const floa
     __syncthreads();
     float L = 0.f;
     for (int w = 0; w < nw; ++w) L += red[w];
-    for (int dim = threadIdx.x; dim < D; dim += blockDim.x) {
-        float acc = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll 8
-            for (int s = 0; s < S; ++s) {
-                const float f = wsplit[s];
-                if (f != 0.f) acc = fmaf(part_o[((base + s) * g.G + h) * D + dim], f, acc);
-            }
+    const int q = tid / D, dim = tid % D;
+    float acc = 0.f;
+    if (M != -INFINITY && q < kMergeLanes) {
+#pragma unroll 4
+        for (int s = q; s < S; s += kMergeLanes) {
+            const float f = wsplit[s];
+            if (f != 0.f) acc = fmaf(part_o[((base + s) * g.G + h) * D + dim], f, acc);
         }
-        out[g.qrow(b, kvh, h) * D + dim] = from_f32<T>(L > 0.f ? acc / L : 0.f);
+    }
+    float *psum = wsplit + S;
+    if (q < kMergeLanes) psum[q * D + dim] = acc;
+    __syncthreads();
+    if (q == 0) {
+        float tot = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMergeLanes; ++k) tot += psum[k * D + dim];
+        out[g.qrow(b, kvh, h) * D + dim] = from_f32<T>(L > 0.f ? tot / L : 0.f);
     }
 }
 
@@ -612,7 +633,7 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
     const int dense = sel == nullptr;
     zha_selection sv{};
     if (sel) sv = *sel;
-    dim3 grid(S, g.groups(), (g.G + 15) / 16);
+    dim3 grid((g.G + 15) / 16, S, g.groups());
     const char *attn_name = dense ? "attn_dense" : "attn_sparse";
     if (g.dtype == ZHA_BF16) {
         auto qq = static_cast<const __nv_bfloat16 *>(q);
@@ -641,7 +662,8 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         ProfScope pm("attn_merge", st);
-        attn_merge_kernel<__nv_bfloat16><<<g.groups() * g.G, g.d, S * sizeof(float), st>>>(
+        attn_merge_kernel<__nv_bfloat16><<<g.groups() * g.G, kMergeLanes * g.d,
+                                           (S + kMergeLanes * g.d) * sizeof(float), st>>>(
             g, S, part_ml, part_o, static_cast<__nv_bfloat16 *>(out));
     } else {
         auto qq = static_cast<const float *>(q);
@@ -657,7 +679,8 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         ProfScope pm("attn_merge", st);
-        attn_merge_kernel<float><<<g.groups() * g.G, g.d, S * sizeof(float), st>>>(
+        attn_merge_kernel<float><<<g.groups() * g.G, kMergeLanes * g.d,
+                                   (S + kMergeLanes * g.d) * sizeof(float), st>>>(
             g, S, part_ml, part_o, static_cast<float *>(out));
     }
     return cudaGetLastError();

@@ -166,15 +166,30 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
     if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
     const uint32_t all = all_heads(g.G);
 
-    uint32_t bq[NT][KP][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int h = nt * 8 + gq;
-#pragma unroll
-        for (int kp = 0; kp < KP; ++kp) {
+    // B fragments (query rows): in registers, or -- with 4 n-tiles, where
+    // registers run out -- in shared memory, one 16-byte fragment per lane
+    constexpr bool QS = NT >= 4;
+    __shared__ uint4 qsm[QS ? NT * KP * 32 : 1];
+    uint32_t bq[QS ? 1 : NT][KP][4];
+    if constexpr (QS) {
+        for (int i = threadIdx.x; i < NT * KP * 32; i += blockDim.x) {
+            const int ln = i & 31, kp = (i >> 5) % KP, nt = (i >> 5) / KP;
+            const int h = nt * 8 + (ln >> 2);
             uint4 w = make_uint4(0, 0, 0, 0);
-            if (h < g.G) w = ldg16(q + g.qrow(b, kvh, h) * D + kp * 32 + t * 8);
-            bq[nt][kp][0] = w.x; bq[nt][kp][1] = w.y; bq[nt][kp][2] = w.z; bq[nt][kp][3] = w.w;
+            if (h < g.G) w = ldg16(q + g.qrow(b, kvh, h) * D + kp * 32 + (ln & 3) * 8);
+            qsm[i] = w;
+        }
+        __syncthreads();
+    } else {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int h = nt * 8 + gq;
+#pragma unroll
+            for (int kp = 0; kp < KP; ++kp) {
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if (h < g.G) w = ldg16(q + g.qrow(b, kvh, h) * D + kp * 32 + t * 8);
+                bq[nt][kp][0] = w.x; bq[nt][kp][1] = w.y; bq[nt][kp][2] = w.z; bq[nt][kp][3] = w.w;
+            }
         }
     }
     float runmax[NT][2], runmin[NT][2];
@@ -186,7 +201,7 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
 
     const float s = g.s;
     // U candidates per warp and iteration, their loads issued together
-    constexpr int U = 2;
+    constexpr int U = QS ? 1 : 2;
     const int stride = gridDim.x * kScoreWarps * U;
     for (int i0 = (blockIdx.x * kScoreWarps + warp) * U; i0 < n; i0 += stride) {
         int node[U];
@@ -244,8 +259,14 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
                     const uint32_t a1[4] = {xa.z, xb.z, xa.w, xb.w};
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        mma_bf16_16816(acc[nt], a0, bq[nt][kp][0], bq[nt][kp][1]);
-                        mma_bf16_16816(acc[nt], a1, bq[nt][kp][2], bq[nt][kp][3]);
+                        if constexpr (QS) {
+                            const uint4 f = qsm[(nt * KP + kp) * 32 + lane];
+                            mma_bf16_16816(acc[nt], a0, f.x, f.y);
+                            mma_bf16_16816(acc[nt], a1, f.z, f.w);
+                        } else {
+                            mma_bf16_16816(acc[nt], a0, bq[nt][kp][0], bq[nt][kp][1]);
+                            mma_bf16_16816(acc[nt], a1, bq[nt][kp][2], bq[nt][kp][3]);
+                        }
                     }
                 }
                 const int r0 = mt * 16 + gq, r1 = r0 + 8;
@@ -472,7 +493,8 @@ __device__ __forceinline__ float e4m3_value(uint32_t byte) {
 // Scoring against MX-FP8 summaries (E4M3 bytes, one power-of-two scale per 32
 // coordinates of a plane) with E4M3 tensor-core MMAs, so the summaries are
 // never converted: mma.sync m16n8k32 (A = planes, B = query heads, one MMA
-// per 32-coordinate block and query term). Each query head is held as two
+// per 32-coordinate block and query term; the stored rows are permuted so that
+// one 16-byte load brings a lane's bytes of two blocks). Each query head is held as two
 // E4M3 terms with one power-of-two scale per head: q ~ 2^e (hi + lo), hi the
 // nearest E4M3 of q / 2^e (e the smallest with max|q| <= 448 * 2^e), lo that
 // of the remainder -- about 8 significant bits, the precision of bf16.
@@ -506,9 +528,15 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
         float amax = 0.f;
 #pragma unroll
         for (int kp = 0; kp < KP; ++kp) {
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (h < g.G) w = ldg16(q + g.qrow(b, kvh, h) * D + kp * 32 + t * 8);
-            const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+            // coordinates 32 kp + 4 t + (0..3) and 32 kp + 16 + 4 t + (0..3): the
+            // k-slots of this lane in an m16n8k32 fragment
+            uint2 lo = make_uint2(0, 0), hi = make_uint2(0, 0);
+            if (h < g.G) {
+                const __nv_bfloat16 *qh = q + g.qrow(b, kvh, h) * D + kp * 32 + t * 4;
+                lo = __ldg(reinterpret_cast<const uint2 *>(qh));
+                hi = __ldg(reinterpret_cast<const uint2 *>(qh + 16));
+            }
+            const uint32_t in[4] = {lo.x, lo.y, hi.x, hi.y};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&in[j]));
@@ -570,8 +598,9 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
                 }
             }
         }
-        // all loads of the U candidates first: E4M3 rows, block scales, biases
-        uint2 ra[U][MT][KP], rb[U][MT][KP];
+        // all loads of the U candidates first: E4M3 rows (one 16-byte load covers
+        // this lane's bytes of two blocks), block scales, biases
+        uint4 ra[U][MT][KP / 2], rb[U][MT][KP / 2];
         uint32_t sa[U][MT], sb[U][MT];
         float ba[U][MT], bb[U][MT];
 #pragma unroll
@@ -582,11 +611,9 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
                 const int r0 = mt * 16 + gq, r1 = r0 + 8;
                 const bool v0 = hm[u] && r0 < g.R, v1 = hm[u] && r1 < g.R;
 #pragma unroll
-                for (int kp = 0; kp < KP; ++kp) {
-                    ra[u][mt][kp] = v0 ? __ldg(reinterpret_cast<const uint2 *>(mu + (rec + r0) * D + kp * 32 + t * 8))
-                                       : make_uint2(0, 0);
-                    rb[u][mt][kp] = v1 ? __ldg(reinterpret_cast<const uint2 *>(mu + (rec + r1) * D + kp * 32 + t * 8))
-                                       : make_uint2(0, 0);
+                for (int pp = 0; pp < KP / 2; ++pp) {
+                    ra[u][mt][pp] = v0 ? ldg16(mu + (rec + r0) * D + pp * 64 + t * 16) : make_uint4(0, 0, 0, 0);
+                    rb[u][mt][pp] = v1 ? ldg16(mu + (rec + r1) * D + pp * 64 + t * 16) : make_uint4(0, 0, 0, 0);
                 }
                 if constexpr (KP == 4) {
                     sa[u][mt] = v0 ? __ldg(reinterpret_cast<const uint32_t *>(scl + (rec + r0) * KP)) : 0u;
@@ -617,7 +644,9 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
                 for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll
                 for (int kp = 0; kp < KP; ++kp) {
-                    const uint2 &xa = ra[u][mt][kp], &xb = rb[u][mt][kp];
+                    const uint4 &pa = ra[u][mt][kp >> 1], &pb = rb[u][mt][kp >> 1];
+                    const uint2 xa = (kp & 1) ? make_uint2(pa.z, pa.w) : make_uint2(pa.x, pa.y);
+                    const uint2 xb = (kp & 1) ? make_uint2(pb.z, pb.w) : make_uint2(pb.x, pb.y);
                     // 2^(byte - 127) of this block for rows r0 and r1
                     const float s0 = __uint_as_float(__byte_perm(sa[u][mt], 0u, 0x4440u + kp) << 23);
                     const float s1 = __uint_as_float(__byte_perm(sb[u][mt], 0u, 0x4440u + kp) << 23);
@@ -1093,8 +1122,65 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
     return (int)block_sum<unsigned long long>((unsigned long long)kept, sh.red);
 }
 
+// Join of a small level (at most blockDim.x blocks of 8 candidates, bitmaps of
+// at most 32 KB) in one CTA: the rows' bitmaps staged in shared memory, row
+// masks, one block scan, the kept candidates written in order.
+__device__ void small_join(const Geo &g, const LevelWs &lw, const uint8_t *keptbits, int level, int grp,
+                           int64_t n, const zha_selection &sel, SelShared &sh) {
+    const int tid = threadIdx.x;
+    const int64_t capv = g.capv[level];
+    const int64_t bstride = g.bits_stride(level);
+    const int64_t nblk = (n + 7) >> 3;
+    uint8_t *sb = reinterpret_cast<uint8_t *>(&sh.hist_lo[0]);
+    const uint4 *src = reinterpret_cast<const uint4 *>(keptbits + (int64_t)grp * g.G * bstride);
+    for (int64_t i = tid; i < g.G * bstride / 16; i += blockDim.x)
+        reinterpret_cast<uint4 *>(sb)[i] = __ldcg(src + i);
+    __syncthreads();
+    uint32_t km[8];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) km[v] = 0u;
+    const bool mine = tid < nblk;
+    if (mine) {
+        for (int h = 0; h < g.G; ++h) {
+            const uint32_t b = sb[h * bstride + tid];
+#pragma unroll
+            for (int v = 0; v < 8; ++v) km[v] |= ((b >> v) & 1u) << h;
+        }
+        uint4 *kp = reinterpret_cast<uint4 *>(lw.kept + grp * capv + ((int64_t)tid << 3));
+        kp[0] = make_uint4(km[0], km[1], km[2], km[3]);
+        kp[1] = make_uint4(km[4], km[5], km[6], km[7]);
+    }
+    int cnt = 0;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) cnt += km[v] != 0u;
+    unsigned long long total;
+    int64_t o = (int64_t)block_exclusive_scan<unsigned long long>((unsigned long long)cnt, sh.red, &total);
+    int32_t *out_idx = level > 1 ? lw.plist + grp * g.cap[level] : sel.leaf_idx + grp * g.cap[1];
+    uint32_t *out_mask = level > 1 ? lw.pmask + grp * g.cap[level] : sel.head_mask + grp * g.cap[1];
+    if (mine && cnt) {
+        const int32_t *cand = lw.cand + grp * capv + ((int64_t)tid << 3);
+        const int4 c0 = *reinterpret_cast<const int4 *>(cand);
+        const int4 c1 = *reinterpret_cast<const int4 *>(cand + 4);
+        const int32_t cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+            if (km[v]) {
+                out_idx[o] = cv[v];
+                out_mask[o] = km[v];
+                ++o;
+            }
+    }
+    if (tid == 0) {
+        if (level > 1)
+            lw.pcount[grp] = (int32_t)total;
+        else
+            sel.count[grp] = (int32_t)total;
+    }
+}
+
 __global__ void __launch_bounds__(kSelThreads)
-select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t *level_kept) {
+select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t *level_kept, int fuse_join,
+              zha_selection sel) {
     __shared__ SelShared sh;
     const int h = blockIdx.x, grp = blockIdx.y;
     const int64_t capv = g.capv[level];
@@ -1126,6 +1212,16 @@ select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t 
         [&](int64_t blk, uint32_t kb) { mybits[blk] = (uint8_t)kb; },
         [&](int64_t i) { mybits[i >> 3] |= (uint8_t)(1u << (i & 7)); });
     if (level_kept && threadIdx.x == 0) level_kept[((int64_t)grp * g.G + h) * g.L + (level - 1)] = nk;
+    if (!fuse_join) return;
+    // small level: the last of the group's G rows to finish joins them here
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) sh.last = atomicAdd(&lw.done[grp], 1u) == (uint32_t)(g.G - 1);
+    __syncthreads();
+    if (!sh.last) return;
+    __threadfence();
+    small_join(g, lw, keptbits, level, grp, n, sel, sh);
+    if (threadIdx.x == 0) lw.done[grp] = 0u;
 }
 
 // ------------------------------------------------- selection over several CTAs per row
@@ -1443,34 +1539,48 @@ join_kernel(Geo g, LevelWs lw, const uint8_t *keptbits, int level, zha_selection
     for (int v = 0; v < 8; ++v) cnt += km[v] != 0u;
     unsigned long long total;
     const unsigned long long local = block_exclusive_scan<unsigned long long>((unsigned long long)cnt, red, &total);
-    // 3. running total of the chunks before this one
-    if (tid == 0) {
-        unsigned long long excl = 0ull;
-        if (chunk == 0) {
+    // 3. running total of the chunks before this one: warp 0 reads the
+    // published words of 32 predecessors at once, adds the counts up to the
+    // nearest running total, and moves on by 32 if there is none yet
+    if (tid < 32) {
+        if (tid == 0) {
             __threadfence();
-            atomicExch(&mylb[0], kLbInclusive | total);
-        } else {
-            __threadfence();
-            atomicExch(&mylb[chunk], kLbAggregate | total);
-            const long long t0 = clock64();
-            for (int64_t pc = chunk - 1; pc >= 0;) {
-                const unsigned long long w = *reinterpret_cast<volatile unsigned long long *>(&mylb[pc]);
-                if ((w >> 62) == 0ull) {
-                    if (clock64() - t0 > kSpinCycles) {
-                        set_status(status, ZHA_ERR_TIMEOUT);
-                        break;
-                    }
-                    __nanosleep(32);
-                    continue;
-                }
-                excl += w & kLbValue;
-                if ((w >> 62) == 2ull) break;
-                --pc;
-            }
-            __threadfence();
-            atomicExch(&mylb[chunk], kLbInclusive | (excl + total));
+            atomicExch(&mylb[chunk], (chunk == 0 ? kLbInclusive : kLbAggregate) | total);
         }
-        s_excl = excl;
+        unsigned long long excl = 0ull;
+        int64_t end_pc = chunk;                   // predecessors [.., end_pc) still to add
+        const long long t0 = clock64();
+        while (end_pc > 0) {
+            const int64_t pc = end_pc - 1 - tid;  // lane 0: nearest predecessor
+            const unsigned long long w =
+                pc >= 0 ? *reinterpret_cast<volatile unsigned long long *>(&mylb[pc]) : (2ull << 62);
+            const uint32_t st = (uint32_t)(w >> 62);
+            // the nearest lane holding a running total (lanes past the first chunk count as one)
+            const uint32_t incl = __ballot_sync(0xffffffffu, st == 2u);
+            const int stop = incl ? __ffs(incl) - 1 : 31;
+            const uint32_t missing = __ballot_sync(0xffffffffu, st == 0u) & (stop == 31 ? 0xffffffffu : ((2u << stop) - 1u));
+            if (missing) {
+                if (__any_sync(0xffffffffu, clock64() - t0 > kSpinCycles)) {   // same decision in every lane
+                    if (tid == 0) set_status(status, ZHA_ERR_TIMEOUT);
+                    break;
+                }
+                __nanosleep(32);
+                continue;
+            }
+            unsigned long long v = (tid <= stop && pc >= 0) ? (w & kLbValue) : 0ull;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            excl += v;
+            if (incl) break;
+            end_pc -= 32;
+        }
+        if (tid == 0) {
+            if (chunk > 0) {
+                __threadfence();
+                atomicExch(&mylb[chunk], kLbInclusive | (excl + total));
+            }
+            s_excl = excl;
+        }
     }
     __syncthreads();
     // 4. the kept candidates, in order
@@ -1589,6 +1699,7 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
         LevelWs lw = level_ws(g, ws, level);
         LevelWs up = level < g.L ? level_ws(g, ws, level + 1) : lw;
         const int64_t capv = g.capv[level];
+        int fuse_join = 0;
         {
             ProfScope ps(score_names[level], st);
             if (g.mx()) {
@@ -1681,6 +1792,10 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
             // rows with many candidates: several CTAs per row, as many as can be resident together
             const int64_t rows = (int64_t)g.G * groups;
             const int S = (int)min64(capv / kSplitMinSlice, split_slots() / rows);
+            // small levels: the join runs in the last select CTA of each group, and
+            // the CTAs are smaller (fewer warps at each of the selection's barriers)
+            const int sel_threads = capv <= 8 * 256 ? 256 : kSelThreads;
+            fuse_join = S < 2 && (capv >> 3) <= sel_threads && g.G * g.bits_stride(level) <= 32768;
             if (S >= 2) {
                 char *base = static_cast<char *>(ws);
                 const SplitWs sw{reinterpret_cast<unsigned long long *>(base + g.ws_ghist),
@@ -1690,13 +1805,14 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                 select_split_kernel<<<dim3(S, g.G, groups), kSplitThreads, 0, st>>>(
                     g, lw, keptbits, level, p_levels[level - 1], sel.level_kept, sw, status);
             } else {
-                select_kernel<<<dim3(g.G, groups), kSelThreads, 0, st>>>(g, lw, keptbits, level,
-                                                                         p_levels[level - 1], sel.level_kept);
+                select_kernel<<<dim3(g.G, groups), sel_threads, 0, st>>>(g, lw, keptbits, level,
+                                                                         p_levels[level - 1], sel.level_kept,
+                                                                         fuse_join, sel);
             }
         }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        {
+        if (!fuse_join) {
             ProfScope ps(join_names[level], st);
             const uint8_t *keptbits = reinterpret_cast<const uint8_t *>(static_cast<char *>(ws) + g.ws_keptbits[level]);
             const int64_t chunks = (capv + kJoinChunk - 1) / kJoinChunk;

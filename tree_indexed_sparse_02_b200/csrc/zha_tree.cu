@@ -37,6 +37,18 @@ struct RawPoints {        // keys of a leaf chunk, or children kept in the KV dt
 // 2^(byte - 127) for a biased scale exponent byte in 1..254
 __device__ __forceinline__ float mx_scale(uint8_t byte) { return __uint_as_float((uint32_t)byte << 23); }
 
+// Byte offset, within a plane's row of E4M3 bytes, of the EPL coordinates
+// a lane owns (coordinates lane*EPL ..). Rows are stored permuted so that a
+// scoring lane fetches, with one 16-byte load, its 8 bytes of two adjacent
+// 32-coordinate blocks: coordinate k (block b = k / 32, w = k % 32) sits at
+// 64 (b / 2) + 16 ((w % 16) / 4) + 8 (b % 2) + 4 (w / 16) + w % 4.
+template <int EPL>
+__device__ __forceinline__ int mx_lane_offset(int lane) {
+    const int k = lane * EPL;
+    const int b = k >> 5, w = k & 31;
+    return 64 * (b >> 1) + 16 * ((w & 15) >> 2) + 8 * (b & 1) + 4 * (w >> 4) + (w & 3);
+}
+
 template <int EPL>
 struct Mx8Points {        // children kept as MX-FP8 (E4M3 bytes + one scale per 32)
     const uint8_t *x0;
@@ -44,7 +56,7 @@ struct Mx8Points {        // children kept as MX-FP8 (E4M3 bytes + one scale per
     int64_t stride, sstride;
     __device__ __forceinline__ void load(int i, int lane, float (&x)[EPL]) const {
         const float sc = mx_scale(s0[(int64_t)i * sstride + (lane * EPL) / 32]);
-        const uint8_t *p = x0 + (int64_t)i * stride + lane * EPL;
+        const uint8_t *p = x0 + (int64_t)i * stride + mx_lane_offset<EPL>(lane);
 #pragma unroll
         for (int e = 0; e < EPL; e += 2) {
             const __nv_fp8x2_storage_t two = *reinterpret_cast<const __nv_fp8x2_storage_t *>(p + e);
@@ -119,9 +131,9 @@ __device__ __forceinline__ void mx_store(uint8_t *mu_out, uint8_t *sc_out, const
         packed |= (uint32_t)q << (8 * e);
     }
     if constexpr (EPL == 4)
-        *reinterpret_cast<uint32_t *>(mu_out + lane * 4) = packed;
+        *reinterpret_cast<uint32_t *>(mu_out + mx_lane_offset<EPL>(lane)) = packed;
     else
-        *reinterpret_cast<uint16_t *>(mu_out + lane * 2) = (uint16_t)packed;
+        *reinterpret_cast<uint16_t *>(mu_out + mx_lane_offset<EPL>(lane)) = (uint16_t)packed;
     if (lane % kLanesPerBlock == 0) sc_out[lane / kLanesPerBlock] = (uint8_t)(ex + 127);
 }
 
