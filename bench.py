@@ -383,6 +383,8 @@ def zha_arm(args, w, world, rank, local):
            "touched_frac_of_hbm": touched_mean / (ms_per_step / 1e3) / 1e9 / peak,
            "keys_attended": keys_share,
            "candidates_per_step": float(cand_per_step.mean()),
+           "candidates_per_level": [float(h[:, l, :].sum(dim=1).mean()) for l in range(w.levels)],
+           "attended_tokens_per_step": float(attn_tokens.mean()),
            "gpu_launches": int(launches), "cuda_graph": graph is not None, "scorer": args.scorer,
            "clocks": clocks}
 

@@ -1227,6 +1227,7 @@ select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t 
 // ------------------------------------------------- selection over several CTAs per row
 
 constexpr int kSplitThreads = 256;
+constexpr int kSplitBuckets = kBuckets;               // buckets of a row's histogram summed across its CTAs
 constexpr int kSplitMinSlice = 4096;                  // candidates per CTA, at least
 constexpr long long kSpinCycles = 2000000000LL;       // about a second: a wait that long is an error
 
@@ -1313,7 +1314,7 @@ select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, in
     };
 
     const float m = key_to_float(kmax);
-    const float W = (float)kBuckets / fminf(m - key_to_float(kmin), kMassRange);
+    const float W = (float)kSplitBuckets / fminf(m - key_to_float(kmin), kMassRange);
     if (kmax == 0u || p >= 1.f) {
         // no member, or every member kept: each slice stores its membership
         int kept = 0;
@@ -1338,10 +1339,10 @@ select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, in
     }
     auto bucket = [&](float e) -> int {
         const float x = (m - e) * W;
-        return x < (float)(kBuckets - 1) ? (int)x : kBuckets - 1;
+        return x < (float)(kSplitBuckets - 1) ? (int)x : kSplitBuckets - 1;
     };
     // 1. this slice's mass histogram into the row's global histogram
-    for (int i = tid; i < kBuckets; i += blockDim.x) sh.hist_lo[i] = sh.hist_hi[i] = 0u;
+    for (int i = tid; i < kSplitBuckets; i += blockDim.x) sh.hist_lo[i] = sh.hist_hi[i] = 0u;
     __syncthreads();
     auto add_block = [&](uint32_t mb, const float (&e)[8]) {
 #pragma unroll
@@ -1356,14 +1357,14 @@ select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, in
         add_block(m1, e1);
     }
     __syncthreads();
-    for (int i = tid; i < kBuckets; i += blockDim.x) {
+    for (int i = tid; i < kSplitBuckets; i += blockDim.x) {
         const unsigned long long v = ((unsigned long long)sh.hist_hi[i] << 32) | sh.hist_lo[i];
         if (v) atomicAdd(&gh[i], v);
     }
     if (!row_barrier(&ctr[0], (uint32_t)S, status, &ok_sh)) return;
     // 2. the crossing bucket (every CTA of the row computes the same); the row's
     // histogram comes in with all loads in flight at once
-    constexpr int per = kBuckets / kSplitThreads;
+    constexpr int per = kSplitBuckets / kSplitThreads;
     unsigned long long hv[per];
 #pragma unroll
     for (int j = 0; j < per; ++j) hv[j] = __ldcg(&gh[tid * per + j]);
@@ -1372,7 +1373,7 @@ select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, in
     for (int j = 0; j < per; ++j) mine += hv[j];
     unsigned long long z;
     if (tid == 0) {
-        sh.digit = kBuckets - 1;
+        sh.digit = kSplitBuckets - 1;
         sh.above = 0ull;
     }
     const unsigned long long excl = block_exclusive_scan<unsigned long long>(mine, sh.red, &z);
@@ -1418,7 +1419,7 @@ select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, in
     if (tid == 0 && kept) atomicAdd(&ctr[2], (uint32_t)kept);
     if (!row_barrier(&ctr[0], 2u * (uint32_t)S, status, &ok_sh)) return;
     // 4. every CTA has read the histogram: clear this CTA's share for the next use
-    for (int i = (int)((int64_t)kBuckets * sidx / S) + tid; i < (int)((int64_t)kBuckets * (sidx + 1) / S);
+    for (int i = (int)((int64_t)kSplitBuckets * sidx / S) + tid; i < (int)((int64_t)kSplitBuckets * (sidx + 1) / S);
          i += blockDim.x)
         gh[i] = 0ull;
     if (sidx != 0) return;
