@@ -184,7 +184,11 @@ ZHA_API zha_status zha_tree_level_offsets(const zha_config *cfg, int32_t level, 
  * ZHA_ERR_INVALID_ARG for the native format. */
 ZHA_API zha_status zha_tree_level_scales(const zha_config *cfg, int32_t level, size_t *scale_off);
 
-/* Bytes of scratch every call below may use (routing state + split-K partials). */
+/* Bytes of scratch every call below may use (routing state + split-K
+ * partials). Zero it once before its first use: some of its counters and
+ * histograms are expected at zero on entry, and every call that returns
+ * ZHA_OK with a zero dev_status leaves them at zero again (after a device
+ * error, zero it again). One workspace serves one call at a time. */
 ZHA_API size_t zha_workspace_bytes(const zha_config *cfg);
 ZHA_API zha_status zha_workspace_level_view(const zha_config *cfg, int32_t level, zha_level_view *v);
 /* The same for the last zha_decode_block call with T query positions (its

@@ -108,6 +108,8 @@ Geo make_geo(const zha_config *c, int T = 1) {
     g.ws_lookback = off;
     for (int l = 1; l <= g.L; ++l) off += groups * ((g.capv[l] + zha::kJoinChunk - 1) / zha::kJoinChunk) * 8;
     off = align256(off);
+    g.ws_arrive = off;
+    off = align256(off + (size_t)g.B * 4);
     int splits = c->attn_splits;
     if (splits == 0) {
         // one wave of two resident CTAs per SM over all groups, at most one per 64 tokens
@@ -299,10 +301,10 @@ zha_status zha_decode(const zha_config *cfg, void *tree, void *K, void *V, const
         return ZHA_ERR_INVALID_ARG;
     Geo g = make_geo(cfg);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = zha::launch_decode_write(g, K, V, lens, k_new, v_new, dev_status, st);
-    if (e == cudaSuccess) e = zha::launch_tree_update(g, tree, K, refs, lens, 1, dev_status, st);
+    cudaError_t e = zha::launch_decode_prologue(g, tree, K, V, refs, lens, k_new, v_new, workspace,
+                                                dev_status, st);
     if (e == cudaSuccess)
-        e = zha::launch_route(g, tree, q, lens, p_levels, *sel, workspace, dev_status, st);
+        e = zha::launch_route(g, tree, q, lens, p_levels, *sel, workspace, dev_status, st, false);
     if (e == cudaSuccess)
         e = zha::launch_attention(g, q, K, V, lens, sel, out, workspace, dev_status, st);
     return cuda_status(e);

@@ -51,6 +51,7 @@ struct Geo {
     size_t ws_plist[kMaxLevels + 1], ws_pmask[kMaxLevels + 1], ws_pcount[kMaxLevels + 1];  // kept
     size_t ws_keptbits[kMaxLevels + 1];  // [B*Hkv][G][bits_stride] bytes: each row's kept bitmap
     size_t ws_lookback;                 // [L][B*Hkv][join chunks] u64 running counts of the compaction
+    size_t ws_arrive;                   // [B] u32 groups of a sequence through the decode prologue
     size_t ws_maxkey, ws_minkey;        // [L][B*Hkv][G] u32 ordered keys of the scores
     size_t ws_done;                     // [L][B*Hkv] u32 finished select CTAs
     size_t ws_part_ml, ws_part_o;       // split-K partials
@@ -194,14 +195,20 @@ struct ProfScope {
 namespace zha {
 cudaError_t launch_tree_update(const Geo &g, void *tree, const void *K, const void *refs,
                                const int32_t *lens, int n_new, int32_t *status, cudaStream_t st);
+// init = false: the route's state was already reset (by launch_decode_prologue)
 cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const int32_t *lens,
                          const float *p_levels, const zha_selection &sel, void *ws,
-                         int32_t *status, cudaStream_t st);
+                         int32_t *status, cudaStream_t st, bool init = true);
 cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const void *V,
                              const int32_t *lens, const zha_selection *sel, void *out, void *ws,
                              int32_t *status, cudaStream_t st);
 cudaError_t launch_decode_write(const Geo &g, void *K, void *V, int32_t *lens, const void *k_new,
                                 const void *v_new, int32_t *status, cudaStream_t st);
+// One decode step's prologue in one launch: write the new token, extend the
+// tree along its rightmost path, reset the route's state, advance lens.
+cudaError_t launch_decode_prologue(const Geo &g, void *tree, void *K, void *V, const void *refs,
+                                   int32_t *lens, const void *k_new, const void *v_new, void *ws,
+                                   int32_t *status, cudaStream_t st);
 Geo make_geo_for(const zha_config *c);
 bool score_tc_supported(const Geo &g);
 cudaError_t launch_score_tc(const Geo &g, const void *mu_level, const float *bias, const void *q,

@@ -24,6 +24,7 @@
 //             kept into the next level's parent list (or, at level 1, into
 //             the selection).
 #include "zha_common.cuh"
+#include "zha_route_state.cuh"
 
 namespace zha {
 
@@ -92,29 +93,13 @@ __device__ __forceinline__ int64_t group_len(const Geo &g, const int32_t *lens, 
 
 // ----------------------------------------------------------------------- init
 
-__global__ void route_init_kernel(Geo g, uint32_t *maxkey, uint32_t *minkey, uint32_t *done,
-                                  uint32_t *gctr, unsigned long long *lookback, const int32_t *lens,
-                                  int32_t *status) {
+__global__ void route_init_kernel(Geo g, RouteState rs, const int32_t *lens, int32_t *status) {
     const int grp = blockIdx.x;
     if (threadIdx.x == 0) {
         const int64_t N = (int64_t)lens[grp / g.Hkv] - g.lag;
         if (N < 0 || N > g.max_len) set_status(status, ZHA_ERR_CAPACITY);
     }
-    for (int i = threadIdx.x; i < g.L * g.G; i += blockDim.x) {
-        const int64_t at = ((int64_t)(i / g.G) * g.groups() + grp) * g.G + i % g.G;
-        maxkey[at] = 0u;
-        minkey[at] = 0xffffffffu;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) gctr[at * 4 + k] = 0u;
-    }
-    for (int l = threadIdx.x; l < g.L; l += blockDim.x) done[(int64_t)l * g.groups() + grp] = 0u;
-    // the joins' look-back words of this group, every level
-    int64_t off = 0;
-    for (int l = 1; l <= g.L; ++l) {
-        const int64_t chunks = (g.capv[l] + kJoinChunk - 1) / kJoinChunk;
-        for (int64_t i = threadIdx.x; i < chunks; i += blockDim.x) lookback[off + grp * chunks + i] = 0ull;
-        off += (int64_t)g.groups() * chunks;
-    }
+    route_reset_group(g, rs, grp);
 }
 
 // ---------------------------------------------------------------------- score
@@ -1671,7 +1656,7 @@ int64_t split_slots() {
 
 cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const int32_t *lens,
                          const float *p_levels, const zha_selection &sel, void *ws,
-                         int32_t *status, cudaStream_t st) {
+                         int32_t *status, cudaStream_t st, bool init) {
     static const char *score_names[] = {"", "score[l1]", "score[l2]", "score[l3]", "score[l4]",
                                         "score[l5]", "score[l6]", "score[l7]", "score[l8]"};
     static const char *select_names[] = {"", "select[l1]", "select[l2]", "select[l3]", "select[l4]",
@@ -1683,18 +1668,13 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
     for (int l = 1; l <= g.L; ++l)
         lb_off[l + 1] = lb_off[l] + (int64_t)g.groups() * ((g.capv[l] + kJoinChunk - 1) / kJoinChunk);
     const int groups = g.groups();
-    {
+    cudaError_t e = cudaSuccess;
+    if (init) {
         ProfScope ps("route_init", st);
-        char *base = static_cast<char *>(ws);
-        route_init_kernel<<<groups, 64, 0, st>>>(
-            g, reinterpret_cast<uint32_t *>(base + g.ws_maxkey),
-            reinterpret_cast<uint32_t *>(base + g.ws_minkey),
-            reinterpret_cast<uint32_t *>(base + g.ws_done),
-            reinterpret_cast<uint32_t *>(base + g.ws_gctr),
-            reinterpret_cast<unsigned long long *>(base + g.ws_lookback), lens, status);
+        route_init_kernel<<<groups, 64, 0, st>>>(g, route_state(g, ws), lens, status);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
     }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
     const char *tb = static_cast<const char *>(tree);
     for (int level = g.L; level >= 1; --level) {
         LevelWs lw = level_ws(g, ws, level);

@@ -17,6 +17,7 @@
 // the dot products end in a warp butterfly (every lane gets bitwise the same
 // sum, so all lanes agree on every branch).
 #include "zha_common.cuh"
+#include "zha_route_state.cuh"
 
 namespace zha {
 
@@ -220,16 +221,14 @@ tree_level_kernel(Geo g, TreePtrs tp, const T *K, const T *refs, const int32_t *
 // block barrier, which also makes the children's global writes visible.
 constexpr int kPathWarps = 16;
 
+// The nodes of group grp that change when its cache grows from n_old to
+// n_now tokens, level by level (a block barrier between levels also makes
+// the children's writes visible).
 template <typename T, int EPL, bool MX>
-__global__ void __launch_bounds__(kPathWarps * 32) tree_path_kernel(Geo g, TreePtrs tp, const T *K, const T *refs,
-                                 const int32_t *lens, int n_new, int32_t *status) {
-    const int grp = blockIdx.x;
-    const int b = grp / g.Hkv;
+__device__ __forceinline__ void tree_path_levels(const Geo &g, const TreePtrs &tp, const T *K, const T *refs,
+                                                 int grp, int64_t n_old, int64_t n_now) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    int64_t n_old, n_now;
-    const bool any = update_range(g, lens, b, n_new, n_old, n_now, status);
-    if (!any) return;  // uniform across the block
     int64_t lo = n_old / g.c;
     for (int level = 1; level <= g.L; ++level) {
         if (level > 1) lo /= g.c;
@@ -241,6 +240,68 @@ __global__ void __launch_bounds__(kPathWarps * 32) tree_path_kernel(Geo g, TreeP
                                    (int)(it % g.R), lane);
         __syncthreads();
     }
+}
+
+template <typename T, int EPL, bool MX>
+__global__ void __launch_bounds__(kPathWarps * 32) tree_path_kernel(Geo g, TreePtrs tp, const T *K, const T *refs,
+                                 const int32_t *lens, int n_new, int32_t *status) {
+    const int grp = blockIdx.x;
+    const int b = grp / g.Hkv;
+    int64_t n_old, n_now;
+    const bool any = update_range(g, lens, b, n_new, n_old, n_now, status);
+    if (!any) return;  // uniform across the block
+    tree_path_levels<T, EPL, MX>(g, tp, K, refs, grp, n_old, n_now);
+}
+
+// A decode step's prologue, one block per (sequence, KV head) group: write
+// the group's new token at position lens[b], extend the tree along its
+// rightmost path if the token completes a chunk, reset the group's routing
+// state, and -- in the last of the sequence's groups to get here, after every
+// group has read the old length -- advance lens[b].
+template <typename T, int EPL, bool MX>
+__global__ void __launch_bounds__(kPathWarps * 32)
+decode_prologue_kernel(Geo g, TreePtrs tp, T *K, T *V, const T *refs, int32_t *lens, const T *k_new,
+                       const T *v_new, uint32_t *arrive, RouteState rs, int32_t *status) {
+    __shared__ int64_t s_n;
+    const int grp = blockIdx.x;
+    const int b = grp / g.Hkv, kvh = grp % g.Hkv;
+    if (threadIdx.x == 0) s_n = lens[b];
+    __syncthreads();
+    const int64_t n = s_n;
+    const bool ok = n >= 0 && n + 1 <= g.max_len;
+    if (ok) {
+        const int64_t dst = ((int64_t)grp * g.max_len + n) * g.d;
+        const int64_t src = ((int64_t)b * g.Hkv + kvh) * g.d;
+        for (int e = threadIdx.x; e < g.d; e += blockDim.x) {
+            K[dst + e] = k_new[src + e];
+            V[dst + e] = v_new[src + e];
+        }
+    }
+    route_reset_group(g, rs, grp);
+    __syncthreads();
+    if (ok && (n + 1) / g.c > n / g.c) tree_path_levels<T, EPL, MX>(g, tp, K, refs, grp, n, n + 1);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&arrive[b], 1u) == (uint32_t)(g.Hkv - 1)) {
+            arrive[b] = 0u;
+            if (ok)
+                lens[b] = (int32_t)(n + 1);
+            else
+                set_status(status, ZHA_ERR_CAPACITY);
+        }
+    }
+}
+
+template <typename T, int EPL, bool MX>
+cudaError_t decode_prologue_t(const Geo &g, const TreePtrs &tp, T *K, T *V, const T *refs, int32_t *lens,
+                              const T *k_new, const T *v_new, uint32_t *arrive, const RouteState &rs,
+                              int32_t *status, cudaStream_t st) {
+    const int warps = g.R < 4 ? 4 : (g.R > kPathWarps ? kPathWarps : g.R);
+    ProfScope ps("decode_prologue", st);
+    decode_prologue_kernel<T, EPL, MX><<<g.groups(), warps * 32, 0, st>>>(g, tp, K, V, refs, lens, k_new, v_new,
+                                                                           arrive, rs, status);
+    return cudaGetLastError();
 }
 
 template <typename T, int EPL, bool MX>
@@ -276,6 +337,43 @@ cudaError_t tree_update_t(const Geo &g, const TreePtrs &tp, const T *K, const T 
 }
 
 }  // namespace
+
+TreePtrs tree_ptrs(const Geo &g, void *tree) {
+    TreePtrs tp{};
+    for (int l = 1; l <= g.L; ++l) {
+        tp.mu[l] = static_cast<char *>(tree) + g.mu_off[l];
+        tp.bias[l] = reinterpret_cast<float *>(static_cast<char *>(tree) + g.bias_off[l]);
+        tp.sc[l] = g.mx() ? reinterpret_cast<uint8_t *>(static_cast<char *>(tree) + g.sc_off[l]) : nullptr;
+    }
+    return tp;
+}
+
+cudaError_t launch_decode_prologue(const Geo &g, void *tree, void *K, void *V, const void *refs,
+                                   int32_t *lens, const void *k_new, const void *v_new, void *ws,
+                                   int32_t *status, cudaStream_t st) {
+    const TreePtrs tp = tree_ptrs(g, tree);
+    const RouteState rs = route_state(g, ws);
+    uint32_t *arrive = reinterpret_cast<uint32_t *>(static_cast<char *>(ws) + g.ws_arrive);
+    if (g.dtype == ZHA_BF16) {
+        auto k = static_cast<__nv_bfloat16 *>(K);
+        auto v = static_cast<__nv_bfloat16 *>(V);
+        auto r = static_cast<const __nv_bfloat16 *>(refs);
+        auto kn = static_cast<const __nv_bfloat16 *>(k_new);
+        auto vn = static_cast<const __nv_bfloat16 *>(v_new);
+        if (g.mx())
+            return g.d == 128 ? decode_prologue_t<__nv_bfloat16, 4, true>(g, tp, k, v, r, lens, kn, vn, arrive, rs, status, st)
+                              : decode_prologue_t<__nv_bfloat16, 2, true>(g, tp, k, v, r, lens, kn, vn, arrive, rs, status, st);
+        return g.d == 128 ? decode_prologue_t<__nv_bfloat16, 4, false>(g, tp, k, v, r, lens, kn, vn, arrive, rs, status, st)
+                          : decode_prologue_t<__nv_bfloat16, 2, false>(g, tp, k, v, r, lens, kn, vn, arrive, rs, status, st);
+    }
+    auto k = static_cast<float *>(K);
+    auto v = static_cast<float *>(V);
+    auto r = static_cast<const float *>(refs);
+    auto kn = static_cast<const float *>(k_new);
+    auto vn = static_cast<const float *>(v_new);
+    return g.d == 128 ? decode_prologue_t<float, 4, false>(g, tp, k, v, r, lens, kn, vn, arrive, rs, status, st)
+                      : decode_prologue_t<float, 2, false>(g, tp, k, v, r, lens, kn, vn, arrive, rs, status, st);
+}
 
 cudaError_t launch_tree_update(const Geo &g, void *tree, const void *K, const void *refs,
                                const int32_t *lens, int n_new, int32_t *status, cudaStream_t st) {
