@@ -503,12 +503,18 @@ def traffic_for(kernel: str, alg_bytes_per_launch: float):
 
 
 def source_sha():
+    """Hash of the kernel sources with comments and blank space removed (a
+    comment edit does not invalidate counters taken on the same code)."""
     import hashlib
+    import re
     hsh = hashlib.sha256()
     csrc = os.path.join(ROOT, "tree_indexed_sparse_02_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")):
-            hsh.update(open(os.path.join(csrc, name), "rb").read())
+            src = open(os.path.join(csrc, name)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            src = re.sub(r"//[^\n]*", "", src)
+            hsh.update(re.sub(r"\s+", " ", src).encode())
     return hsh.hexdigest()[:16]
 
 

@@ -98,9 +98,9 @@ enum {
  *       max|x| <= 448 * 2^e, elements round to nearest even. A node record
  *       shrinks from R*d*2 + 4R bytes to R*d + R*d/32 + 4R. Parents are built
  *       from the stored (rounded) children. Requires dtype ZHA_BF16. Scoring
- *       against these summaries runs on E4M3 tensor-core MMAs: each query
- *       head is held as 2^e (hi + lo/16) with hi, lo E4M3 and one power-of-two
- *       scale per head (about 8 significant bits, as bf16). */
+ *       against these summaries uses warp-level E4M3 MMAs: each query head is
+ *       held as 2^e (hi + lo) with hi, lo E4M3 and one power-of-two scale per
+ *       head (about 8 significant bits, as bf16). */
 enum { ZHA_SUMMARY_NATIVE = 0, ZHA_SUMMARY_MXFP8 = 1 };
 
 typedef struct zha_config {

@@ -476,10 +476,15 @@ __device__ __forceinline__ float e4m3_value(uint32_t byte) {
 }
 
 // Scoring against MX-FP8 summaries (E4M3 bytes, one power-of-two scale per 32
-// coordinates of a plane) with E4M3 tensor-core MMAs, so the summaries are
-// never converted: mma.sync m16n8k32 (A = planes, B = query heads, one MMA
-// per 32-coordinate block and query term; the stored rows are permuted so that
-// one 16-byte load brings a lane's bytes of two blocks). Each query head is held as two
+// coordinates of a plane) with warp-level E4M3 MMAs: mma.sync m16n8k32
+// (A = planes, B = query heads, one MMA per 32-coordinate block and query
+// term; the stored rows are permuted so that one 16-byte load brings a lane's
+// bytes of two blocks). On sm_100a this warp-level FP8 form is not a native
+// tensor-core instruction: the compiler expands each into conversions and
+// fp16 MMAs (ncu per-opcode counts per candidate: 66 F2FP, 33 FADD, 16 HMMA),
+// which makes this kernel instruction-bound at about half the HBM bandwidth;
+// native FP8 (and hardware block scaling) is tcgen05's kind::mxf8f6f4.
+// Each query head is held as two
 // E4M3 terms with one power-of-two scale per head: q ~ 2^e (hi + lo), hi the
 // nearest E4M3 of q / 2^e (e the smallest with max|q| <= 448 * 2^e), lo that
 // of the remainder -- about 8 significant bits, the precision of bf16.
