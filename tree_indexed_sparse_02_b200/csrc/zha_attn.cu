@@ -234,7 +234,6 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gq = lane >> 2, t = lane & 3;
-    const TokenPlan tp = make_plan(g, lens, grp, &sel, dense != 0, status);
     const __nv_bfloat16 *Kg = K + (int64_t)grp * g.max_len * D;
     const __nv_bfloat16 *Vg = V + (int64_t)grp * g.max_len * D;
 
@@ -252,6 +251,9 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
             qf[st][3] = h1 < g.G ? q1[st * 8 + 4 + t] : 0u;
         }
     }
+    // the queries are the call's input; the cache, lengths and selection come from earlier kernels
+    pdl_wait();
+    const TokenPlan tp = make_plan(g, lens, grp, &sel, dense != 0, status);
 
     const int ntiles = (tp.nv + kTile - 1) / kTile;
     const int t_lo = (int)((int64_t)ntiles * split / S), t_hi = (int)((int64_t)ntiles * (split + 1) / S);
@@ -450,6 +452,7 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
             part_ml[(pbase + h) * 2 + 1] = L;
         }
     }
+    pdl_trigger();
 }
 
 // CUDA-core variant (fp32 inputs, or any dtype for checking): one token per lane.
@@ -469,9 +472,10 @@ attn_simt_kernel(Geo g, const T *q, const T *K, const T *V, const int32_t *lens,
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int G = min(16, g.G - rbase);
-    const TokenPlan tp = make_plan(g, lens, grp, &sel, dense != 0, status);
     for (int i = threadIdx.x; i < G * D; i += blockDim.x)
         qs[i / D][i % D] = to_f32(q[g.qrow(b, kvh, rbase + i / D) * D + i % D]);
+    pdl_wait();
+    const TokenPlan tp = make_plan(g, lens, grp, &sel, dense != 0, status);
     __syncthreads();
     const T *Kg = K + (int64_t)grp * g.max_len * D;
     const T *Vg = V + (int64_t)grp * g.max_len * D;
@@ -560,6 +564,7 @@ attn_simt_kernel(Geo g, const T *q, const T *K, const T *V, const int32_t *lens,
             part_ml[(pbase + h) * 2 + 1] = L;
         }
     }
+    pdl_trigger();
 }
 
 // Log-sum-exp merge of the split-K partials: one block per (group, head).
@@ -579,6 +584,7 @@ __global__ void attn_merge_kernel(Geo g, int S, const float *part_ml, const floa
     const int D = g.d;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const int64_t base = (int64_t)grp * S;
+    pdl_wait();
     float mx = -INFINITY;
     for (int s = tid; s < S; s += blockDim.x) mx = fmaxf(mx, part_ml[((base + s) * g.G + h) * 2]);
 #pragma unroll
@@ -620,6 +626,7 @@ __global__ void attn_merge_kernel(Geo g, int S, const float *part_ml, const floa
         for (int k = 0; k < kMergeLanes; ++k) tot += psum[k * D + dim];
         out[g.qrow(b, kvh, h) * D + dim] = from_f32<T>(L > 0.f ? tot / L : 0.f);
     }
+    pdl_trigger();
 }
 
 }  // namespace
@@ -652,38 +659,38 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
                 attr_set[dev] = true;
             }
             ProfScope ps(attn_name, st);
-            if (g.d == 128)
-                attn_mma_kernel<128><<<grid, kAttnWarps * 32, attn_smem_bytes<128>(), st>>>(
-                    g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
-            else
-                attn_mma_kernel<64><<<grid, kAttnWarps * 32, attn_smem_bytes<64>(), st>>>(
-                    g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
+            const cudaError_t e = g.d == 128
+                ? launch_pdl(attn_mma_kernel<128>, grid, dim3(kAttnWarps * 32), attn_smem_bytes<128>(), st,
+                             g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status)
+                : launch_pdl(attn_mma_kernel<64>, grid, dim3(kAttnWarps * 32), attn_smem_bytes<64>(), st,
+                             g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
+            if (e != cudaSuccess) return e;
         }
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
         ProfScope pm("attn_merge", st);
-        attn_merge_kernel<__nv_bfloat16><<<g.groups() * g.G, kMergeLanes * g.d,
-                                           (S + kMergeLanes * g.d) * sizeof(float), st>>>(
-            g, S, part_ml, part_o, static_cast<__nv_bfloat16 *>(out));
+        const cudaError_t e = launch_pdl(attn_merge_kernel<__nv_bfloat16>, dim3(g.groups() * g.G),
+                                         dim3(kMergeLanes * g.d), (S + kMergeLanes * g.d) * sizeof(float), st,
+                                         g, S, part_ml, part_o, static_cast<__nv_bfloat16 *>(out));
+        if (e != cudaSuccess) return e;
     } else {
         auto qq = static_cast<const float *>(q);
         auto kk = static_cast<const float *>(K);
         auto vv = static_cast<const float *>(V);
         {
         ProfScope ps(attn_name, st);
-        if (g.d == 128)
-            attn_simt_kernel<float, 128><<<grid, kAttnWarps * 32, 0, st>>>(g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
-        else
-            attn_simt_kernel<float, 64><<<grid, kAttnWarps * 32, 0, st>>>(g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
-        }
-        cudaError_t e = cudaGetLastError();
+        const cudaError_t e = g.d == 128
+            ? launch_pdl(attn_simt_kernel<float, 128>, grid, dim3(kAttnWarps * 32), 0, st,
+                         g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status)
+            : launch_pdl(attn_simt_kernel<float, 64>, grid, dim3(kAttnWarps * 32), 0, st,
+                         g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
         if (e != cudaSuccess) return e;
+        }
         ProfScope pm("attn_merge", st);
-        attn_merge_kernel<float><<<g.groups() * g.G, kMergeLanes * g.d,
-                                   (S + kMergeLanes * g.d) * sizeof(float), st>>>(
-            g, S, part_ml, part_o, static_cast<float *>(out));
+        const cudaError_t e = launch_pdl(attn_merge_kernel<float>, dim3(g.groups() * g.G), dim3(kMergeLanes * g.d),
+                                         (S + kMergeLanes * g.d) * sizeof(float), st,
+                                         g, S, part_ml, part_o, static_cast<float *>(out));
+        if (e != cudaSuccess) return e;
     }
-    return cudaGetLastError();
+    return cudaSuccess;
 }
 
 }  // namespace zha

@@ -95,11 +95,13 @@ __device__ __forceinline__ int64_t group_len(const Geo &g, const int32_t *lens, 
 
 __global__ void route_init_kernel(Geo g, RouteState rs, const int32_t *lens, int32_t *status) {
     const int grp = blockIdx.x;
+    pdl_wait();
     if (threadIdx.x == 0) {
         const int64_t N = (int64_t)lens[grp / g.Hkv] - g.lag;
         if (N < 0 || N > g.max_len) set_status(status, ZHA_ERR_CAPACITY);
     }
     route_reset_group(g, rs, grp);
+    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------- score
@@ -146,10 +148,6 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gq = lane >> 2, t = lane & 3;
     const int64_t cap = g.cap[level], capv = g.capv[level];
-    const CandSource src = cand_source(g, up, level, grp, group_len(g, lens, grp));
-    const int n = (int)cand_count(g, up, level, grp, src.n_here);
-    if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
-    const uint32_t all = all_heads(g.G);
 
     // B fragments (query rows): in registers, or -- with 4 n-tiles, where
     // registers run out -- in shared memory, one 16-byte fragment per lane
@@ -177,6 +175,12 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
             }
         }
     }
+    // the queries are the call's input; everything below depends on earlier kernels
+    pdl_wait();
+    const CandSource src = cand_source(g, up, level, grp, group_len(g, lens, grp));
+    const int n = (int)cand_count(g, up, level, grp, src.n_here);
+    if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
+    const uint32_t all = all_heads(g.G);
     float runmax[NT][2], runmin[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -302,6 +306,7 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
                 }
             }
     }
+    pdl_trigger();
 }
 
 // bf16 scoring for R = 2^RL < 16 planes per node: the 16 rows of an MMA tile
@@ -322,10 +327,6 @@ score_pack_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gq = lane >> 2, t = lane & 3;
     const int64_t cap = g.cap[level], capv = g.capv[level];
-    const CandSource src = cand_source(g, up, level, grp, group_len(g, lens, grp));
-    const int n = (int)cand_count(g, up, level, grp, src.n_here);
-    if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
-    const uint32_t all = all_heads(g.G);
 
     uint32_t bq[NT][KP][4];
 #pragma unroll
@@ -338,6 +339,11 @@ score_pack_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_
             bq[nt][kp][0] = w.x; bq[nt][kp][1] = w.y; bq[nt][kp][2] = w.z; bq[nt][kp][3] = w.w;
         }
     }
+    pdl_wait();
+    const CandSource src = cand_source(g, up, level, grp, group_len(g, lens, grp));
+    const int n = (int)cand_count(g, up, level, grp, src.n_here);
+    if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
+    const uint32_t all = all_heads(g.G);
     float runmax[NT][2], runmin[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -456,6 +462,7 @@ score_pack_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_
                 atomicMin(&lw.minkey[(int64_t)grp * g.G + h], ordered_key(mn));
             }
         }
+    pdl_trigger();
 }
 
 __device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -502,10 +509,6 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gq = lane >> 2, t = lane & 3;
     const int64_t cap = g.cap[level], capv = g.capv[level];
-    const CandSource src = cand_source(g, up, level, grp, group_len(g, lens, grp));
-    const int n = (int)cand_count(g, up, level, grp, src.n_here);
-    if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
-    const uint32_t all = all_heads(g.G);
 
     // B fragments: head nt*8 + gq, block kp, bytes [32 kp + 8 t, +8) as two words,
     // for the hi and lo terms; hscale[nt][j]: 2^e of the head in C column 2t + j
@@ -563,6 +566,11 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
         hscale[nt][0] = __shfl_sync(0xffffffffu, myscale, (2 * t) * 4);
         hscale[nt][1] = __shfl_sync(0xffffffffu, myscale, (2 * t + 1) * 4);
     }
+    pdl_wait();
+    const CandSource src = cand_source(g, up, level, grp, group_len(g, lens, grp));
+    const int n = (int)cand_count(g, up, level, grp, src.n_here);
+    if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
+    const uint32_t all = all_heads(g.G);
     float runmax[NT][2], runmin[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -698,6 +706,7 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
                 }
             }
     }
+    pdl_trigger();
 }
 
 // fp32 scoring on CUDA cores: one block per candidate per iteration, one
@@ -710,12 +719,13 @@ __global__ void score_f32_kernel(Geo g, const float *mu, const float *bias, cons
     const int grp = blockIdx.y;
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int64_t cap = g.cap[level], capv = g.capv[level];
+    for (int i = threadIdx.x; i < g.G * D; i += blockDim.x)
+        qs[i / D][i % D] = q[g.qrow(b, kvh, i / D) * D + i % D];
+    pdl_wait();
     const CandSource src = cand_source(g, up, level, grp, group_len(g, lens, grp));
     const int n = (int)cand_count(g, up, level, grp, src.n_here);
     if (blockIdx.x == 0 && threadIdx.x == 0) lw.count[grp] = n;
     const uint32_t all = all_heads(g.G);
-    for (int i = threadIdx.x; i < g.G * D; i += blockDim.x)
-        qs[i / D][i % D] = q[g.qrow(b, kvh, i / D) * D + i % D];
     float runmax = -INFINITY, runmin = INFINITY;
     __syncthreads();
     for (int i = blockIdx.x; i < n; i += gridDim.x) {
@@ -755,6 +765,7 @@ __global__ void score_f32_kernel(Geo g, const float *mu, const float *bias, cons
         atomicMax(&lw.maxkey[(int64_t)grp * g.G + threadIdx.x], ordered_key(runmax));
         atomicMin(&lw.minkey[(int64_t)grp * g.G + threadIdx.x], ordered_key(runmin));
     }
+    pdl_trigger();
 }
 
 // --------------------------------------------------------------------- select
@@ -1172,6 +1183,7 @@ __global__ void __launch_bounds__(kSelThreads)
 select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t *level_kept, int fuse_join,
               zha_selection sel) {
     __shared__ SelShared sh;
+    pdl_wait();
     const int h = blockIdx.x, grp = blockIdx.y;
     const int64_t capv = g.capv[level];
     const int64_t bstride = g.bits_stride(level);  // bytes of one row's bitmap
@@ -1202,7 +1214,10 @@ select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t 
         [&](int64_t blk, uint32_t kb) { mybits[blk] = (uint8_t)kb; },
         [&](int64_t i) { mybits[i >> 3] |= (uint8_t)(1u << (i & 7)); });
     if (level_kept && threadIdx.x == 0) level_kept[((int64_t)grp * g.G + h) * g.L + (level - 1)] = nk;
-    if (!fuse_join) return;
+    if (!fuse_join) {
+        pdl_trigger();
+        return;
+    }
     // small level: the last of the group's G rows to finish joins them here
     __threadfence();
     __syncthreads();
@@ -1212,6 +1227,7 @@ select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t 
     __threadfence();
     small_join(g, lw, keptbits, level, grp, n, sel, sh);
     if (threadIdx.x == 0) lw.done[grp] = 0u;
+    pdl_trigger();
 }
 
 // ------------------------------------------------- selection over several CTAs per row
@@ -1265,6 +1281,7 @@ __global__ void __launch_bounds__(kSplitThreads, 4)
 select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t *level_kept,
                     SplitWs sw, int32_t *status) {
     __shared__ SelShared sh;
+    pdl_wait();
     __shared__ int ok_sh;
     __shared__ int nk_sh;
     const int sidx = blockIdx.x, S = gridDim.x, h = blockIdx.y, grp = blockIdx.z;
@@ -1472,6 +1489,7 @@ __global__ void __launch_bounds__(kJoinThreads)
 join_kernel(Geo g, LevelWs lw, const uint8_t *keptbits, int level, zha_selection sel,
             unsigned long long *lb, int32_t *status) {
     __shared__ __align__(16) uint8_t sbits[32][kJoinChunk / 8];
+    pdl_wait();
     __shared__ unsigned long long red[kJoinThreads / 32];
     __shared__ unsigned long long s_excl;
     const int chunk = blockIdx.x, grp = blockIdx.y;
@@ -1606,6 +1624,7 @@ join_kernel(Geo g, LevelWs lw, const uint8_t *keptbits, int level, zha_selection
         else
             sel.count[grp] = m;
     }
+    pdl_trigger();
 }
 
 __global__ void __launch_bounds__(kSelThreads)
@@ -1659,6 +1678,12 @@ int64_t split_slots() {
 
 }  // namespace
 
+#define ZHA_TRY(call)                         \
+    do {                                      \
+        const cudaError_t le_ = (call);       \
+        if (le_ != cudaSuccess) return le_;   \
+    } while (0)
+
 cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const int32_t *lens,
                          const float *p_levels, const zha_selection &sel, void *ws,
                          int32_t *status, cudaStream_t st, bool init) {
@@ -1676,8 +1701,7 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
     cudaError_t e = cudaSuccess;
     if (init) {
         ProfScope ps("route_init", st);
-        route_init_kernel<<<groups, 64, 0, st>>>(g, route_state(g, ws), lens, status);
-        e = cudaGetLastError();
+        e = launch_pdl(route_init_kernel, dim3(groups), dim3(64), 0, st, g, route_state(g, ws), lens, status);
         if (e != cudaSuccess) return e;
     }
     const char *tb = static_cast<const char *>(tree);
@@ -1698,7 +1722,8 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                 dim3 grid(per_group, groups);
                 const int mt = g.R > 16 ? 2 : 1, nt = g.G > 16 ? 4 : (g.G > 8 ? 2 : 1);
 #define ZHA_SCORE_MX(D, MT, NT, U) \
-    score_mx8_kernel<D, MT, NT, U><<<grid, kScoreWarps * 32, 0, st>>>(g, mu, scl, bias, qq, lens, lw, up, level)
+    ZHA_TRY(launch_pdl(score_mx8_kernel<D, MT, NT, U>, grid, dim3(kScoreWarps * 32), 0, st, g, mu, scl, bias, qq, \
+                       lens, lw, up, level))
 #define ZHA_SCORE_MX_N(D, MT, U1) \
     do { if (nt == 1) ZHA_SCORE_MX(D, MT, 1, U1); else if (nt == 2) ZHA_SCORE_MX(D, MT, 2, 2); \
          else ZHA_SCORE_MX(D, MT, 4, 1); } while (0)
@@ -1724,7 +1749,8 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                 dim3 grid(per_group, groups);
                 const int rl = __builtin_ctz(g.R);
 #define ZHA_SCORE_PACK(D, NT, RL) \
-    score_pack_kernel<D, NT, RL, 2><<<grid, kScoreWarps * 32, 0, st>>>(g, mu, bias, qq, lens, lw, up, level)
+    ZHA_TRY(launch_pdl(score_pack_kernel<D, NT, RL, 2>, grid, dim3(kScoreWarps * 32), 0, st, g, mu, bias, qq, lens, \
+                       lw, up, level))
 #define ZHA_SCORE_PACK_R(D, NT) \
     do { if (rl == 0) ZHA_SCORE_PACK(D, NT, 0); else if (rl == 1) ZHA_SCORE_PACK(D, NT, 1); \
          else if (rl == 2) ZHA_SCORE_PACK(D, NT, 2); else ZHA_SCORE_PACK(D, NT, 3); } while (0)
@@ -1748,7 +1774,8 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                 dim3 grid(per_group, groups);
                 const int mt = g.R > 16 ? 2 : 1, nt = g.G > 16 ? 4 : (g.G > 8 ? 2 : 1);
 #define ZHA_SCORE(D, MT, NT) \
-    score_mma_kernel<D, MT, NT><<<grid, kScoreWarps * 32, 0, st>>>(g, mu, bias, qq, lens, lw, up, level)
+    ZHA_TRY(launch_pdl(score_mma_kernel<D, MT, NT>, grid, dim3(kScoreWarps * 32), 0, st, g, mu, bias, qq, lens, lw, \
+                       up, level))
 #define ZHA_SCORE_N(D, MT) \
     do { if (nt == 1) ZHA_SCORE(D, MT, 1); else if (nt == 2) ZHA_SCORE(D, MT, 2); else ZHA_SCORE(D, MT, 4); } while (0)
                 if (g.d == 128) {
@@ -1765,9 +1792,11 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                 const int per_group = (int)max64(1, min64(capv, (148 * 8 + groups - 1) / groups));
                 dim3 grid(per_group, groups);
                 if (g.d == 128)
-                    score_f32_kernel<128><<<grid, 128, 0, st>>>(g, mu, bias, qq, lens, lw, up, level);
+                    ZHA_TRY(launch_pdl(score_f32_kernel<128>, grid, dim3(128), 0, st, g, mu, bias, qq, lens, lw, up,
+                                       level));
                 else
-                    score_f32_kernel<64><<<grid, 128, 0, st>>>(g, mu, bias, qq, lens, lw, up, level);
+                    ZHA_TRY(launch_pdl(score_f32_kernel<64>, grid, dim3(128), 0, st, g, mu, bias, qq, lens, lw, up,
+                                       level));
             }
         }
         e = cudaGetLastError();
@@ -1788,12 +1817,11 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                                  reinterpret_cast<int32_t *>(base + g.ws_glidx),
                                  reinterpret_cast<uint32_t *>(base + g.ws_glkey),
                                  reinterpret_cast<uint32_t *>(base + g.ws_gctr)};
-                select_split_kernel<<<dim3(S, g.G, groups), kSplitThreads, 0, st>>>(
-                    g, lw, keptbits, level, p_levels[level - 1], sel.level_kept, sw, status);
+                ZHA_TRY(launch_pdl(select_split_kernel, dim3(S, g.G, groups), dim3(kSplitThreads), 0, st, g, lw,
+                                   keptbits, level, p_levels[level - 1], sel.level_kept, sw, status));
             } else {
-                select_kernel<<<dim3(g.G, groups), sel_threads, 0, st>>>(g, lw, keptbits, level,
-                                                                         p_levels[level - 1], sel.level_kept,
-                                                                         fuse_join, sel);
+                ZHA_TRY(launch_pdl(select_kernel, dim3(g.G, groups), dim3(sel_threads), 0, st, g, lw, keptbits, level,
+                                   p_levels[level - 1], sel.level_kept, fuse_join, sel));
             }
         }
         e = cudaGetLastError();
@@ -1804,8 +1832,8 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
             const int64_t chunks = (capv + kJoinChunk - 1) / kJoinChunk;
             unsigned long long *lb = reinterpret_cast<unsigned long long *>(static_cast<char *>(ws) + g.ws_lookback) +
                                      lb_off[level];
-            join_kernel<<<dim3((unsigned)chunks, groups), kJoinThreads, 0, st>>>(g, lw, keptbits, level, sel, lb,
-                                                                                status);
+            ZHA_TRY(launch_pdl(join_kernel, dim3((unsigned)chunks, groups), dim3(kJoinThreads), 0, st, g, lw,
+                               keptbits, level, sel, lb, status));
         }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

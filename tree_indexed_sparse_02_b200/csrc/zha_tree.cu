@@ -265,6 +265,7 @@ decode_prologue_kernel(Geo g, TreePtrs tp, T *K, T *V, const T *refs, int32_t *l
     __shared__ int64_t s_n;
     const int grp = blockIdx.x;
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
+    pdl_wait();
     if (threadIdx.x == 0) s_n = lens[b];
     __syncthreads();
     const int64_t n = s_n;
@@ -291,6 +292,7 @@ decode_prologue_kernel(Geo g, TreePtrs tp, T *K, T *V, const T *refs, int32_t *l
                 set_status(status, ZHA_ERR_CAPACITY);
         }
     }
+    pdl_trigger();
 }
 
 template <typename T, int EPL, bool MX>
@@ -299,9 +301,8 @@ cudaError_t decode_prologue_t(const Geo &g, const TreePtrs &tp, T *K, T *V, cons
                               int32_t *status, cudaStream_t st) {
     const int warps = g.R < 4 ? 4 : (g.R > kPathWarps ? kPathWarps : g.R);
     ProfScope ps("decode_prologue", st);
-    decode_prologue_kernel<T, EPL, MX><<<g.groups(), warps * 32, 0, st>>>(g, tp, K, V, refs, lens, k_new, v_new,
-                                                                           arrive, rs, status);
-    return cudaGetLastError();
+    return launch_pdl(decode_prologue_kernel<T, EPL, MX>, dim3(g.groups()), dim3(warps * 32), 0, st, g, tp, K, V,
+                      refs, lens, k_new, v_new, arrive, rs, status);
 }
 
 template <typename T, int EPL, bool MX>
