@@ -22,7 +22,10 @@
 //             and the last CTA of a group to finish joins the G bitmaps into
 //             per-candidate head masks and compacts the candidates some head
 //             kept into the next level's parent list (or, at level 1, into
-//             the selection).
+//             the selection). Small levels (at most 512 candidate slots per
+//             group) use one CTA per group instead, a warp per query row and
+//             the join in the same CTA; levels with many candidates spread
+//             each row over several CTAs.
 #include "zha_common.cuh"
 #include "zha_route_state.cuh"
 
@@ -898,7 +901,7 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
     }
     const float m = key_to_float(kmax);
     // Common case, two passes: a histogram of the masses over the score's
-    // distance below the max, in kBuckets equal steps of at most kMassRange
+    // distance below the max, in nvb equal steps of at most kMassRange
     // nats (monotone in the score, so the buckets are contiguous in the
     // (score desc) order), finds the bucket where the running mass crosses
     // p; the members of that bucket are then ordered exactly by (score desc,
@@ -906,13 +909,16 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
     // members (near-equal scores), the radix search below decides instead.
     {
         const float span = m - key_to_float(kmin);
-        const float W = (float)kBuckets / fminf(span, kMassRange);
+        // buckets: about one per candidate (a power of two), at least one per thread, at most kBuckets
+        int nvb = (int)blockDim.x;
+        while (nvb < kBuckets && nvb < n) nvb <<= 1;
+        const float W = (float)nvb / fminf(span, kMassRange);
         if (kmax != kmin && W < 1e30f) {
             auto bucket = [&](float e) -> int {
                 const float x = (m - e) * W;
-                return x < (float)(kBuckets - 1) ? (int)x : kBuckets - 1;
+                return x < (float)(nvb - 1) ? (int)x : nvb - 1;
             };
-            for (int i = tid; i < kBuckets; i += blockDim.x) sh.hist_lo[i] = sh.hist_hi[i] = 0u;
+            for (int i = tid; i < nvb; i += blockDim.x) sh.hist_lo[i] = sh.hist_hi[i] = 0u;
             if (tid == 0) {
                 sh.above = 0ull;
                 sh.ntie = 0;
@@ -931,7 +937,7 @@ __device__ int topp_core(SelShared &sh, int64_t n, float p, uint32_t kmax_in, ui
                 add_block(m1, e1);
             }
             __syncthreads();
-            const int per = kBuckets / (int)blockDim.x;
+            const int per = nvb / (int)blockDim.x;
             unsigned long long mine = 0ull;
             for (int j = 0; j < per; ++j)
                 mine += ((unsigned long long)sh.hist_hi[tid * per + j] << 32) | sh.hist_lo[tid * per + j];
@@ -1227,6 +1233,303 @@ select_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, int32_t 
     __threadfence();
     small_join(g, lw, keptbits, level, grp, n, sel, sh);
     if (threadIdx.x == 0) lw.done[grp] = 0u;
+    pdl_trigger();
+}
+
+// ------------------------------------------------------ small levels: one CTA per group
+//
+// Levels with at most kSmallMax candidate slots per group: one CTA per group,
+// one warp per query row (rows w, w + kSmallWarps, ...). The same exact
+// selection as topp_core, every step warp-synchronous: a 256-bucket mass
+// histogram over the score's distance below the max finds the crossing
+// bucket; its members, listed in index order, are ordered by (score desc,
+// index asc) in shared memory, or -- when more than kSmallList of them share
+// it -- a radix search over the ordered key inside that bucket finds the
+// crossing key, whose equal-score members are taken in index order. Kept
+// candidates are OR-ed into a per-candidate head mask, and after one barrier
+// the CTA joins the rows into the compacted candidate list itself.
+
+constexpr int kSmallWarps = 8;
+constexpr int kSmallThreads = kSmallWarps * 32;
+constexpr int kSmallMax = 512;
+constexpr int kSmallBuckets = 256;
+constexpr int kSmallList = 128;
+
+struct SmallShared {
+    uint32_t kmask[kSmallMax];                      // heads that kept candidate i
+    uint32_t hlo[kSmallWarps][kSmallBuckets];       // each warp's mass histogram: low words ...
+    uint32_t hhi[kSmallWarps][kSmallBuckets];       // ... and carry words
+    int32_t lidx[kSmallWarps][kSmallList];          // crossing-bucket members, index order
+    uint32_t lkey[kSmallWarps][kSmallList];         // their ordered keys
+    int32_t lord[kSmallWarps][kSmallList];          // list positions in (score desc, index asc) order
+    unsigned long long red[kSmallWarps];
+};
+
+__device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long long x, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    return x;
+}
+
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// One warp's histogram: lane l owns buckets [8 l, 8 l + 8).
+struct WarpHist {
+    static constexpr int kPer = kSmallBuckets / 32;
+    unsigned long long h[kPer];
+    unsigned long long excl;    // mass of the buckets before this lane's
+    unsigned long long total;   // mass of all buckets
+};
+
+__device__ __forceinline__ void warp_hist_scan(const uint32_t *lo, const uint32_t *hi, int lane, WarpHist &wh) {
+    unsigned long long mine = 0ull;
+#pragma unroll
+    for (int j = 0; j < WarpHist::kPer; ++j) {
+        const int b = lane * WarpHist::kPer + j;
+        wh.h[j] = ((unsigned long long)hi[b] << 32) | lo[b];
+        mine += wh.h[j];
+    }
+    const unsigned long long incl = warp_incl_scan64(mine, lane);
+    wh.excl = incl - mine;
+    wh.total = __shfl_sync(0xffffffffu, incl, 31);
+}
+
+// First bucket at which the running mass, starting from run0 before bucket 0,
+// reaches target (-1 if none); *above gets the running mass before it.
+__device__ __forceinline__ int warp_hist_cross(const WarpHist &wh, int lane, unsigned long long run0,
+                                               unsigned long long target, unsigned long long *above) {
+    unsigned long long run = run0 + wh.excl, ab = 0ull;
+    int found = -1;
+#pragma unroll
+    for (int j = 0; j < WarpHist::kPer; ++j) {
+        if (found < 0 && wh.h[j] && run < target && run + wh.h[j] >= target) {
+            found = lane * WarpHist::kPer + j;
+            ab = run;
+        }
+        run += wh.h[j];
+    }
+    const unsigned ball = __ballot_sync(0xffffffffu, found >= 0);
+    if (!ball) return -1;
+    const int src = __ffs(ball) - 1;
+    *above = __shfl_sync(0xffffffffu, ab, src);
+    return __shfl_sync(0xffffffffu, found, src);
+}
+
+// Exact top-p of one query row by one warp: members are candidates i < n with
+// (cmask[i] & bit); their kept bits are OR-ed into sh.kmask. Returns (in every
+// lane) the number kept.
+__device__ int small_row_topp(SmallShared &sh, int w, const float *sc, const uint32_t *cmask, int n, uint32_t bit,
+                              float p, uint32_t kmax, uint32_t kmin) {
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    if (kmax == 0u) return 0;  // no member
+    int kept = 0;
+    if (p >= 1.f) {
+        for (int i = lane; i < n; i += 32)
+            if (__ldg(cmask + i) & bit) {
+                atomicOr(&sh.kmask[i], bit);
+                ++kept;
+            }
+        return warp_sum_int(kept);
+    }
+    uint32_t *lo = sh.hlo[w], *hi = sh.hhi[w];
+    const float m = key_to_float(kmax);
+    float W = (float)kSmallBuckets / fminf(m - key_to_float(kmin), kMassRange);
+    if (kmax == kmin || !(W < 1e30f)) W = 0.f;  // one score value (or a sub-denormal span): one bucket
+    auto bucket = [&](float e) -> int {
+        const float x = (m - e) * W;
+        return x < (float)(kSmallBuckets - 1) ? (int)x : kSmallBuckets - 1;
+    };
+    for (int j = lane; j < kSmallBuckets; j += 32) lo[j] = hi[j] = 0u;
+    __syncwarp();
+    constexpr int kU = 4;
+    for (int i0 = 0; i0 < n; i0 += 32 * kU) {
+        float e[kU];
+        uint32_t c[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * 32 + lane;
+            c[u] = i < n ? __ldg(cmask + i) : 0u;
+            e[u] = i < n ? __ldg(sc + i) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+            if (c[u] & bit) hist_add(lo, hi, bucket(e[u]), fixed_mass(e[u], m));
+    }
+    __syncwarp();
+    WarpHist wh;
+    warp_hist_scan(lo, hi, lane, wh);
+    const unsigned long long target = (unsigned long long)ceil((double)p * (double)wh.total);
+    unsigned long long above = 0ull;
+    int bstar = warp_hist_cross(wh, lane, 0ull, target, &above);
+    if (bstar < 0) bstar = kSmallBuckets;  // unreachable (target <= total): keep every member
+    __syncwarp();
+
+    // buckets before bstar are kept; bstar's members are listed in index order
+    int ntie = 0;
+    for (int i0 = 0; i0 < n; i0 += 32 * kU) {
+        float e[kU];
+        uint32_t c[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * 32 + lane;
+            c[u] = i < n ? __ldg(cmask + i) : 0u;
+            e[u] = i < n ? __ldg(sc + i) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * 32 + lane;
+            const int bk = (c[u] & bit) ? bucket(e[u]) : kSmallBuckets + 1;
+            if (bk < bstar) {
+                atomicOr(&sh.kmask[i], bit);
+                ++kept;
+            }
+            const unsigned tb = __ballot_sync(0xffffffffu, bk == bstar);
+            if (bk == bstar) {
+                const int slot = ntie + __popc(tb & lt);
+                if (slot < kSmallList) {
+                    sh.lidx[w][slot] = i;
+                    sh.lkey[w][slot] = ordered_key(e[u]);
+                }
+            }
+            ntie += __popc(tb);
+        }
+    }
+    __syncwarp();
+    if (ntie <= kSmallList) {
+        // order the list by (key desc, index asc): it is in index order already
+        for (int j = lane; j < ntie; j += 32) {
+            const uint32_t kj = sh.lkey[w][j];
+            int rank = 0;
+            for (int v = 0; v < ntie; ++v) {
+                const uint32_t kv = sh.lkey[w][v];
+                rank += (kv > kj) || (kv == kj && v < j);
+            }
+            sh.lord[w][rank] = j;
+        }
+        __syncwarp();
+        unsigned long long cum = above;
+        for (int r0 = 0; r0 < ntie && cum < target; r0 += 32) {
+            const int r = r0 + lane;
+            const int j = r < ntie ? sh.lord[w][r] : 0;
+            const unsigned long long ms = r < ntie ? fixed_mass(key_to_float(sh.lkey[w][j]), m) : 0ull;
+            const unsigned long long incl = warp_incl_scan64(ms, lane);
+            if (r < ntie && cum + (incl - ms) < target) {
+                atomicOr(&sh.kmask[sh.lidx[w][j]], bit);
+                ++kept;
+            }
+            cum += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    } else {
+        // many members in the crossing bucket: radix search over u = kmax - key
+        // among them (8-bit digits), then equal-score members in index order
+        const uint32_t uspan = kmax - kmin;
+        int hb = uspan ? 32 - __clz(uspan) : 0;
+        uint32_t prefix = 0u;
+        unsigned long long ab = above;
+        while (hb > 0) {
+            const int bits = hb < 8 ? hb : 8;
+            const int shift = hb - bits;
+            for (int j = lane; j < kSmallBuckets; j += 32) lo[j] = hi[j] = 0u;
+            __syncwarp();
+            for (int i = lane; i < n; i += 32) {
+                if (!(__ldg(cmask + i) & bit)) continue;
+                const float e = __ldg(sc + i);
+                if (bucket(e) != bstar) continue;
+                const uint32_t u = kmax - ordered_key(e);
+                if (hb < 32 && (u >> hb) != (prefix >> hb)) continue;
+                hist_add(lo, hi, (int)((u >> shift) & ((1u << bits) - 1u)), fixed_mass(e, m));
+            }
+            __syncwarp();
+            WarpHist rh;
+            warp_hist_scan(lo, hi, lane, rh);
+            unsigned long long a2 = ab;
+            const int dg = warp_hist_cross(rh, lane, ab, target, &a2);
+            __syncwarp();
+            if (dg < 0) break;  // unreachable: the bucket's mass crosses target
+            prefix |= (uint32_t)dg << shift;
+            ab = a2;
+            hb = shift;
+        }
+        const uint32_t tau = prefix;
+        unsigned long long cum = ab;
+        for (int i0 = 0; i0 < n; i0 += 32) {
+            const int i = i0 + lane;
+            const bool mem = i < n && (__ldg(cmask + i) & bit);
+            const float e = mem ? __ldg(sc + i) : 0.f;
+            const bool inb = mem && bucket(e) == bstar;
+            const uint32_t u = inb ? kmax - ordered_key(e) : 0u;
+            if (inb && u < tau) {
+                atomicOr(&sh.kmask[i], bit);
+                ++kept;
+            }
+            const bool tie = inb && u == tau;
+            const unsigned long long ms = (tie && cum < target) ? (unsigned long long)fixed_mass(e, m) : 0ull;
+            const unsigned long long incl = warp_incl_scan64(ms, lane);
+            if (tie && cum + (incl - ms) < target) {
+                atomicOr(&sh.kmask[i], bit);
+                ++kept;
+            }
+            cum += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    __syncwarp();
+    return warp_sum_int(kept);
+}
+
+__global__ void __launch_bounds__(kSmallThreads)
+select_small_kernel(Geo g, LevelWs lw, int level, float p, int32_t *level_kept, zha_selection sel) {
+    __shared__ SmallShared sh;
+    const int grp = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int64_t capv = g.capv[level];
+    pdl_wait();
+    const int n = (int)min64((int64_t)lw.count[grp], min64(capv, kSmallMax));
+    for (int i = tid; i < n; i += kSmallThreads) sh.kmask[i] = 0u;
+    __syncthreads();
+    const uint32_t *cmask = lw.cmask + grp * capv;
+    for (int h = w; h < g.G; h += kSmallWarps) {
+        const uint32_t kmax = lw.maxkey[(int64_t)grp * g.G + h];
+        const uint32_t kmin = lw.minkey[(int64_t)grp * g.G + h];
+        const int nk = small_row_topp(sh, w, lw.scores + (grp * g.G + h) * capv, cmask, n, 1u << h, p, kmax, kmin);
+        if (level_kept && lane == 0) level_kept[((int64_t)grp * g.G + h) * g.L + (level - 1)] = nk;
+    }
+    __syncthreads();
+    // join: the candidates some row kept, in index order, each thread a run of consecutive slots
+    const int per = (n + kSmallThreads - 1) / kSmallThreads;
+    const int i0 = tid * per;
+    int cnt = 0;
+    for (int k = 0; k < per; ++k) {
+        const int i = i0 + k;
+        cnt += (i < n && sh.kmask[i] != 0u);
+    }
+    unsigned long long total;
+    int64_t o = (int64_t)block_exclusive_scan<unsigned long long>((unsigned long long)cnt, sh.red, &total);
+    int32_t *out_idx = level > 1 ? lw.plist + grp * g.cap[level] : sel.leaf_idx + grp * g.cap[1];
+    uint32_t *out_mask = level > 1 ? lw.pmask + grp * g.cap[level] : sel.head_mask + grp * g.cap[1];
+    for (int k = 0; k < per; ++k) {
+        const int i = i0 + k;
+        if (i >= n) break;
+        const uint32_t km = sh.kmask[i];
+        lw.kept[grp * capv + i] = km;
+        if (km) {
+            out_idx[o] = lw.cand[grp * capv + i];
+            out_mask[o] = km;
+            ++o;
+        }
+    }
+    if (tid == 0) {
+        if (level > 1)
+            lw.pcount[grp] = (int32_t)total;
+        else
+            sel.count[grp] = (int32_t)total;
+    }
     pdl_trigger();
 }
 
@@ -1811,7 +2114,11 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
             // the CTAs are smaller (fewer warps at each of the selection's barriers)
             const int sel_threads = capv <= 8 * 256 ? 256 : kSelThreads;
             fuse_join = S < 2 && (capv >> 3) <= sel_threads && g.G * g.bits_stride(level) <= 32768;
-            if (S >= 2) {
+            if (S < 2 && capv <= kSmallMax) {
+                fuse_join = 1;
+                ZHA_TRY(launch_pdl(select_small_kernel, dim3(groups), dim3(kSmallThreads), 0, st, g, lw, level,
+                                   p_levels[level - 1], sel.level_kept, sel));
+            } else if (S >= 2) {
                 char *base = static_cast<char *>(ws);
                 const SplitWs sw{reinterpret_cast<unsigned long long *>(base + g.ws_ghist),
                                  reinterpret_cast<int32_t *>(base + g.ws_glidx),
