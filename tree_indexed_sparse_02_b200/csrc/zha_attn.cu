@@ -51,29 +51,6 @@ struct TokenPlan {
         return k >= 32 ? 0u : (all & ~((1u << k) - 1u));
     }
 
-    // Split form of at(): fetch() issues the selection loads, finish() uses them.
-    __device__ __forceinline__ void fetch(int v, int &lf, uint32_t &hm) const {
-        if (v < sel_tokens) {
-            lf = __ldg(&leaf[v >> lc]);
-            hm = __ldg(&hmask[v >> lc]);
-        }
-    }
-    __device__ __forceinline__ void finish(int v, int lf, uint32_t hm, int &pos, uint32_t &mask,
-                                           int32_t *status) const {
-        if (v < sel_tokens) {
-            if ((unsigned)lf >= (unsigned)n1) {
-                set_status(status, ZHA_ERR_INVALID_ARG);
-                pos = 0;
-                mask = 0u;
-                return;
-            }
-            pos = (lf << lc) | (v & ((1 << lc) - 1));
-            mask = hm | ((pos == 0 || pos >= cur_start) ? span_mask(pos) : 0u);
-            return;
-        }
-        at(v, pos, mask, status);
-    }
-
     __device__ __forceinline__ void at(int v, int &pos, uint32_t &mask, int32_t *status) const {
         if (v < sel_tokens) {
             const int e = v >> lc;
@@ -185,6 +162,10 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool v
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
                  "r"(valid ? 16 : 0));
 }
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src));
+}
+__device__ __forceinline__ uint32_t sbase_of(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -258,27 +239,56 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     const int ntiles = (tp.nv + kTile - 1) / kTile;
     const int t_lo = (int)((int64_t)ntiles * split / S), t_hi = (int)((int64_t)ntiles * (split + 1) / S);
 
-    // Each warp owns rows 16 w .. 16 w + 15 of every tile: it looks up their
-    // cache positions and head masks (one iteration ahead of their copies, so
-    // that the lookups' latency overlaps a tile of compute), copies them, and
-    // computes on them, so the pipeline needs no block-wide barrier.
-    constexpr int kSlots = kStages + 1;
+    // Each warp owns rows 16 w .. 16 w + 15 of every tile: it copies their
+    // selection entries (kept leaf, head mask) into a shared-memory ring
+    // kAhead tiles ahead of their compute, with cp.async in the same commit
+    // groups as the K/V copies (so waiting on them costs nothing extra),
+    // turns them into cache positions and masks when it issues the tile's K/V
+    // copies, and computes on the tile, so the pipeline needs no block-wide
+    // barrier.
+    constexpr int kAhead = kStages + 1;         // lookups copied this many tiles ahead
+    constexpr int kLook = kAhead;               // lookup ring slots (tile x: slot x % kLook)
+    constexpr int kSlots = kStages + 1;         // position/mask slots (tile x: slot x % kSlots)
     __shared__ int spos[kSlots][kTile];
     __shared__ uint32_t smask[kSlots][kTile];
-    auto resolve = [&](int tile, int slot) {
+    __shared__ int32_t lk_leaf[kLook][kTile];
+    __shared__ uint32_t lk_hm[kLook][kTile];
+    const int lrow = warp * 16 + (lane & 15);
+    // selection entries of the warp's rows of tile `tile` (lanes 0..15, one row each)
+    auto look = [&](int tile) {
+        const int v = tile * kTile + lrow;
+        if (lane < 16 && tile < t_hi && v < tp.sel_tokens) {
+            const int slot = (tile - t_lo) % kLook;
+            cp_async4(sbase_of(&lk_leaf[slot][lrow]), tp.leaf + (v >> tp.lc));
+            cp_async4(sbase_of(&lk_hm[slot][lrow]), tp.hmask + (v >> tp.lc));
+        }
+    };
+    // positions and masks of the warp's rows of `tile` from its (completed) entries
+    auto resolve = [&](int tile) {
         if (lane < 16) {
-            const int row = warp * 16 + lane;
-            const int v = tile * kTile + row;
-            int pos;
-            uint32_t m;
-            tp.at(v, pos, m, status);
-            spos[slot][row] = pos;
-            smask[slot][row] = v < tp.nv ? m : 0u;
+            const int v = tile * kTile + lrow;
+            int pos = 0;
+            uint32_t m = 0u;
+            if (v < tp.sel_tokens) {
+                const int slot = (tile - t_lo) % kLook;
+                const int lf = lk_leaf[slot][lrow];
+                if ((unsigned)lf >= (unsigned)tp.n1) {
+                    set_status(status, ZHA_ERR_INVALID_ARG);
+                } else {
+                    pos = (lf << tp.lc) | (v & ((1 << tp.lc) - 1));
+                    m = lk_hm[slot][lrow] | ((pos == 0 || pos >= tp.cur_start) ? tp.span_mask(pos) : 0u);
+                }
+            } else if (v < tp.nv) {
+                tp.at(v, pos, m, status);
+            }
+            spos[(tile - t_lo) % kSlots][lrow] = pos;
+            smask[(tile - t_lo) % kSlots][lrow] = m;
         }
     };
     // the warp's 16 rows, one 16-byte chunk of K and of V per lane and step
-    auto issue = [&](int tile, int stage, int slot) {
+    auto issue = [&](int tile, int stage) {
         const uint32_t kb = sbase + stage * STAGE_B, vb = kb + TILE_B;
+        const int slot = (tile - t_lo) % kSlots;
 #pragma unroll
         for (int k = 0; k < 16 * CH / 32; ++k) {
             const int c = lane + k * 32;
@@ -299,14 +309,23 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     for (int j = 0; j < NJ; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
     const uint32_t mrow[2] = {h0 < g.G ? (1u << h0) : 0u, h1 < g.G ? (1u << h1) : 0u};
 
-    // tile t_lo + i: copies in stage i % kStages, positions in slot i % kSlots
+    // Commit groups: the prologue's lookups of tiles t_lo .. t_lo + kAhead - 1
+    // (waited for at once), then one group per tile of the first kStages - 1
+    // tiles' K/V, then, in iteration it, the K/V of tile it + kStages - 1 with
+    // the lookups of tile it + kAhead. The wait at the top of iteration it
+    // leaves only the newest group pending, so the K/V of tile it and the
+    // lookups of tile it + kStages - 1 (committed kStages - 1 groups earlier
+    // or in the prologue) are complete.
 #pragma unroll
-    for (int st = 0; st < kStages; ++st)
-        if (t_lo + st < t_hi) resolve(t_lo + st, st);
+    for (int st = 0; st < kAhead; ++st) look(t_lo + st);
+    cp_async_commit();
+    cp_async_wait<0>();
     __syncwarp();
 #pragma unroll
     for (int st = 0; st < kStages - 1; ++st) {
-        if (t_lo + st < t_hi) issue(t_lo + st, st, st);
+        if (t_lo + st < t_hi) resolve(t_lo + st);
+        __syncwarp();
+        if (t_lo + st < t_hi) issue(t_lo + st, st);
         cp_async_commit();
     }
     for (int it = 0; t_lo + it < t_hi; ++it) {
@@ -317,18 +336,12 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
         else __syncwarp();
         {
             const int nt = t_lo + it + kStages - 1;
-            if (nt < t_hi) issue(nt, (it + kStages - 1) % kStages, (it + kStages - 1) % kSlots);
+            if (nt < t_hi) resolve(nt);
+            __syncwarp();
+            if (nt < t_hi) issue(nt, (it + kStages - 1) % kStages);
+            look(t_lo + it + kAhead);
             cp_async_commit();
         }
-        // look up the tile after that: loads now, results stored after this
-        // tile's compute (its slot was last read by tile it - 1)
-        // (16 lanes of every warp, one row each, so no warp lags at the barrier)
-        const int rt = t_lo + it + kStages;
-        const int lrow = (threadIdx.x >> 5) * 16 + (threadIdx.x & 15);
-        const bool look = (threadIdx.x & 31) < 16 && rt < t_hi;
-        int f_leaf = 0;
-        uint32_t f_hm = 0u;
-        if (look) tp.fetch(rt * kTile + lrow, f_leaf, f_hm);
         const int stage = it % kStages;
         const uint32_t kb = sbase + stage * STAGE_B, vb = kb + TILE_B;
         const int row0 = warp * 16;
@@ -392,14 +405,6 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
             ldsm_x4_t(vb + row * ROWB + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
             mma16816(o[2 * jp], pa0, pa1, pa2, pa3, b0, b1);
             mma16816(o[2 * jp + 1], pa0, pa1, pa2, pa3, b2, b3);
-        }
-        if (look) {
-            const int v = rt * kTile + lrow;
-            int pos;
-            uint32_t m;
-            tp.finish(v, f_leaf, f_hm, pos, m, status);
-            spos[(it + kStages) % kSlots][lrow] = pos;
-            smask[(it + kStages) % kSlots][lrow] = v < tp.nv ? m : 0u;
         }
     }
     cp_async_wait<0>();
