@@ -1536,7 +1536,8 @@ select_small_kernel(Geo g, LevelWs lw, int level, float p, int32_t *level_kept, 
 // ------------------------------------------------- selection over several CTAs per row
 
 constexpr int kSplitThreads = 256;
-constexpr int kSplitBuckets = kBuckets;               // buckets of a row's histogram summed across its CTAs
+constexpr int kSplitMinBuckets = 1024;                // buckets of a row's histogram summed across its CTAs:
+constexpr int kSplitPerBucket = 64;                   // about n / 64 (a power of two), from 1024 to kBuckets
 constexpr int kSplitMinSlice = 4096;                  // candidates per CTA, at least
 constexpr long long kSpinCycles = 2000000000LL;       // about a second: a wait that long is an error
 
@@ -1586,7 +1587,6 @@ select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, in
     __shared__ SelShared sh;
     pdl_wait();
     __shared__ int ok_sh;
-    __shared__ int nk_sh;
     const int sidx = blockIdx.x, S = gridDim.x, h = blockIdx.y, grp = blockIdx.z;
     const int tid = threadIdx.x;
     const int64_t step = blockDim.x;
@@ -1624,7 +1624,9 @@ select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, in
     };
 
     const float m = key_to_float(kmax);
-    const float W = (float)kSplitBuckets / fminf(m - key_to_float(kmin), kMassRange);
+    int nb = kSplitMinBuckets;
+    while (nb < kBuckets && (int64_t)nb * kSplitPerBucket < n) nb <<= 1;
+    const float W = (float)nb / fminf(m - key_to_float(kmin), kMassRange);
     if (kmax == 0u || p >= 1.f) {
         // no member, or every member kept: each slice stores its membership
         int kept = 0;
@@ -1649,10 +1651,10 @@ select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, in
     }
     auto bucket = [&](float e) -> int {
         const float x = (m - e) * W;
-        return x < (float)(kSplitBuckets - 1) ? (int)x : kSplitBuckets - 1;
+        return x < (float)(nb - 1) ? (int)x : nb - 1;
     };
     // 1. this slice's mass histogram into the row's global histogram
-    for (int i = tid; i < kSplitBuckets; i += blockDim.x) sh.hist_lo[i] = sh.hist_hi[i] = 0u;
+    for (int i = tid; i < nb; i += blockDim.x) sh.hist_lo[i] = sh.hist_hi[i] = 0u;
     __syncthreads();
     auto add_block = [&](uint32_t mb, const float (&e)[8]) {
 #pragma unroll
@@ -1667,30 +1669,31 @@ select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, in
         add_block(m1, e1);
     }
     __syncthreads();
-    for (int i = tid; i < kSplitBuckets; i += blockDim.x) {
+    for (int i = tid; i < nb; i += blockDim.x) {
         const unsigned long long v = ((unsigned long long)sh.hist_hi[i] << 32) | sh.hist_lo[i];
         if (v) atomicAdd(&gh[i], v);
     }
     if (!row_barrier(&ctr[0], (uint32_t)S, status, &ok_sh)) return;
     // 2. the crossing bucket (every CTA of the row computes the same); the row's
     // histogram comes in with all loads in flight at once
-    constexpr int per = kSplitBuckets / kSplitThreads;
-    unsigned long long hv[per];
+    constexpr int kMaxPer = kBuckets / kSplitThreads;
+    const int per = nb / kSplitThreads;
+    unsigned long long hv[kMaxPer];
 #pragma unroll
-    for (int j = 0; j < per; ++j) hv[j] = __ldcg(&gh[tid * per + j]);
+    for (int j = 0; j < kMaxPer; ++j) hv[j] = j < per ? __ldcg(&gh[tid * per + j]) : 0ull;
     unsigned long long mine = 0ull;
 #pragma unroll
-    for (int j = 0; j < per; ++j) mine += hv[j];
+    for (int j = 0; j < kMaxPer; ++j) mine += hv[j];
     unsigned long long z;
     if (tid == 0) {
-        sh.digit = kSplitBuckets - 1;
+        sh.digit = nb - 1;
         sh.above = 0ull;
     }
     const unsigned long long excl = block_exclusive_scan<unsigned long long>(mine, sh.red, &z);
     const unsigned long long target = (unsigned long long)ceil((double)p * (double)z);
     unsigned long long run = excl;
 #pragma unroll
-    for (int j = 0; j < per; ++j) {
+    for (int j = 0; j < kMaxPer; ++j) {
         const int bk = tid * per + j;
         const unsigned long long hgt = hv[j];
         if (hgt && run < target && run + hgt >= target) {
@@ -1729,7 +1732,7 @@ select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, in
     if (tid == 0 && kept) atomicAdd(&ctr[2], (uint32_t)kept);
     if (!row_barrier(&ctr[0], 2u * (uint32_t)S, status, &ok_sh)) return;
     // 4. every CTA has read the histogram: clear this CTA's share for the next use
-    for (int i = (int)((int64_t)kSplitBuckets * sidx / S) + tid; i < (int)((int64_t)kSplitBuckets * (sidx + 1) / S);
+    for (int i = (int)((int64_t)nb * sidx / S) + tid; i < (int)((int64_t)nb * (sidx + 1) / S);
          i += blockDim.x)
         gh[i] = 0ull;
     if (sidx != 0) return;
@@ -1752,22 +1755,27 @@ select_split_kernel(Geo g, LevelWs lw, uint8_t *keptbits, int level, float p, in
             sh.sorted_ties[rank] = (int)j;
         }
         __syncthreads();
-        if (tid == 0) {
-            int added = 0;
-            unsigned long long cum = above;
-            for (uint32_t r = 0; r < nl && cum < target; ++r) {
-                const int j = sh.sorted_ties[r];
+        // the ordered list, a block of members at a time: a member is kept
+        // while the running mass before it is below target
+        int added = 0;
+        unsigned long long cum = above;
+        for (uint32_t r0 = 0; r0 < nl && cum < target; r0 += blockDim.x) {
+            const uint32_t r = r0 + tid;
+            const int j = r < nl ? sh.sorted_ties[r] : 0;
+            const unsigned long long ms = r < nl ? fixed_mass(key_to_float(sh.tkey[j]), m) : 0ull;
+            unsigned long long tot;
+            const unsigned long long excl = block_exclusive_scan<unsigned long long>(ms, sh.red, &tot);
+            if (r < nl && cum + excl < target) {
                 const int64_t i = sh.ties[j];
                 // other CTAs wrote neighbouring bytes: set the bit with a word atomic
                 const uintptr_t a = reinterpret_cast<uintptr_t>(mybits + (i >> 3));
                 atomicOr(reinterpret_cast<uint32_t *>(a & ~uintptr_t(3)), 1u << (((a & 3u) << 3) + (i & 7)));
                 ++added;
-                cum += fixed_mass(key_to_float(sh.tkey[j]), m);
             }
-            nk_sh = (int)*reinterpret_cast<volatile uint32_t *>(&ctr[2]) + added;
+            cum += tot;
         }
-        __syncthreads();
-        finalise(nk_sh);
+        added = (int)block_sum<unsigned long long>((unsigned long long)added, sh.red);
+        finalise((int)*reinterpret_cast<volatile uint32_t *>(&ctr[2]) + added);
         return;
     }
     // too many members in the crossing bucket (near-equal scores): the row on this CTA
