@@ -7,25 +7,29 @@
 // "Building the tree": a node's estimate is its largest reference-plane
 // value, E = max_r (s q.mu_r + bias_r).
 //
-// Per level, for all (sequence, KV head) groups at once, two launches:
+// Per level, for all (sequence, KV head) groups at once, two launches (three
+// on the largest levels):
 //   score  -- candidate i of a group is child i % c of the (i / c)-th node
 //             the group kept one level up (all nodes at the top level); each
 //             candidate's summary is read once and scored for all G query
 //             heads of the group on tensor cores (mma.sync bf16: planes x
 //             heads), and the per-head max and min score are kept;
-//   select -- one CTA per (group, query head): exact threshold search for the
-//             shortest (score desc, index asc) prefix holding p of the mass,
-//             a radix select over the score's distance below the max (the
-//             range is known, so 12-bit digits are spread over buckets that
-//             are actually used) with masses summed in 2^-31 fixed point
-//             (exact and order-independent); each head writes a kept bitmap,
-//             and the last CTA of a group to finish joins the G bitmaps into
-//             per-candidate head masks and compacts the candidates some head
-//             kept into the next level's parent list (or, at level 1, into
-//             the selection). Small levels (at most 512 candidate slots per
-//             group) use one CTA per group instead, a warp per query row and
-//             the join in the same CTA; levels with many candidates spread
-//             each row over several CTAs.
+//   select -- exact threshold search for the shortest (score desc, index
+//             asc) prefix holding p of the mass, with masses summed in 2^-31
+//             fixed point (exact and order-independent): a histogram of the
+//             masses over the score's distance below the max finds the bucket
+//             where the running mass crosses p, whose members are then
+//             ordered exactly (a radix search over the ordered score keys
+//             when too many share it). Levels with at most 512 candidate
+//             slots per group: one CTA per group, a warp per query row, and
+//             the join in the same CTA. Larger levels: one CTA per (group,
+//             query head), or several per head on levels with many
+//             candidates; each head writes a kept bitmap;
+//   join   -- the G bitmaps become per-candidate head masks and the
+//             candidates some head kept are compacted into the next level's
+//             parent list (or, at level 1, into the selection): by the last
+//             of a group's select CTAs to finish, or, on the largest levels,
+//             by a launch of its own.
 #include "zha_common.cuh"
 #include "zha_route_state.cuh"
 
@@ -2118,7 +2122,7 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
             // rows with many candidates: several CTAs per row, as many as can be resident together
             const int64_t rows = (int64_t)g.G * groups;
             const int S = (int)min64(capv / kSplitMinSlice, split_slots() / rows);
-            // small levels: the join runs in the last select CTA of each group, and
+            // mid-size levels: the join runs in the last select CTA of each group, and
             // the CTAs are smaller (fewer warps at each of the selection's barriers)
             const int sel_threads = capv <= 8 * 256 ? 256 : kSelThreads;
             fuse_join = S < 2 && (capv >> 3) <= sel_threads && g.G * g.bits_stride(level) <= 32768;
