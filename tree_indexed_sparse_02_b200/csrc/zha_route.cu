@@ -199,20 +199,30 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
     // U candidates per warp and iteration, their loads issued together
     constexpr int U = QS ? 1 : 2;
     const int stride = gridDim.x * kScoreWarps * U;
+    // a warp's candidates are looked up an iteration ahead, while the
+    // previous ones' summaries load: one round trip per iteration, not two
+    int nnode[U];
+    uint32_t nhm[U];
+    auto lookup = [&](int j0) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            nnode[u] = 0;
+            nhm[u] = 0u;
+            if (j0 + u < n) src.at(j0 + u, nnode[u], nhm[u], all);
+        }
+    };
+    lookup((blockIdx.x * kScoreWarps + warp) * U);
     for (int i0 = (blockIdx.x * kScoreWarps + warp) * U; i0 < n; i0 += stride) {
         int node[U];
         uint32_t hm[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int i = i0 + u;
-            node[u] = 0;
-            hm[u] = 0u;
-            if (i < n) {
-                src.at(i, node[u], hm[u], all);
-                if (lane == 0) {
-                    lw.cand[grp * capv + i] = node[u];
-                    lw.cmask[grp * capv + i] = hm[u];
-                }
+            node[u] = nnode[u];
+            hm[u] = nhm[u];
+            if (i < n && lane == 0) {
+                lw.cand[grp * capv + i] = node[u];
+                lw.cmask[grp * capv + i] = hm[u];
             }
         }
         uint4 ra[U][MT][KP], rb[U][MT][KP];
@@ -231,6 +241,7 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
                 }
             }
         }
+        lookup(i0 + stride);
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int i = i0 + u;
@@ -587,20 +598,30 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
 
     const float s = g.s;
     const int stride = gridDim.x * kScoreWarps * U;
+    // a warp's candidates are looked up an iteration ahead, while the
+    // previous ones' summaries load: one round trip per iteration, not two
+    int nnode[U];
+    uint32_t nhm[U];
+    auto lookup = [&](int j0) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            nnode[u] = 0;
+            nhm[u] = 0u;
+            if (j0 + u < n) src.at(j0 + u, nnode[u], nhm[u], all);
+        }
+    };
+    lookup((blockIdx.x * kScoreWarps + warp) * U);
     for (int i0 = (blockIdx.x * kScoreWarps + warp) * U; i0 < n; i0 += stride) {
         int node[U];
         uint32_t hm[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int i = i0 + u;
-            node[u] = 0;
-            hm[u] = 0u;
-            if (i < n) {
-                src.at(i, node[u], hm[u], all);
-                if (lane == 0) {
-                    lw.cand[grp * capv + i] = node[u];
-                    lw.cmask[grp * capv + i] = hm[u];
-                }
+            node[u] = nnode[u];
+            hm[u] = nhm[u];
+            if (i < n && lane == 0) {
+                lw.cand[grp * capv + i] = node[u];
+                lw.cmask[grp * capv + i] = hm[u];
             }
         }
         // all loads of the U candidates first: E4M3 rows (one 16-byte load covers
@@ -631,6 +652,7 @@ score_mx8_kernel(Geo g, const uint8_t *mu, const uint8_t *scl, const float *bias
                 bb[u][mt] = v1 ? __ldg(bias + rec + r1) : -INFINITY;
             }
         }
+        lookup(i0 + stride);
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int i = i0 + u;
