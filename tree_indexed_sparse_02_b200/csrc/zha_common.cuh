@@ -94,9 +94,10 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
+// pdl = false launches plainly (full serialisation with the kernel before).
 template <typename... P, typename... A>
-inline cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                              A &&...args) {
+inline cudaError_t launch_pdl_if(bool pdl, void (*kernel)(P...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t st, A &&...args) {
     cudaLaunchConfig_t c{};
     c.gridDim = grid;
     c.blockDim = block;
@@ -104,10 +105,15 @@ inline cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_
     c.stream = st;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[0].val.programmaticStreamSerializationAllowed = 1;
+    at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     c.attrs = at;
     c.numAttrs = 1;
     return cudaLaunchKernelEx(&c, kernel, std::forward<A>(args)...);
+}
+template <typename... P, typename... A>
+inline cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              A &&...args) {
+    return launch_pdl_if(true, kernel, grid, block, smem, st, std::forward<A>(args)...);
 }
 
 // First error wins.

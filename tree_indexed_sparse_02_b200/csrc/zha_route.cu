@@ -1997,6 +1997,20 @@ select_sets_kernel(const float *scores, const int32_t *counts, int64_t stride, f
         [&](int64_t i) { kp[i] = 1; });
 }
 
+// Scoring CTAs (128 threads, up to ~170 registers) resident on the current
+// device at once: three per SM.
+int64_t score_wave() {
+    static int64_t wave[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (wave[dev] == 0) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        wave[dev] = (int64_t)sms * 3;
+    }
+    return wave[dev];
+}
+
 // CTAs of select_split_kernel that fit on the current device at once (0: none known)
 int64_t split_slots() {
     static int64_t slots[64] = {};
@@ -2049,6 +2063,11 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
         int fuse_join = 0;
         {
             ProfScope ps(score_names[level], st);
+            // a scoring grid of several waves starts plainly: launched early
+            // behind the kernel before it, its first wave lands unevenly on
+            // the SMs that kernel still holds, and the whole grid pays for it
+            // (programmatic launch: 256K B=4 step +29 us; one-wave grids gain)
+            bool one_wave = true;
             if (g.mx()) {
                 const auto *mu = reinterpret_cast<const uint8_t *>(tb + g.mu_off[level]);
                 const auto *scl = reinterpret_cast<const uint8_t *>(tb + g.sc_off[level]);
@@ -2057,9 +2076,10 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                 const int64_t want = (capv + kScoreWarps - 1) / kScoreWarps;
                 const int per_group = (int)max64(1, min64(want, (148 * 8 + groups - 1) / groups));
                 dim3 grid(per_group, groups);
+                one_wave = (int64_t)per_group * groups <= score_wave();
                 const int mt = g.R > 16 ? 2 : 1, nt = g.G > 16 ? 4 : (g.G > 8 ? 2 : 1);
 #define ZHA_SCORE_MX(D, MT, NT, U) \
-    ZHA_TRY(launch_pdl(score_mx8_kernel<D, MT, NT, U>, grid, dim3(kScoreWarps * 32), 0, st, g, mu, scl, bias, qq, \
+    ZHA_TRY(launch_pdl_if(one_wave, score_mx8_kernel<D, MT, NT, U>, grid, dim3(kScoreWarps * 32), 0, st, g, mu, scl, bias, qq, \
                        lens, lw, up, level))
 #define ZHA_SCORE_MX_N(D, MT, U1) \
     do { if (nt == 1) ZHA_SCORE_MX(D, MT, 1, U1); else if (nt == 2) ZHA_SCORE_MX(D, MT, 2, 2); \
@@ -2084,9 +2104,10 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                 const int64_t want = (capv + kScoreWarps * cpt - 1) / (kScoreWarps * cpt);
                 const int per_group = (int)max64(1, min64(want, (148 * 8 + groups - 1) / groups));
                 dim3 grid(per_group, groups);
+                one_wave = (int64_t)per_group * groups <= score_wave();
                 const int rl = __builtin_ctz(g.R);
 #define ZHA_SCORE_PACK(D, NT, RL) \
-    ZHA_TRY(launch_pdl(score_pack_kernel<D, NT, RL, 2>, grid, dim3(kScoreWarps * 32), 0, st, g, mu, bias, qq, lens, \
+    ZHA_TRY(launch_pdl_if(one_wave, score_pack_kernel<D, NT, RL, 2>, grid, dim3(kScoreWarps * 32), 0, st, g, mu, bias, qq, lens, \
                        lw, up, level))
 #define ZHA_SCORE_PACK_R(D, NT) \
     do { if (rl == 0) ZHA_SCORE_PACK(D, NT, 0); else if (rl == 1) ZHA_SCORE_PACK(D, NT, 1); \
@@ -2109,9 +2130,10 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                 const int64_t want = (capv + kScoreWarps - 1) / kScoreWarps;
                 const int per_group = (int)max64(1, min64(want, (148 * 8 + groups - 1) / groups));
                 dim3 grid(per_group, groups);
+                one_wave = (int64_t)per_group * groups <= score_wave();
                 const int mt = g.R > 16 ? 2 : 1, nt = g.G > 16 ? 4 : (g.G > 8 ? 2 : 1);
 #define ZHA_SCORE(D, MT, NT) \
-    ZHA_TRY(launch_pdl(score_mma_kernel<D, MT, NT>, grid, dim3(kScoreWarps * 32), 0, st, g, mu, bias, qq, lens, lw, \
+    ZHA_TRY(launch_pdl_if(one_wave, score_mma_kernel<D, MT, NT>, grid, dim3(kScoreWarps * 32), 0, st, g, mu, bias, qq, lens, lw, \
                        up, level))
 #define ZHA_SCORE_N(D, MT) \
     do { if (nt == 1) ZHA_SCORE(D, MT, 1); else if (nt == 2) ZHA_SCORE(D, MT, 2); else ZHA_SCORE(D, MT, 4); } while (0)
@@ -2128,11 +2150,12 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
                 const auto *qq = static_cast<const float *>(q);
                 const int per_group = (int)max64(1, min64(capv, (148 * 8 + groups - 1) / groups));
                 dim3 grid(per_group, groups);
+                one_wave = (int64_t)per_group * groups <= score_wave();
                 if (g.d == 128)
-                    ZHA_TRY(launch_pdl(score_f32_kernel<128>, grid, dim3(128), 0, st, g, mu, bias, qq, lens, lw, up,
+                    ZHA_TRY(launch_pdl_if(one_wave, score_f32_kernel<128>, grid, dim3(128), 0, st, g, mu, bias, qq, lens, lw, up,
                                        level));
                 else
-                    ZHA_TRY(launch_pdl(score_f32_kernel<64>, grid, dim3(128), 0, st, g, mu, bias, qq, lens, lw, up,
+                    ZHA_TRY(launch_pdl_if(one_wave, score_f32_kernel<64>, grid, dim3(128), 0, st, g, mu, bias, qq, lens, lw, up,
                                        level));
             }
         }
