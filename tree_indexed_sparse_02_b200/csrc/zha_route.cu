@@ -2064,9 +2064,9 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
         {
             ProfScope ps(score_names[level], st);
             // a scoring grid of several waves starts plainly: launched early
-            // behind the kernel before it, its first wave lands unevenly on
-            // the SMs that kernel still holds, and the whole grid pays for it
-            // (programmatic launch: 256K B=4 step +29 us; one-wave grids gain)
+            // behind the kernel before it, such grids made the 256K B=4 step
+            // 29 us slower (most likely their first wave starts unevenly on
+            // the SMs that kernel still holds), while one-wave grids gain
             bool one_wave = true;
             if (g.mx()) {
                 const auto *mu = reinterpret_cast<const uint8_t *>(tb + g.mu_off[level]);
