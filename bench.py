@@ -204,40 +204,85 @@ def replica(w, rank: int):
 # --------------------------------------------------------------- CPU oracle
 
 
-def oracle_sample(w, inp, steps: int, warmup: int = 0):
-    """Time the oracle's decode step (route + exact attention) for ONE
-    (sequence, KV head) group on a prebuilt oracle tree; returns (seconds per
-    whole-batch step, threads, sample description)."""
+def _oracle():
     sys.path.insert(0, os.path.join(ROOT, "oracle"))
-    import numpy as np
-    import torch
-
     import zha_oracle as orc
     orc.build_library()
-    G, N, d = w.group, w.context, w.head_dim
+    return orc
+
+
+def oracle_batch_steps(w, inp, qs, k_new, v_new, first: int, steps: int, warmup: int = 0):
+    """Time the oracle on whole-batch decode steps: for EVERY (sequence, KV
+    head) group of the batch, append the step's token to the group's oracle
+    tree, route its query heads and attend each over its token set -- the
+    same work as one zha_decode call. Groups run concurrently on the host's
+    cores (one task per group for the append and the routing, whose head loop
+    the oracle spreads over its OpenMP threads; one task per query head for
+    the attention); as many groups are held at once as half the free host
+    memory allows (their fp64 caches and trees), the rest in later rounds,
+    each round's time added to the step. Returns (seconds of each timed
+    whole-batch step, threads used, sample description)."""
+    import concurrent.futures as cf
+
+    import numpy as np
+    import psutil
+    import torch
+
+    orc = _oracle()
+    B, Hkv, G, N, d, c = w.batch, w.n_kv_heads, w.group, w.context, w.head_dim, w.chunk
     s = 1.0 / math.sqrt(d)
-    K = inp.K[0, 0, :N].to("cpu", torch.float64).numpy()
-    V = inp.V[0, 0, :N].to("cpu", torch.float64).numpy()
-    refs = inp.refs[0].to("cpu", torch.float64).numpy()
-    t0 = time.perf_counter()
+    n_steps = warmup + steps
+    cap = N + n_steps
     storage = "mxfp8" if w.summary == "mxfp8" else ("bf16" if w.dtype == "bf16" else "f32")
-    tree = orc.build_tree(K, refs, N, w.chunk, w.levels, s, storage=storage)
-    build_s = time.perf_counter() - t0
-    q = inp.q[0, :G].to("cpu", torch.float64).numpy()
-    rng = np.random.default_rng(0)
-    times = []
-    for i in range(warmup + steps):
-        qi = q if i == 0 else rng.normal(size=q.shape)
+    p = oracle_p(orc, w)
+    groups = [(b, g) for b in range(B) for g in range(Hkv)]
+    nodes = sum(orc.level_nodes(cap, c, l) for l in range(1, w.levels + 1))
+    per_group = 8 * d * (2 * cap + w.n_refs * nodes)
+    at_once = max(1, min(len(groups), int(0.5 * psutil.virtual_memory().available // per_group)))
+    cores = len(os.sched_getaffinity(0))
+    pool = cf.ThreadPoolExecutor(max_workers=max(cores, at_once))
+    step_s = [0.0] * steps
+    build_s = 0.0
+
+    def prep(bg):
+        b, g = bg
+        K = np.empty((cap, d))
+        V = np.empty((cap, d))
+        K[:N] = inp.K[b, g, :N].to("cpu", torch.float64).numpy()
+        V[:N] = inp.V[b, g, :N].to("cpu", torch.float64).numpy()
+        K[N:] = k_new[first:first + n_steps, b, g].to("cpu", torch.float64).numpy()
+        V[N:] = v_new[first:first + n_steps, b, g].to("cpu", torch.float64).numpy()
+        refs = inp.refs[g].to("cpu", torch.float64).numpy()
+        q = qs[first:first + n_steps, b, g * G:(g + 1) * G].to("cpu", torch.float64).numpy()
+        tree = orc.build_tree(K, refs, N, c, w.levels, s, storage=storage, cap_tokens=cap)
+        return {"K": K, "V": V, "refs": refs, "q": q, "tree": tree, "route": None}
+
+    def append_route(st, i):
+        orc.tree_update(st["tree"], st["K"], st["refs"], N + i + 1)
+        st["route"] = orc.route(st["tree"], st["q"][i], p)
+
+    def attend(st, i, h):
+        kept = st["route"].kept[0][h] if st["tree"].n(1) > 0 else np.zeros(0, dtype=bool)
+        n = N + i + 1
+        orc.attend(st["q"][i][h], st["K"], st["V"], n, s, orc.token_set(n, c, kept))
+
+    for lo in range(0, len(groups), at_once):
         t0 = time.perf_counter()
-        orc.decode_group(tree, qi, K, V, oracle_p(orc, w))
-        if i >= warmup:
-            times.append(time.perf_counter() - t0)
-    groups = w.batch * w.n_kv_heads
-    per_group = sum(times) / len(times)
-    sample = (f"oracle route+attend of 1 of {groups} (sequence, KV head) groups per step on a prebuilt "
-              f"oracle tree (build {build_s:.1f}s untimed), {len(times)} steps; whole-batch step time = "
-              f"{groups} x group time")
-    return per_group * groups, orc.num_threads(), sample
+        part = list(pool.map(prep, groups[lo:lo + at_once]))
+        build_s += time.perf_counter() - t0
+        for i in range(n_steps):
+            t0 = time.perf_counter()
+            list(pool.map(lambda st: append_route(st, i), part))
+            list(pool.map(lambda a: attend(*a), [(st, i, h) for st in part for h in range(G)]))
+            if i >= warmup:
+                step_s[i - warmup] += time.perf_counter() - t0
+        del part
+    pool.shutdown()
+    sample = (f"whole batch: all {len(groups)} (sequence, KV head) groups of every step (token append to the "
+              f"oracle tree, routing of every query head, exact attention over each head's token set), "
+              f"{steps} timed steps after {warmup} untimed, {at_once} groups held at once; oracle trees built "
+              f"beforehand in {build_s:.1f} s (untimed)")
+    return step_s, max(cores, orc.num_threads()), sample
 
 
 def reference_arm(args, w, world, rank):
@@ -245,9 +290,11 @@ def reference_arm(args, w, world, rank):
     if rank != 0:
         return
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    from tree_indexed_sparse_02_b200.inputs import make_inputs
+    from tree_indexed_sparse_02_b200.inputs import decode_stream, make_inputs
     inp = make_inputs(w, device=dev)
-    step_s, cores, sample = oracle_sample(w, inp, args.steps, args.warmup)
+    k_new, v_new, qs = decode_stream(w, args.warmup + args.steps, device=dev)
+    times, cores, sample = oracle_batch_steps(w, inp, qs, k_new, v_new, 0, args.steps, args.warmup)
+    step_s = sum(times) / len(times)
     value = w.batch / step_s
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
@@ -478,12 +525,112 @@ def zha_arm(args, w, world, rank, local):
                       "h2d_bytes_per_step": (qd.numel() + kd.numel() + vd.numel()) * qd.element_size(),
                       "d2h_bytes_per_step": out.numel() * out.element_size()}
 
+    # routing quality of one more (untimed) step: needle recall of every head
+    # from the GPU's selection; for one sampled group, the oracle's routing of
+    # the same step (boundary flips) and each head's captured softmax mass
+    zha.decode(cfg, buf.tree, K, V, refs, lens, qs[step_i], k_new[step_i], v_new[step_i], p, buf.sel, out,
+               buf.workspace, buf.status)
+    torch.cuda.synchronize()
+    buf.check_status("quality step")
+    with_oracle = rank == 0 and world == 1 and not args.no_cpu_baseline
+    res["routing_quality"] = routing_quality(w, inp, buf, K, refs, lens, qs[step_i], p, with_oracle)
+    if "sampled_group" in res["routing_quality"]:
+        sg = res["routing_quality"]["sampled_group"]
+        res["routing_flips"] = {"group": sg["group"], "heads": w.group, "flips": sg["flips"],
+                                "max_dist_from_p": sg["flip_dist_max"], "dists": sg["flip_dists"]}
+    step_i += 1
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        step_s, cores, sample = oracle_sample(w, inp, steps=2)
-        res["cpu_baseline"] = {"value": w.batch / step_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                               "sample": sample}
+        times, cores, sample = oracle_batch_steps(w, inp, qs, k_new, v_new, W_steps, steps=2)
+        res["cpu_baseline"] = {"value": w.batch * len(times) / sum(times), "unit": "tokens/s", "cores": cores,
+                               "kind": "oracle", "sample": sample}
     if world > 1:
         torch.distributed.barrier()
+    return res
+
+
+def routing_quality(w, inp, buf, K, refs, lens, q_step, p_levels, with_oracle: bool):
+    """What the GPU's routing of the last decode step retrieves.
+
+    needle_recall: share of the planted needles (each head's own; the
+    diffuse heads' ones spread over many top nodes reported apart) whose leaf
+    chunk that head kept. With the oracle (with_oracle): for sequence 0, KV
+    head 0, the oracle routes the same step on a tree built from the same
+    cache; flips are nodes kept by one side only among the candidates both
+    had (followed per head down to its first flip), each with the distance of
+    the oracle's running mass before it from p; captured_mass is, per head,
+    the share of its dense softmax mass (exact attention over every cached
+    token) that its token set holds."""
+    import numpy as np
+    import torch
+
+    G, c, L = w.group, w.chunk, w.levels
+    cnt = buf.sel["count"].cpu().numpy()
+    idx = buf.sel["leaf_idx"].cpu().numpy()
+    hmask = buf.sel["head_mask"].cpu().numpy().astype(np.uint32)
+
+    def kept_leaf(b, h, leaf):
+        kvh, j = h // G, h % G
+        row = idx[b, kvh, :cnt[b, kvh]]
+        k = int(np.searchsorted(row, leaf))
+        return k < row.size and row[k] == leaf and (int(hmask[b, kvh, k]) >> j) & 1 == 1
+
+    hits = {"regular": [0, 0], "diffuse": [0, 0]}
+    for b, placed in enumerate(inp.needle_pos):
+        for k, (h, pos) in enumerate(placed):
+            kind = "regular" if k < w.needles else "diffuse"
+            hits[kind][1] += 1
+            hits[kind][0] += kept_leaf(b, h, pos // c)
+    res = {"needle_recall": hits["regular"][0] / max(hits["regular"][1], 1), "needles": hits["regular"][1]}
+    if hits["diffuse"][1]:
+        res["needle_recall_diffuse"] = hits["diffuse"][0] / hits["diffuse"][1]
+        res["needles_diffuse"] = hits["diffuse"][1]
+    if not with_oracle:
+        return res
+    orc = _oracle()
+    N = int(lens[0])
+    s = 1.0 / math.sqrt(w.head_dim)
+    storage = "mxfp8" if w.summary == "mxfp8" else ("bf16" if w.dtype == "bf16" else "f32")
+    K64 = K[0, 0, :N].to("cpu", torch.float64).numpy()
+    tree = orc.build_tree(K64, refs[0].to("cpu", torch.float64).numpy(), N, c, L, s, storage=storage)
+    qg = q_step[0, :G].to("cpu", torch.float64).numpy()
+    r = orc.route(tree, qg, p_levels)
+    flips = []
+    states = {l: buf.level_state(l) for l in range(1, L + 1)}
+    for h in range(G):
+        bit = np.uint32(1 << h)
+        for level in range(L, 0, -1):
+            st = states[level]
+            n = int(st["count"][0, 0])
+            ci = st["cand_idx"][0, 0, :n].cpu().numpy().astype(np.int64)
+            cm = st["cand_mask"][0, 0, :n].cpu().numpy().astype(np.uint32)
+            km = st["kept_mask"][0, 0, :n].cpu().numpy().astype(np.uint32)
+            n_l = orc.level_nodes(N, c, level)
+            cand_g = np.zeros(n_l, dtype=bool)
+            kept_g = np.zeros(n_l, dtype=bool)
+            mem = (cm & bit) != 0
+            cand_g[ci[mem]] = True
+            kept_g[ci[mem & ((km & bit) != 0)]] = True
+            common = cand_g & r.cand[level - 1][h]
+            diff = np.nonzero(common & (kept_g != r.kept[level - 1][h]))[0]
+            pl = float(p_levels[level - 1])
+            flips += [abs(float(r.cumb[level - 1][h][j]) - pl) for j in diff]
+            if diff.size:
+                break
+    logits = s * (K64 @ qg.T)                         # [N, G]
+    wts = np.exp(logits - logits.max(axis=0))
+    wts /= wts.sum(axis=0)
+    n1 = N // c
+    leaves, masks = idx[0, 0, :cnt[0, 0]], hmask[0, 0, :cnt[0, 0]]
+    captured = []
+    for h in range(G):
+        kl = np.zeros(n1, dtype=bool)
+        kl[leaves[(masks >> np.uint32(h)) & 1 == 1]] = True
+        captured.append(float(wts[orc.token_set(N, c, kl), h].sum()))
+    res["sampled_group"] = {"group": [0, 0], "tokens": N, "flips": len(flips),
+                            "flip_dist_max": max(flips) if flips else None, "flip_dists": flips,
+                            "captured_mass": captured, "captured_mass_min": min(captured),
+                            "captured_mass_mean": sum(captured) / len(captured)}
     return res
 
 

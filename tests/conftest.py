@@ -27,3 +27,22 @@ def orc():
     import zha_oracle
     zha_oracle.build_library()
     return zha_oracle
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Report the routing boundary flips (nodes kept by the GPU or by the
+    oracle only, all within the score-error band of p) that the routing
+    parity tests met, with each flip's distance from p."""
+    mod = sys.modules.get("zha_testlib")
+    if mod is None or not mod.ROUTES_COMPARED["heads"]:
+        return
+    flips = mod.FLIPS
+    tr = terminalreporter
+    tr.section("routing boundary flips vs the oracle")
+    tr.write_line(f"head routings compared: {mod.ROUTES_COMPARED['heads']}; flips: {len(flips)}"
+                  + (f"; largest distance of a flip's running mass from p: {max(f['dist'] for f in flips):.3e}"
+                     if flips else ""))
+    for f in flips:
+        tr.write_line(f"  {f['test']} group {f['group']} level {f['level']} head {f['head']} node {f['node']}: "
+                      f"running mass before it {f['cum_before']:.7f}, p {f['p']}, |diff| {f['dist']:.2e} "
+                      f"(band {f['band']:.2e}), kept by the {f['kept_by']} only")

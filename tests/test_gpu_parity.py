@@ -132,6 +132,37 @@ def test_topp_select_matches_oracle(zha, p, stride):
     assert boundary <= 2
 
 
+def test_topp_select_many_near_equal_masses(zha):
+    """Sets of more than 2^17 candidates at p = 0.99, where the fixed-point
+    mass sum's error bound (n 2^-32 of the largest mass) matters most: close
+    but distinct scores, exactly equal scores, and a few large masses over a
+    sea of near-equal small ones. Differences from the oracle are allowed only
+    within 1e-5 + n 2^-32 / Z of p."""
+    n = 140_000
+    g = torch.Generator().manual_seed(9)
+    scores = torch.empty((4, n))
+    scores[0] = 0.5 + torch.rand(n, generator=g) * 1e-4
+    scores[1] = -2.0
+    scores[2] = torch.rand(n, generator=g) * 1e-3 - 12.0
+    scores[2, torch.randint(0, n, (8,), generator=g)] = 0.0
+    scores[3] = torch.randn(n, generator=g) * 0.01
+    counts = torch.full((4,), n, dtype=torch.int32)
+    kept = torch.zeros((4, n), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    zha.topp_select(scores.cuda(), counts.cuda(), 0.99, kept, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kept = kept.cpu().numpy().astype(bool)
+    for i in range(4):
+        E = scores[i].double().numpy()
+        ko, cb = orc.topp_select(E, 0.99)
+        band = 1e-5 + T.fixed_point_band(E)
+        diff = np.nonzero(ko != kept[i])[0]
+        for j in diff:
+            assert abs(cb[j] - 0.99) <= band, (i, j, cb[j])
+        assert diff.size <= 2, (i, diff.size)
+
+
 # ------------------------------------------------------------------ routing
 
 

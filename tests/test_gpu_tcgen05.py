@@ -1,6 +1,8 @@
-"""The tcgen05 (tensor-memory) scoring kernel against the mma.sync one: same
-tree, same queries, scores within fp32 summation-order rounding, and the same
-routing except at exact-score boundary ties."""
+"""The tcgen05 (tensor-memory) scoring kernel: routing with it against the
+fp64 oracle on the same inputs (level by level, the selection and the
+attention outputs), and, as an extra check, against the mma.sync scorer (same
+tree, same queries, scores within fp32 summation-order rounding, the same
+routing except at exact-score boundary ties)."""
 import numpy as np
 import pytest
 import torch
@@ -51,3 +53,27 @@ def test_tcgen05_scores_match_mma_sync(w):
                 assert np.allclose(sa, sb, rtol=1e-5, atol=1e-5), (level, bb, kvh, np.abs(sa - sb).max())
     # the final selections agree (a boundary tie could flip one leaf; none expected here)
     assert torch.equal(tc.sel["count"], ref.sel["count"])
+
+
+@pytest.mark.parametrize("w", CASES, ids=[w.name for w in CASES])
+def test_tcgen05_route_matches_oracle(w):
+    """ZHA_FLAG_TCGEN05 routing and attention of every group against the oracle."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from tree_indexed_sparse_02_b200 import zha
+    cap = w.context + 64
+    inp = make_inputs(w, capacity=cap)
+    dev = T.to_device(inp)
+    cfg = T.make_cfg(zha, w, cap, flags=zha.ZHA_FLAG_TCGEN05)
+    buf = zha.Buffers(cfg)
+    zha.tree_build(cfg, buf.tree, dev.K, dev.refs, dev.lens, buf.status)
+    zha.route(cfg, buf.tree, dev.q, dev.lens, w.p, buf.sel, buf.workspace, buf.status)
+    out = torch.zeros_like(dev.q)
+    zha.sparse_attn(cfg, dev.q, dev.K, dev.V, dev.lens, buf.sel, out, buf.workspace, buf.status)
+    torch.cuda.synchronize()
+    buf.check_status()
+    flipped = 0
+    for b in range(w.batch):
+        for kvh in range(w.n_kv_heads):
+            flipped += len(T.check_group_vs_oracle(w, inp, buf, b, kvh, [w.p] * w.levels, out=out))
+    assert flipped <= max(2, w.batch * w.n_q_heads // 8), flipped

@@ -3,6 +3,7 @@ the CUDA path gets, and compare the two the way the method allows."""
 from __future__ import annotations
 
 import math
+import os
 
 import numpy as np
 import torch
@@ -102,13 +103,42 @@ def gpu_level_candidates(state, b, kvh, h, n_l):
     return cand, kept, score
 
 
+def fixed_point_band(E) -> float:
+    """Bound on the error of a running-mass fraction that the GPU's selection
+    sums in fixed point: each candidate's mass e^(E - max) is rounded to a
+    multiple of 2^-31 (error <= 2^-32), so a running sum of up to n of them is
+    off by at most n 2^-32, and a fraction of the total Z = sum e^(E - max)
+    (>= 1) by at most n 2^-32 / Z."""
+    E = np.asarray(E, dtype=np.float64)
+    E = E[np.isfinite(E)]
+    if E.size == 0:
+        return 0.0
+    Z = float(np.sum(np.exp(E - E.max())))
+    return E.size * 2.0 ** -32 / Z
+
+
+# Every boundary flip the routing comparisons meet, reported at the end of
+# the pytest run (tests/conftest.py): which test, level, query head and node,
+# the oracle's running mass before the node and its distance from p.
+FLIPS: list = []
+ROUTES_COMPARED = {"heads": 0}
+
+
+def _current_test() -> str:
+    return os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+
+
 def compare_routing(route_o, states, b, kvh, G, N, w: Workload, p_levels):
     """Level-by-level comparison of one group's routing. Flips (nodes kept by
     one side only) are allowed only where the oracle's running mass before the
-    node is within the score-error band of p. Returns (flipped_heads, max score err)."""
+    node is within the band of p that the score error and the fixed-point mass
+    sum allow (4 x score error + 1e-5 + fixed_point_band); each one is
+    recorded in FLIPS.
+    Returns (flipped_heads, max score err)."""
     L = w.levels
     flipped = set()
     worst = 0.0
+    ROUTES_COMPARED["heads"] += G
     for h in range(G):
         diverged = False
         for level in range(L, 0, -1):
@@ -128,9 +158,13 @@ def compare_routing(route_o, states, b, kvh, G, N, w: Workload, p_levels):
             flips = np.nonzero((kept_g != kept_o) & common)[0]
             if flips.size:
                 p = float(p_levels[level - 1])
-                band = 4.0 * err + 1e-5
+                band = 4.0 * err + 1e-5 + fixed_point_band(route_o.score[level - 1][h][cand_o])
                 cb = route_o.cumb[level - 1][h]
                 for n in flips:
+                    FLIPS.append({"test": _current_test(), "group": (int(b), int(kvh)), "level": level,
+                                  "head": h, "node": int(n), "cum_before": float(cb[n]), "p": p,
+                                  "dist": float(abs(cb[n] - p)), "band": band,
+                                  "kept_by": "gpu" if kept_g[n] else "oracle"})
                     assert abs(cb[n] - p) <= band, (
                         f"head {h} level {level} node {n}: cum {cb[n]:.6f} vs p {p} (band {band:.2e})")
                 diverged = True
@@ -172,3 +206,40 @@ def build_case(zha, w: Workload, extra_cap: int = 64, lens=None, device="cuda", 
     cfg = make_cfg(zha, w, cap)
     buf = zha.Buffers(cfg, device=device)
     return cfg, inp, dev, buf
+
+
+def check_group_vs_oracle(w: Workload, inp, buf, b: int, kvh: int, p_levels, out=None, tol=None,
+                          max_flipped: int = 2):
+    """One (sequence, KV head) group of a routed (and optionally attended) call
+    against the oracle on the same inputs: routing level by level
+    (compare_routing), the selection's per-head leaf sets and kept counts for
+    every head without a boundary flip, and -- if `out` is given -- each such
+    head's attention output. Returns the set of flipped heads."""
+    G, s = w.group, scale_of(w)
+    N = int(inp.lens[b])
+    t = oracle_tree(w, inp, b, kvh, N, s)
+    K = np64(inp.K[b, kvh, :N])
+    V = np64(inp.V[b, kvh, :N])
+    q = np64(inp.q[b, kvh * G:(kvh + 1) * G])
+    o, r, _ = orc.decode_group(t, q, K, V, p_levels)
+    states = {l: buf.level_state(l) for l in range(1, w.levels + 1)}
+    flipped, worst = compare_routing(r, states, b, kvh, G, N, w, p_levels)
+    tol = TOL[w.dtype] if tol is None else tol
+    assert worst <= tol, worst
+    assert len(flipped) <= max_flipped, flipped
+    cnt = int(buf.sel["count"][b, kvh])
+    idx = buf.sel["leaf_idx"][b, kvh, :cnt].cpu().numpy()
+    assert np.all(np.diff(idx) > 0)
+    hm = buf.sel["head_mask"][b, kvh, :cnt].cpu().numpy().astype(np.uint32)
+    got = None if out is None else np64(out[b, kvh * G:(kvh + 1) * G])
+    for h in range(G):
+        if h in flipped:
+            continue
+        assert np.array_equal(np.sort(idx[(hm >> np.uint32(h)) & 1 != 0]), np.nonzero(r.kept[0][h])[0]), h
+        if buf.sel.get("level_kept") is not None:
+            lk = buf.sel["level_kept"][b, kvh * G + h].cpu().numpy()
+            for level in range(1, w.levels + 1):
+                assert lk[level - 1] == r.kept[level - 1][h].sum(), (h, level)
+        if got is not None:
+            assert rel_err(got[h], o[h]) <= tol, h
+    return flipped

@@ -9,11 +9,15 @@ fp32 draws are rounded once, round-to-nearest-even, to the storage dtype):
 
 * keys    k_t = z_t + m_{floor(t/c)},  z ~ N(0, I_d),  per-chunk offset
   m ~ N(0, 0.5 I_d) (variance 0.5), c = the tree's chunk size;
-* values  ~ N(0, I_d); decode queries q_h ~ N(0, I_d);
-* reference queries ("random" mode) ~ N(0, I_d / d); in "aligned" mode the
-  first min(G, R) references of KV head g are its query heads' vectors q_h and
-  the rest are drawn as in "random" mode (a training-free stand-in for learned
-  references);
+* values  ~ N(0, I_d); queries q_{b,h} ~ N(0, I_d);
+* reference queries ("random" mode) ~ N(0, I_d / d); in "aligned" mode (a
+  training-free stand-in for learned references, which serve every sequence)
+  each query head h has one direction u_h ~ N(0, I_d) shared by the whole
+  batch, sequence b's query is q_{b,h} = u_h + 0.1 e_{b,h} (e ~ N(0, I_d)),
+  and the first min(G, R) references of KV head g are its query heads' u_h
+  (the rest drawn as in "random" mode);
+* decode steps: query of step i = q_{b,h} + 0.1 N(0, I_d), so every step asks
+  for what the needles of its head were planted for;
 * needles: ``needles`` per sequence, assigned round-robin to the query heads;
   needle j of head h sits at a position drawn without replacement from
   [1, N - c) in KV head h // G, with key 3 sqrt(d) q_h/|q_h| + z;
@@ -93,6 +97,23 @@ def _randn(gen, shape, device, std=1.0):
     return x * std if std != 1.0 else x
 
 
+def _draw_queries(w: Workload, gen, device):
+    """Queries [B, Hq, d] and references [Hkv, R, d] (fp32), the generator's
+    first draws."""
+    B, Hq, Hkv, d, G = w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.group
+    q = _randn(gen, (B, Hq, d), device)
+    refs = _randn(gen, (Hkv, w.n_refs, d), device, std=1.0 / math.sqrt(d))
+    if w.refs_mode == "aligned":
+        # one direction per query head for the whole batch (sequence 0's draws),
+        # which is what references trained on many sequences would point at
+        u = q[0].clone()
+        for g in range(Hkv):
+            for r in range(min(G, w.n_refs)):
+                refs[g, r] = u[g * G + r]
+        q = u.unsqueeze(0) + 0.1 * _randn(gen, (B, Hq, d), device)
+    return q, refs
+
+
 def make_inputs(w: Workload, device="cpu", capacity: int | None = None, lens=None) -> Inputs:
     """Draw K, V (for `capacity` >= N slots), q, refs and place the needles.
 
@@ -109,13 +130,7 @@ def make_inputs(w: Workload, device="cpu", capacity: int | None = None, lens=Non
     gen = torch.Generator(device=device)
     gen.manual_seed(w.seed)
 
-    q = _randn(gen, (B, Hq, d), device)
-    refs = _randn(gen, (Hkv, w.n_refs, d), device, std=1.0 / math.sqrt(d))
-    if w.refs_mode == "aligned":
-        # batch 0's query heads stand in for what trained references would learn
-        for g in range(Hkv):
-            for r in range(min(G, w.n_refs)):
-                refs[g, r] = q[0, g * G + r]
+    q, refs = _draw_queries(w, gen, device)
     K = torch.empty((B, Hkv, cap, d), dtype=dt, device=device)
     V = torch.empty((B, Hkv, cap, d), dtype=dt, device=device)
     n_chunks = (cap + c - 1) // c
@@ -163,9 +178,9 @@ def decode_stream(w: Workload, steps: int, device="cpu", seed_offset: int = 1000
     """New tokens and queries for `steps` decode steps.
 
     Returns (k_new [steps, B, Hkv, d], v_new [steps, B, Hkv, d], q [steps, B, Hq, d]);
-    new keys follow the key recipe with fresh per-chunk offsets, queries are
-    N(0, I) in "random" mode and the base queries plus 0.1 N(0, I) noise in
-    "aligned" mode.
+    new keys follow the key recipe with fresh per-chunk offsets; the queries
+    are the workload's queries (those the needles were planted for) plus
+    0.1 N(0, I) noise per step.
     """
     B, Hq, Hkv, d = w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim
     dt = w.torch_dtype()
@@ -174,19 +189,16 @@ def decode_stream(w: Workload, steps: int, device="cpu", seed_offset: int = 1000
     k_new = (_randn(gen, (steps, B, Hkv, d), device)
              + _randn(gen, (1, B, Hkv, d), device, std=math.sqrt(0.5))).to(dt)
     v_new = _randn(gen, (steps, B, Hkv, d), device).to(dt)
-    if w.refs_mode == "aligned":
-        base = make_query_base(w, device)
-        q = (base.unsqueeze(0) + 0.1 * _randn(gen, (steps, B, Hq, d), device)).to(dt)
-    else:
-        q = _randn(gen, (steps, B, Hq, d), device).to(dt)
+    base = make_query_base(w, device)
+    q = (base.unsqueeze(0) + 0.1 * _randn(gen, (steps, B, Hq, d), device)).to(dt)
     return k_new, v_new, q
 
 
 def make_query_base(w: Workload, device="cpu") -> torch.Tensor:
-    """The fp32 base queries make_inputs draws first (same seed, same order)."""
+    """The fp32 queries make_inputs draws first (same seed, same order)."""
     gen = torch.Generator(device=device)
     gen.manual_seed(w.seed)
-    return _randn(gen, (w.batch, w.n_q_heads, w.head_dim), device)
+    return _draw_queries(w, gen, device)[0]
 
 
 def random_selection(n_leaves: int, G: int, frac: float, seed: int, device="cpu"):
