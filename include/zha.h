@@ -175,6 +175,15 @@ ZHA_API size_t zha_tree_bytes(const zha_config *cfg);
 ZHA_API zha_status zha_tree_level_offsets(const zha_config *cfg, int32_t level, size_t *mu_off,
                                   size_t *bias_off);
 
+/* Byte offset of level l's log-masses inside the tree buffer,
+ *   F [batch][n_kv_heads][cap_l][n_refs]  float,
+ * F_r = log sum over the node's keys of e^{s r.k}: the node's log attention
+ * mass at reference r, where its plane is exact (in exact arithmetic
+ * F_r = s r.mu_r + bias_r before mu is rounded for storage). A parent weights
+ * child i of reference r by e^{F_{i,r}} (section "Building the tree": a
+ * parent summarises its children by the same rule as a chunk its keys). */
+ZHA_API zha_status zha_tree_level_logmass(const zha_config *cfg, int32_t level, size_t *lm_off);
+
 /* ZHA_SUMMARY_MXFP8 only: byte offset of level l's block scales,
  *   scale [batch][n_kv_heads][cap_l][n_refs][head_dim / 32]  uint8 = e + 127,
  * mu_r[k] = e4m3(mu byte o(k)) * 2^(scale[k / 32] - 127), where a plane's
@@ -202,9 +211,10 @@ ZHA_API zha_status zha_workspace_level_view_block(const zha_config *cfg, int32_t
  * Leaf j, reference r, keys k_t of chunk j:  l_t = s r.k_t,
  * F = log sum_t e^{l_t}, w_t = e^{l_t - F}, mu_r = sum_t w_t k_t,
  * bias_r = F - s r.mu_r. A parent applies the same rule to its existing
- * children, child i entering as the point mu_{i,r} with log-weight
- * bias_{i,r}; the rightmost node of a level may have fewer than c children.
- * mu is rounded to dtype once computed; parents read the rounded children.
+ * children, child i entering as the point mu_{i,r} with log-weight F_{i,r},
+ * its log-mass at r (see zha_tree_level_logmass); the rightmost node of a
+ * level may have fewer than c children. mu is rounded to dtype once
+ * computed; parents read the rounded children.
  */
 ZHA_API zha_status zha_tree_build(const zha_config *cfg, void *tree, const void *K, const void *refs,
                           const int32_t *lens, int32_t *dev_status, void *stream);

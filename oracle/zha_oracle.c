@@ -33,9 +33,14 @@
  *      (This is the first-order expansion of F(q) = log sum_t e^{s q.k_t}
  *      at q = r, since grad F(r) = s mu.)
  *   R2 parent rule: a parent applies R1 to its children, child i acting as
- *      one point at mu_{i,r} carrying log-weight b_{i,r}, with the SAME r:
- *      l_i = s r.mu_{i,r} + b_{i,r}. In exact arithmetic this equals R1 over
- *      all raw keys under the parent.
+ *      one point at its summary key mu_{i,r} (as stored) carrying, as
+ *      log-weight, its log-mass at the SAME reference r,
+ *      l_i = F_{i,r} = log sum over the keys under child i of e^{s r.k}
+ *      (the child's plane evaluated at r, where it is exact: in exact
+ *      arithmetic F_{i,r} = s r.mu_{i,r} + b_{i,r}); F = log sum_i e^{l_i},
+ *      mu = sum_i e^{l_i - F} mu_{i,r}, b = F - s r.mu. Every node keeps its
+ *      F beside its planes. In exact arithmetic this equals R1 over all raw
+ *      keys under the parent.
  *   R3 only complete leaf chunks enter the tree: n_1 = floor(N/c); a node at
  *      level l > 1 exists iff at least one of its children exists, and uses
  *      only the existing ones: n_l = ceil(n_{l-1}/c).
@@ -186,7 +191,7 @@ int64_t orc_level_nodes(int64_t N, int c, int level)
  * log-weights a[i] (a == NULL: all zero, i.e. raw keys).
  */
 static void plane_one_ref(int64_t n, int d, const double *const *x, const double *a,
-                          const double *r, double s, double *mu, double *b)
+                          const double *r, double s, double *mu, double *b, double *F_out)
 {
     double *l = (double *)malloc((size_t)n * sizeof(double));
     double lmax = -INFINITY;
@@ -207,7 +212,35 @@ static void plane_one_ref(int64_t n, int d, const double *const *x, const double
             mu[k] += w * x[i][k];
     }
     *b = F - s * dot(r, mu, d);
+    if (F_out)
+        *F_out = F;
     free(l);
+}
+
+/*
+ * R2 for ONE reference r over n children: points x[i] (their summary keys)
+ * whose log-weights are their log-masses lw[i] at r.
+ */
+static void plane_from_children(int64_t n, int d, const double *const *x, const double *lw,
+                                const double *r, double s, double *mu, double *b, double *F_out)
+{
+    double lmax = -INFINITY;
+    for (int64_t i = 0; i < n; ++i)
+        if (lw[i] > lmax)
+            lmax = lw[i];
+    double sum = 0.0;
+    for (int64_t i = 0; i < n; ++i)
+        sum += exp(lw[i] - lmax);
+    double F = lmax + log(sum);
+    for (int k = 0; k < d; ++k)
+        mu[k] = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        double w = exp(lw[i] - F);
+        for (int k = 0; k < d; ++k)
+            mu[k] += w * x[i][k];
+    }
+    *b = F - s * dot(r, mu, d);
+    *F_out = F;
 }
 
 /*
@@ -223,28 +256,29 @@ void orc_direct_planes(const double *K, int64_t t0, int64_t t1, int d,
     for (int64_t i = 0; i < n; ++i)
         x[i] = K + (t0 + i) * d;
     for (int r = 0; r < R; ++r)
-        plane_one_ref(n, d, x, NULL, refs + (int64_t)r * d, s, mu + (int64_t)r * d, b + r);
+        plane_one_ref(n, d, x, NULL, refs + (int64_t)r * d, s, mu + (int64_t)r * d, b + r, NULL);
     free(x);
 }
 
 /*
- * R2 for one parent from given children: cmu [nch][R][d] and cb [nch][R]
- * (for instance the children a GPU stored), with the result stored as
- * `storage` would keep it. mu: [R][d], b: [R].
+ * R2 for one parent from given children: cmu [nch][R][d] and their log-masses
+ * cF [nch][R] (for instance the children a GPU stored), with the result
+ * stored as `storage` would keep it. mu: [R][d], b: [R], F: [R].
  */
-void orc_parent_planes(const double *cmu, const double *cb, int64_t nch, int d,
-                       const double *refs, int R, double s, int storage, double *mu, double *b)
+void orc_parent_planes(const double *cmu, const double *cF, int64_t nch, int d,
+                       const double *refs, int R, double s, int storage, double *mu, double *b, double *F)
 {
     const double **x = (const double **)malloc((size_t)nch * sizeof(double *));
     double *a = (double *)malloc((size_t)nch * sizeof(double));
     for (int r = 0; r < R; ++r) {
         for (int64_t i = 0; i < nch; ++i) {
             x[i] = cmu + (i * R + r) * d;
-            a[i] = cb[i * R + r];
+            a[i] = cF[i * R + r];
         }
-        plane_one_ref(nch, d, x, a, refs + (int64_t)r * d, s, mu + (int64_t)r * d, b + r);
+        plane_from_children(nch, d, x, a, refs + (int64_t)r * d, s, mu + (int64_t)r * d, b + r, F + r);
         store_plane(mu + (int64_t)r * d, d, storage);
         b[r] = store_round(b[r], storage == ORC_STORE_F64 ? ORC_STORE_F64 : ORC_STORE_F32);
+        F[r] = store_round(F[r], storage == ORC_STORE_F64 ? ORC_STORE_F64 : ORC_STORE_F32);
     }
     free(a);
     free(x);
@@ -252,7 +286,8 @@ void orc_parent_planes(const double *cmu, const double *cb, int64_t nch, int d,
 
 /*
  * Build or extend the tree of ONE (sequence, KV head) from old_N to new_N
- * tokens. mu[l-1]: [n_l][R][d], b[l-1]: [n_l][R] for the caller's capacity.
+ * tokens. mu[l-1]: [n_l][R][d], b[l-1]: [n_l][R], F[l-1]: [n_l][R] (each
+ * plane's log-mass at its reference) for the caller's capacity.
  * Nodes that a longer cache adds or changes are (R3) the new leaf chunks and,
  * at each level above, every node from the parent of the first changed child
  * to the last node; those are recomputed, everything else is left as is.
@@ -260,7 +295,7 @@ void orc_parent_planes(const double *cmu, const double *cb, int64_t nch, int d,
  */
 void orc_tree_update(const double *K, int64_t old_N, int64_t new_N, int d,
                      const double *refs, int R, int c, int L, double s, int storage,
-                     double **mu, double **b)
+                     double **mu, double **b, double **F)
 {
     int64_t lo = old_N / c;              /* first leaf that is new */
     int64_t hi = new_N / c;              /* leaves after the update */
@@ -276,9 +311,11 @@ void orc_tree_update(const double *K, int64_t old_N, int64_t new_N, int d,
         for (int r = 0; r < R; ++r) {
             double *m = mu[0] + (j * R + r) * d;
             double *bb = b[0] + j * R + r;
-            plane_one_ref(c, d, xp, NULL, refs + (int64_t)r * d, s, m, bb);
+            double *ff = F[0] + j * R + r;
+            plane_one_ref(c, d, xp, NULL, refs + (int64_t)r * d, s, m, bb, ff);
             store_plane(m, d, storage);
             *bb = store_round(*bb, storage == ORC_STORE_F64 ? ORC_STORE_F64 : ORC_STORE_F32);
+            *ff = store_round(*ff, storage == ORC_STORE_F64 ? ORC_STORE_F64 : ORC_STORE_F32);
         }
         if (xp != x)
             free(xp);
@@ -289,7 +326,7 @@ void orc_tree_update(const double *K, int64_t old_N, int64_t new_N, int d,
         lo = lo / c;
         int64_t nl = (nprev + c - 1) / c;
         const double *cmu = mu[l - 2];
-        const double *cb = b[l - 2];
+        const double *cF = F[l - 2];
 #pragma omp parallel for schedule(dynamic, 16)
         for (int64_t p = lo; p < nl; ++p) {
             int64_t c0 = p * c;
@@ -302,13 +339,15 @@ void orc_tree_update(const double *K, int64_t old_N, int64_t new_N, int d,
             for (int r = 0; r < R; ++r) {
                 for (int64_t i = 0; i < nch; ++i) {
                     xp[i] = cmu + ((c0 + i) * R + r) * d;
-                    ap[i] = cb[(c0 + i) * R + r];
+                    ap[i] = cF[(c0 + i) * R + r];
                 }
                 double *m = mu[l - 1] + (p * R + r) * d;
                 double *bb = b[l - 1] + p * R + r;
-                plane_one_ref(nch, d, xp, ap, refs + (int64_t)r * d, s, m, bb);
+                double *ff = F[l - 1] + p * R + r;
+                plane_from_children(nch, d, xp, ap, refs + (int64_t)r * d, s, m, bb, ff);
                 store_plane(m, d, storage);
                 *bb = store_round(*bb, storage == ORC_STORE_F64 ? ORC_STORE_F64 : ORC_STORE_F32);
+                *ff = store_round(*ff, storage == ORC_STORE_F64 ? ORC_STORE_F64 : ORC_STORE_F32);
             }
             if (xp != x)
                 free(xp);

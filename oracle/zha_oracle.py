@@ -56,12 +56,12 @@ def lib():
         L.orc_e4m3_round.argtypes = [f64]
         L.orc_e4m3_round.restype = f64
         L.orc_mx_round.argtypes = [P, i32, P]
-        L.orc_parent_planes.argtypes = [P, P, i64, i32, P, i32, f64, i32, P, P]
+        L.orc_parent_planes.argtypes = [P, P, i64, i32, P, i32, f64, i32, P, P, P]
         L.orc_num_threads.restype = i32
         L.orc_level_nodes.argtypes = [i64, i32, i32]
         L.orc_level_nodes.restype = i64
         L.orc_direct_planes.argtypes = [P, i64, i64, i32, P, i32, f64, P, P]
-        L.orc_tree_update.argtypes = [P, i64, i64, i32, P, i32, i32, i32, f64, i32, P, P]
+        L.orc_tree_update.argtypes = [P, i64, i64, i32, P, i32, i32, i32, f64, i32, P, P, P]
         L.orc_estimate.argtypes = [P, P, P, i32, i32, f64]
         L.orc_estimate.restype = f64
         L.orc_topp_select.argtypes = [i64, P, f64, P, P]
@@ -118,7 +118,9 @@ def level_nodes(N: int, c: int, level: int) -> int:
 
 @dataclass
 class Tree:
-    """Summary tree of one (sequence, KV head): mu[l-1] [cap_l, R, d], b[l-1] [cap_l, R]."""
+    """Summary tree of one (sequence, KV head): mu[l-1] [cap_l, R, d], b[l-1] [cap_l, R],
+    F[l-1] [cap_l, R] (each plane's log-mass at its reference, which parents weight
+    their children by)."""
     c: int
     L: int
     R: int
@@ -128,6 +130,7 @@ class Tree:
     N: int = 0
     mu: list = field(default_factory=list)
     b: list = field(default_factory=list)
+    F: list = field(default_factory=list)
 
     def n(self, level: int) -> int:
         return level_nodes(self.N, self.c, level)
@@ -141,6 +144,7 @@ def new_tree(cap_tokens: int, c: int, L: int, R: int, d: int, s: float | None = 
         n = max(level_nodes(cap_tokens, c, level), 1)
         t.mu.append(np.zeros((n, R, d)))
         t.b.append(np.zeros((n, R)))
+        t.F.append(np.zeros((n, R)))
     return t
 
 
@@ -152,8 +156,9 @@ def tree_update(tree: Tree, K: np.ndarray, refs: np.ndarray, new_N: int) -> Tree
     assert tree.mu[0].shape[0] >= level_nodes(new_N, tree.c, 1) or level_nodes(new_N, tree.c, 1) == 0
     mus = (ctypes.c_void_p * tree.L)(*[m.ctypes.data for m in tree.mu])
     bs = (ctypes.c_void_p * tree.L)(*[b.ctypes.data for b in tree.b])
+    Fs = (ctypes.c_void_p * tree.L)(*[f.ctypes.data for f in tree.F])
     lib().orc_tree_update(_ptr(K), int(tree.N), int(new_N), tree.d, _ptr(refs), tree.R, tree.c,
-                          tree.L, tree.s, _STORAGE[tree.storage], mus, bs)
+                          tree.L, tree.s, _STORAGE[tree.storage], mus, bs, Fs)
     tree.N = int(new_N)
     return tree
 
@@ -177,15 +182,18 @@ def direct_planes(K: np.ndarray, t0: int, t1: int, refs: np.ndarray, s: float):
     return mu, b
 
 
-def parent_planes(child_mu: np.ndarray, child_b: np.ndarray, refs: np.ndarray, s: float,
+def parent_planes(child_mu: np.ndarray, child_F: np.ndarray, refs: np.ndarray, s: float,
                   storage: str = "f64"):
-    """Planes of one parent from given children (child_mu [n, R, d], child_b [n, R])."""
-    cm, cb, refs = _f64(child_mu), _f64(child_b), _f64(refs)
+    """Planes of one parent from given children (child_mu [n, R, d] and their
+    log-masses child_F [n, R]) -> (mu [R, d], b [R], F [R])."""
+    cm, cf, refs = _f64(child_mu), _f64(child_F), _f64(refs)
     n, R, d = cm.shape
     mu = np.zeros((R, d))
     b = np.zeros(R)
-    lib().orc_parent_planes(_ptr(cm), _ptr(cb), n, d, _ptr(refs), R, float(s), _STORAGE[storage], _ptr(mu), _ptr(b))
-    return mu, b
+    F = np.zeros(R)
+    lib().orc_parent_planes(_ptr(cm), _ptr(cf), n, d, _ptr(refs), R, float(s), _STORAGE[storage], _ptr(mu),
+                            _ptr(b), _ptr(F))
+    return mu, b, F
 
 
 def estimate(q: np.ndarray, mu: np.ndarray, b: np.ndarray, s: float) -> float:

@@ -45,4 +45,4 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
     for f in flips:
         tr.write_line(f"  {f['test']} group {f['group']} level {f['level']} head {f['head']} node {f['node']}: "
                       f"running mass before it {f['cum_before']:.7f}, p {f['p']}, |diff| {f['dist']:.2e} "
-                      f"(band {f['band']:.2e}), kept by the {f['kept_by']} only")
+                      f"(band {f['band']:.2e}, near-tie mass {f['near_tie_mass']:.2e}), kept by the {f['kept_by']} only")

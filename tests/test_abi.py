@@ -114,7 +114,8 @@ def test_p_schedule_host_rule(zha, orc):
 
 def test_mx_summary_config_and_layout(zha):
     """MX-FP8 summaries need bf16 KV; their records take R*d + R*d/32 + 4R bytes
-    (2,176 at R=16, d=128) instead of R*2d + 4R (4,160), and the block scales
+    (2,176 at R=16, d=128) instead of R*2d + 4R (4,160), plus 4R bytes of each
+    plane's value at its own reference in both formats, and the block scales
     have their own offset, which the native format refuses."""
     with pytest.raises(zha.ZhaError):
         zha.config(1, 2, 1, 64, 4, 3, 16, "f32", 4096, summary="mxfp8")
@@ -127,6 +128,6 @@ def test_mx_summary_config_and_layout(zha):
     off = ctypes.c_size_t()
     assert zha.lib().zha_tree_level_scales(ctypes.byref(mx), 1, ctypes.byref(off)) == 0
     assert mu_off == 0 and off.value >= n1 * 16 * 128 and b_off >= off.value + n1 * 16 * 4
-    assert zha.tree_bytes(mx) == pytest.approx(n1 * 2176, rel=0.01)
-    assert zha.tree_bytes(nat) == pytest.approx(n1 * 4160, rel=0.01)
+    assert zha.tree_bytes(mx) == pytest.approx(n1 * (2176 + 64), rel=0.01)
+    assert zha.tree_bytes(nat) == pytest.approx(n1 * (4160 + 64), rel=0.01)
     assert zha.lib().zha_tree_level_scales(ctypes.byref(nat), 1, ctypes.byref(off)) == 1

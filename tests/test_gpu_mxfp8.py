@@ -46,8 +46,9 @@ def _flips_within_one_step(got, ref, X):
 
 def _check_mx_level(buf, level, b, kvh, n, t, w, inp, s):
     """Level 1 against the oracle's leaves (same raw keys); a level above
-    against the oracle's parent rule applied to the GPU's own stored children,
-    so that each level is checked on its own inputs."""
+    against the oracle's parent rule applied to the GPU's own stored children
+    (summary keys and log-masses), so that each level is checked on its own
+    inputs."""
     mu8, b_g = buf.tree_level(level)
     sc = buf.tree_level_scales(level)[b, kvh, :n]
     got = T.mx_decode(mu8[b, kvh, :n], sc)
@@ -60,15 +61,17 @@ def _check_mx_level(buf, level, b, kvh, n, t, w, inp, s):
         ref, bref = t.mu[0][:n], t.b[0][:n]
     else:
         n_below = orc.level_nodes(int(inp.lens[b]), w.chunk, level - 1)
-        cmu8, cb = buf.tree_level(level - 1)
+        cmu8, _ = buf.tree_level(level - 1)
         kids = T.mx_decode(cmu8[b, kvh, :n_below], buf.tree_level_scales(level - 1)[b, kvh, :n_below])
-        kb = T.np64(cb[b, kvh, :n_below])
+        kF = T.np64(buf.tree_level_logmass(level - 1)[b, kvh, :n_below])
         refs = T.np64(inp.refs[kvh])
         ref = np.zeros_like(got)
         bref = np.zeros_like(bg)
+        Fref = np.zeros_like(bg)
         for node in range(n):
             c0, c1 = node * w.chunk, min(node * w.chunk + w.chunk, n_below)
-            ref[node], bref[node] = orc.parent_planes(kids[c0:c1], kb[c0:c1], refs, s, "mxfp8")
+            ref[node], bref[node], Fref[node] = orc.parent_planes(kids[c0:c1], kF[c0:c1], refs, s, "mxfp8")
+        assert T.rel_err(T.np64(buf.tree_level_logmass(level)[b, kvh, :n]), Fref) <= 1e-5
     _flips_within_one_step(got, ref, X)
     eb = T.rel_err(bg, bref)
     assert eb <= 1e-4, eb

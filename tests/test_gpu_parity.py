@@ -56,12 +56,15 @@ def test_tree_build_matches_oracle(zha, w):
                 mu_g, b_g = buf.tree_level(level)
                 emu = T.rel_err(T.np64(mu_g[b, kvh, :n]), t.mu[level - 1][:n])
                 eb = T.rel_err(T.np64(b_g[b, kvh, :n]), t.b[level - 1][:n])
-                assert emu <= tol and eb <= tol, (b, kvh, level, emu, eb)
+                eF = T.rel_err(T.np64(buf.tree_level_logmass(level)[b, kvh, :n]), t.F[level - 1][:n])
+                assert emu <= tol and eb <= tol and eF <= tol, (b, kvh, level, emu, eb, eF)
 
 
-@pytest.mark.parametrize("w", [CASES[0], CASES[1], CASES[3]], ids=[IDS[0], IDS[1], IDS[3]])
+@pytest.mark.parametrize("w", CASES, ids=IDS)
 @pytest.mark.parametrize("block", [1, 3, 4, 9, 1000, 4096])
 def test_append_equals_build_bitexact(zha, w, block):
+    """Appending in blocks (decode-sized ones through the single-leaf path,
+    larger ones through the bulk leaf kernel) equals a build at once, bit for bit."""
     cfg, inp, dev, buf = T.build_case(zha, w)
     N = w.context
     ref = zha.Buffers(cfg)
@@ -82,6 +85,7 @@ def test_append_equals_build_bitexact(zha, w, block):
         mu_r, b_r = ref.tree_level(level)
         assert torch.equal(mu_a[:, :, :k], mu_r[:, :, :k]), level
         assert torch.equal(b_a[:, :, :k], b_r[:, :, :k]), level
+        assert torch.equal(buf.tree_level_logmass(level)[:, :, :k], ref.tree_level_logmass(level)[:, :, :k]), level
 
 
 # ------------------------------------------------------------- top-p select

@@ -144,7 +144,8 @@ def test_parent_rule_equals_direct_planes(orc, N, c, L):
 
 
 def test_parent_rule_wrong_variant_would_fail(orc):
-    """The same check rejects a parent that ignores its children's biases."""
+    """The same check rejects a parent that treats its children as plain keys,
+    or weights them by their plane offsets (biases) instead of their log-masses."""
     d, R, c = 8, 3, 4
     K = _keys(9, 64, d, c)
     refs = rng(10).normal(size=(R, d))
@@ -154,7 +155,34 @@ def test_parent_rule_wrong_variant_would_fail(orc):
     # a parent built from children as plain keys (no log-weights) differs
     mu_plain, b_plain = orc.direct_planes(t.mu[0][0:4, 0], 0, 4, refs[:1], s)
     assert not np.isclose(b_plain[0], b_direct[0], rtol=1e-6)
+    # ... and so does one that weights them by their biases
+    mu_b, b_b, _ = orc.parent_planes(t.mu[0][0:4], t.b[0][0:4], refs, s)
+    assert not np.allclose(b_b, b_direct, rtol=1e-6)
+    mu_f, b_f, _ = orc.parent_planes(t.mu[0][0:4], t.F[0][0:4], refs, s)
+    assert np.allclose(mu_f, mu_direct, rtol=1e-10, atol=1e-10) and np.allclose(b_f, b_direct, rtol=1e-10)
     assert np.isclose(t.b[1][0, 0], b_direct[0], rtol=1e-10)
+
+
+@pytest.mark.parametrize("N,c,L", [(4096, 4, 3), (777, 8, 3), (300, 256, 1)])
+def test_node_logmass_is_exact_log_sum_exp(orc, N, c, L):
+    """Each node's kept log-mass F_r is log sum e^{s r.k} over its raw keys
+    (scipy), and equals its plane's value at its own reference."""
+    from scipy.special import logsumexp
+    d, R = 16, 3
+    K = _keys(N + 5, N, d, c)
+    refs = rng(N + 6).normal(size=(R, d)) * 0.7
+    s = 1.0 / math.sqrt(d)
+    t = orc.build_tree(K, refs, N, c, L, s)
+    n1 = N // c
+    for level in range(1, L + 1):
+        span = c ** level
+        for n in range(0, t.n(level), max(1, t.n(level) // 7)):
+            t0, t1 = n * span, min((n + 1) * span, n1 * c)
+            for r in range(R):
+                exact = logsumexp(s * K[t0:t1] @ refs[r])
+                assert abs(t.F[level - 1][n, r] - exact) <= 1e-11 * max(1.0, abs(exact))
+                own = s * refs[r] @ t.mu[level - 1][n, r] + t.b[level - 1][n, r]
+                assert abs(own - exact) <= 1e-11 * max(1.0, abs(exact))
 
 
 @pytest.mark.parametrize("block", [1, 3, 4, 37, 4096])
@@ -497,8 +525,9 @@ def test_mxfp8_storage_tree_builds_from_rounded_children(orc):
     for level in range(1, L):
         for node in range(t.n(level + 1)):
             c0, c1 = node * c, min(node * c + c, t.n(level))
-            pm, pb = orc.parent_planes(t.mu[level - 1][c0:c1], t.b[level - 1][c0:c1], refs, s, "mxfp8")
+            pm, pb, pf = orc.parent_planes(t.mu[level - 1][c0:c1], t.F[level - 1][c0:c1], refs, s, "mxfp8")
             assert np.array_equal(pm, t.mu[level][node]) and np.array_equal(pb, t.b[level][node])
+            assert np.array_equal(pf, t.F[level][node])
     # estimates stay close to the exact tree's (the router's purpose)
     q = rng(94).normal(size=d)
     for level in range(L):

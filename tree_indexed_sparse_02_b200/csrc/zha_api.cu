@@ -71,6 +71,8 @@ Geo make_geo(const zha_config *c, int T = 1) {
         }
         g.bias_off[l] = off;
         off = align256(off + groups * g.cap[l] * g.R * sizeof(float));
+        g.lm_off[l] = off;
+        off = align256(off + groups * g.cap[l] * g.R * sizeof(float));
     }
     g.tree_bytes = off;
     off = 0;
@@ -184,6 +186,14 @@ zha_status zha_tree_level_offsets(const zha_config *cfg, int32_t level, size_t *
     Geo g = make_geo(cfg);
     *mu_off = g.mu_off[level];
     *bias_off = g.bias_off[level];
+    return ZHA_OK;
+}
+
+zha_status zha_tree_level_logmass(const zha_config *cfg, int32_t level, size_t *lm_off) {
+    zha_status s = check_config(cfg);
+    if (s != ZHA_OK) return s;
+    if (!lm_off || level < 1 || level > cfg->levels) return ZHA_ERR_INVALID_ARG;
+    *lm_off = make_geo(cfg).lm_off[level];
     return ZHA_OK;
 }
 

@@ -45,6 +45,7 @@ struct Geo {
     size_t mu_off[kMaxLevels + 1];      // tree buffer offsets
     size_t bias_off[kMaxLevels + 1];
     size_t sc_off[kMaxLevels + 1];      // MX-FP8 block scales (0 for the native format)
+    size_t lm_off[kMaxLevels + 1];      // each plane's log-mass at its own reference (fp32)
     size_t tree_bytes;
     // workspace
     size_t ws_cand[kMaxLevels + 1], ws_cmask[kMaxLevels + 1], ws_scores[kMaxLevels + 1],

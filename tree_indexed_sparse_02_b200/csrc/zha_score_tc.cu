@@ -25,10 +25,7 @@
 // Every mbarrier wait is bounded; on expiry the kernel records
 // ZHA_ERR_TIMEOUT, stops issuing work, lets copies in flight land, frees its
 // tensor memory and returns.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "zha_common.cuh"
+#include "zha_tc.cuh"
 
 namespace zha {
 
@@ -50,102 +47,13 @@ constexpr int kTcSmem = kTcStages * kStageBytes + kMetaSlots * kMetaBytes + kMax
 constexpr uint32_t kTmemCols = 32;
 constexpr long long kWaitCycles = 4000000000ll;  // ~2 s at the boost clock
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, N = 16, M = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
-// 1024 bytes apart.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
-    return (uint64_t)((addr & 0x3ffffu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
-           (2ull << 61);
-}
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
+constexpr uint32_t kIdesc = tc_idesc_bf16(16);
 
 // Bounded wait: false if the barrier did not complete in time or the CTA is
 // aborting (then also raises the abort flag and the status).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
                                           int32_t *status) {
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort) return false;
-        if (clock64() - t0 > kWaitCycles) {
-            *abort = 1;
-            set_status(status, ZHA_ERR_TIMEOUT);
-            return false;
-        }
-    }
-    return true;
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-        : "memory");
-}
-
-// Plain (untiled) bulk copy, global -> shared, completing on an mbarrier.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-}
-
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
-        "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate));
-}
-
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+    return mbar_wait_bounded(bar, parity, kWaitCycles, abort, status);
 }
 
 struct TcArgs {
@@ -255,12 +163,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap mu_map, Geo g, TcArgs a) {
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // q stores -> async proxy
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_slot)),
-                     "r"(kTmemCols));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
-    }
+    fence_proxy_async_smem();  // q stores -> async proxy
+    if (warp == 1) tc_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -373,7 +277,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap mu_map, Geo g, TcArgs a) {
                     const uint32_t off = (kk & 3) * 32;
                     const uint64_t ad = smem_desc(abase + (kk >> 2) * kHalfBytes + off);
                     const uint64_t bd = smem_desc(qbase + grp * kQBytes + (kk >> 2) * 2048 + off);
-                    tc_mma(tmem + acc * 16, ad, bd, kk > 0 ? 1u : 0u);
+                    tc_mma(tmem + acc * 16, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(empty0 + 8 * s);     // A stage free once these MMAs have read it
                 tc_commit(tfull0 + 8 * acc);
@@ -460,11 +364,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap mu_map, Geo g, TcArgs a) {
         }
     }
     tc_fence_after();
-    if (warp == 1)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
+    if (warp == 1) tc_dealloc(tmem, kTmemCols);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+}  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
         cudaDriverEntryPointQueryResult q;
@@ -476,11 +381,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-}  // namespace
 
 bool score_tc_supported(const Geo &g) {
     return g.dtype == ZHA_BF16 && !g.mx() && g.T == 1 && g.lag == 0 && g.d == 128 && g.R == 16 && g.G <= 16 && g.groups() <= kMaxGroups &&
-           encode_fn() != nullptr;
+           tensor_map_encoder() != nullptr;
 }
 
 // One level of scoring on tcgen05; the layout of the inputs and outputs is
@@ -506,7 +410,7 @@ cudaError_t launch_score_tc(const Geo &g, const void *mu_level, const float *bia
     const cuuint64_t strides[1] = {128 * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)(kRows / runs)};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode_fn()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(mu_level), dims, strides,
+    CUresult r = tensor_map_encoder()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(mu_level), dims, strides,
                              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;

@@ -71,6 +71,7 @@ def _load():
         "zha_tree_bytes": ([CP], sz),
         "zha_tree_level_offsets": ([CP, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)], i32),
         "zha_tree_level_scales": ([CP, i32, ctypes.POINTER(sz)], i32),
+        "zha_tree_level_logmass": ([CP, i32, ctypes.POINTER(sz)], i32),
         "zha_workspace_bytes": ([CP], sz),
         "zha_workspace_level_view": ([CP, i32, ctypes.POINTER(LevelView)], i32),
         "zha_workspace_level_view_block": ([CP, i32, i32, ctypes.POINTER(LevelView)], i32),
@@ -331,6 +332,17 @@ class Buffers:
         n = cfg.batch * cfg.n_kv_heads * cap * cfg.n_refs * (cfg.head_dim // 32)
         return self.tree[off.value:off.value + n].view(cfg.batch, cfg.n_kv_heads, cap, cfg.n_refs,
                                                         cfg.head_dim // 32)
+
+    def tree_level_logmass(self, level: int):
+        """Log-masses F [B, Hkv, cap, R] of one level (each plane's log attention
+        mass at its own reference)."""
+        cfg = self.cfg
+        off = ctypes.c_size_t()
+        check(_lib.zha_tree_level_logmass(ctypes.byref(cfg), level, ctypes.byref(off)), "zha_tree_level_logmass")
+        cap = level_nodes(cfg, cfg.max_len, level)
+        n = cfg.batch * cfg.n_kv_heads * cap * cfg.n_refs
+        return self.tree[off.value:off.value + n * 4].view(torch.float32).view(cfg.batch, cfg.n_kv_heads, cap,
+                                                                               cfg.n_refs)
 
     def level_state(self, level: int, T: int = 1):
         """Routing state of one level from the last route/decode call (T: query
