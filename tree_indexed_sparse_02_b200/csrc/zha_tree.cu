@@ -55,21 +55,50 @@ struct TreePtrs {
     float *lm[kMaxLevels + 1];      // each plane's log-mass F at its reference
 };
 
-// d = fma(a, b, d) on two fp32 lanes at once (one packed instruction on sm_100)
-__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
-    unsigned long long ra, rb, rd;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a0), "f"(a1));
-    asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b0), "f"(b1));
-    asm("mov.b64 %0, {%1, %2};" : "=l"(rd) : "f"(d0), "f"(d1));
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(rd) : "l"(ra), "l"(rb));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(rd));
+// Two fp32 values in one 64-bit register pair, for the packed fp32
+// instructions of sm_100 (fma.rn.f32x2: two FMAs per instruction).
+typedef unsigned long long f2x;
+__device__ __forceinline__ f2x pk2(float lo, float hi) {
+    f2x r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 upk2(f2x v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ f2x fma2(f2x a, f2x b, f2x c) {
+    f2x d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ f2x mul2(f2x a, f2x b) {
+    f2x d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// bf16 pair (element 0 in the low half) -> packed fp32 pair
+__device__ __forceinline__ f2x bf2_to_f2x(uint32_t w) {
+    return pk2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
-// acc[e] = fma(w, x[e], acc[e]) for every e, two at a time.
-template <int E>
-__device__ __forceinline__ void axpy(float (&acc)[E], float w, const float (&x)[E]) {
+// acc[e] = fma(w, x[e], acc[e]) for every pair e.
+template <int H>
+__device__ __forceinline__ void axpy2(f2x (&acc)[H], float w, const f2x (&x)[H]) {
+    const f2x ww = pk2(w, w);
 #pragma unroll
-    for (int e = 0; e < E; e += 2) ffma2(acc[e], acc[e + 1], w, w, x[e], x[e + 1]);
+    for (int e = 0; e < H; ++e) acc[e] = fma2(ww, x[e], acc[e]);
+}
+template <int H, int E>
+__device__ __forceinline__ void unpack_all(const f2x (&v)[H], float (&out)[E]) {
+    static_assert(2 * H == E, "");
+#pragma unroll
+    for (int e = 0; e < H; ++e) {
+        const float2 f = upk2(v[e]);
+        out[2 * e] = f.x;
+        out[2 * e + 1] = f.y;
+    }
 }
 
 // ------------------------------------------------------------ loads and stores
@@ -205,6 +234,31 @@ struct RawPoints {        // keys of a leaf chunk, or children kept in the KV dt
     __device__ __forceinline__ void load(int i, int sl, float (&x)[E]) const {
         load_n<E>(x0 + (int64_t)i * stride + sl * E, x);
     }
+    __device__ __forceinline__ void load2(int i, int sl, f2x (&x)[E / 2]) const {
+        const T *p = x0 + (int64_t)i * stride + sl * E;
+        if constexpr (sizeof(T) == 2 && E % 8 == 0) {
+#pragma unroll
+            for (int e = 0; e < E; e += 8) {
+                const uint4 t = *reinterpret_cast<const uint4 *>(p + e);
+                x[e / 2] = bf2_to_f2x(t.x);
+                x[e / 2 + 1] = bf2_to_f2x(t.y);
+                x[e / 2 + 2] = bf2_to_f2x(t.z);
+                x[e / 2 + 3] = bf2_to_f2x(t.w);
+            }
+        } else if constexpr (sizeof(T) == 2) {
+            static_assert(E == 4, "coordinates per lane: 4 or a multiple of 8");
+            const uint2 t = *reinterpret_cast<const uint2 *>(p);   // 8 bytes, 8-byte aligned
+            x[0] = bf2_to_f2x(t.x);
+            x[1] = bf2_to_f2x(t.y);
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; e += 4) {
+                const float4 t = *reinterpret_cast<const float4 *>(p + e);
+                x[e / 2] = pk2(t.x, t.y);
+                x[e / 2 + 1] = pk2(t.z, t.w);
+            }
+        }
+    }
 };
 
 template <int E>
@@ -226,6 +280,12 @@ struct Mx8Points {        // children kept as MX-FP8 (E4M3 bytes + one scale per
             x[e0 + 2] = hi.x * sc;
             x[e0 + 3] = hi.y * sc;
         }
+    }
+    __device__ __forceinline__ void load2(int i, int sl, f2x (&x)[E / 2]) const {
+        float v[E];
+        load(i, sl, v);
+#pragma unroll
+        for (int e = 0; e < E; e += 2) x[e / 2] = pk2(v[e], v[e + 1]);
     }
 };
 
@@ -337,16 +397,19 @@ __device__ __forceinline__ void sub_plane_np(const P &pts, const float *a0, int6
 // loaded before any arithmetic; NP = 0: any number, streamed.
 template <int NP, class P, int E>
 __device__ __forceinline__ void parent_plane(const P &pts, const float *lm0, int64_t stride, int npts,
-                                             float (&acc)[E], float &F_out, int sl) {
+                                             float (&out)[E], float &F_out, int sl) {
+    constexpr int H = E / 2;
     float z = 0.f, m = -INFINITY;
+    f2x acc[H];
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    for (int e = 0; e < H; ++e) acc[e] = 0ull;
     if constexpr (NP > 0) {
-        float x[NP][E], l[NP];
+        f2x x[NP][H];
+        float l[NP];
 #pragma unroll
         for (int i = 0; i < NP; ++i) {
             if (i < npts) {
-                pts.load(i, sl, x[i]);
+                pts.load2(i, sl, x[i]);
                 l[i] = lm0[(int64_t)i * stride];
                 m = fmaxf(m, l[i]);
             }
@@ -356,21 +419,23 @@ __device__ __forceinline__ void parent_plane(const P &pts, const float *lm0, int
             if (i >= npts) continue;
             const float w = expf(l[i] - m);
             z += w;
-            axpy<E>(acc, w, x[i]);
+            axpy2<H>(acc, w, x[i]);
         }
     } else {
         for (int i = 0; i < npts; ++i) m = fmaxf(m, lm0[(int64_t)i * stride]);
         for (int i = 0; i < npts; ++i) {
-            float x[E];
-            pts.load(i, sl, x);
+            f2x x[H];
+            pts.load2(i, sl, x);
             const float w = expf(lm0[(int64_t)i * stride] - m);
             z += w;
-            axpy<E>(acc, w, x);
+            axpy2<H>(acc, w, x);
         }
     }
     const float inv = 1.f / z;
+    const f2x ii = pk2(inv, inv);
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] *= inv;
+    for (int e = 0; e < H; ++e) acc[e] = mul2(acc[e], ii);
+    unpack_all(acc, out);
     F_out = m + logf(z);
 }
 
@@ -481,6 +546,21 @@ __host__ __device__ inline LeafLayout leaf_layout(int d, int R, int c, int tiles
 __host__ __device__ inline uint32_t tmem_cols_for(int npad, int tiles) {
     const int need = npad * tiles;
     return need <= 32 ? 32u : (need <= 64 ? 64u : 128u);
+}
+
+// The same key coordinates as packed fp32 pairs.
+template <int E>
+__device__ __forceinline__ void tile_key2(const uint8_t *A, int d, int row, int k0, f2x (&x)[E / 2]) {
+    const int t = row >> 7, rr = row & 127;
+    const int byte = k0 * 2;
+    const uint8_t *p = A + (size_t)t * kTileRows * d * 2 + swz_offset(rr, byte >> 4, kTileRows) + (byte & 15);
+    if constexpr (E == 4) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(p);
+        x[0] = bf2_to_f2x(v.x);
+        x[1] = bf2_to_f2x(v.y);
+    } else {
+        x[0] = bf2_to_f2x(*reinterpret_cast<const uint32_t *>(p));
+    }
 }
 
 // Key row `row` (0 .. tiles*128) of an item, coordinates k0 .. k0+E-1 (E = 2 or 4), from the swizzled tiles.
@@ -644,11 +724,12 @@ __device__ __forceinline__ void leaf_mu(const Geo &g, const TreePtrs &tp, const 
     const float *W = reinterpret_cast<const float *>(smem + Ly.w);
     const uint8_t *A = smem + Ly.a;
     const int k0 = lane * E;
+    constexpr int H = E / 2;
     if constexpr (C > 0) {
         for (int j = store_lo + warp; j < store_hi; j += nwarps) {
-            float k[C][E];
+            f2x k[C][H];
 #pragma unroll
-            for (int t = 0; t < C; ++t) tile_key<E>(A, g.d, j * C + t, k0, k[t]);
+            for (int t = 0; t < C; ++t) tile_key2<E>(A, g.d, j * C + t, k0, k[t]);
             const int64_t rec0 = (grp * g.cap[1] + leaf0 + j) * (int64_t)R;
             const float *wj = W + j * Ly.wstride;
             for (int r = 0; r < R; ++r) {
@@ -660,12 +741,14 @@ __device__ __forceinline__ void leaf_mu(const Geo &g, const TreePtrs &tp, const 
 #pragma unroll
                     for (int t = 0; t < C; ++t) w[t] = wj[r * C + t];
                 }
-                float acc[E];
+                f2x acc[H];
 #pragma unroll
-                for (int e = 0; e < E; ++e) acc[e] = 0.f;
+                for (int e = 0; e < H; ++e) acc[e] = 0ull;
 #pragma unroll
-                for (int t = 0; t < C; ++t) axpy<E>(acc, w[t], k[t]);
-                store_plane<T, E, MX>(g, tp, 1, rec0 + r, acc, k0, true);
+                for (int t = 0; t < C; ++t) axpy2<H>(acc, w[t], k[t]);
+                float v[E];
+                unpack_all(acc, v);
+                store_plane<T, E, MX>(g, tp, 1, rec0 + r, v, k0, true);
             }
         }
     } else {
@@ -675,25 +758,27 @@ __device__ __forceinline__ void leaf_mu(const Geo &g, const TreePtrs &tp, const 
         const int nrb = (R + rb - 1) / rb;
         for (int u = warp; u < leaves * nrb; u += nwarps) {
             const int j = store_lo + u / nrb, r0 = (u % nrb) * rb;
-            float acc[kRB][E];
+            f2x acc[kRB][H];
 #pragma unroll
             for (int i = 0; i < kRB; ++i)
 #pragma unroll
-                for (int e = 0; e < E; ++e) acc[i][e] = 0.f;
+                for (int e = 0; e < H; ++e) acc[i][e] = 0ull;
             for (int t = 0; t < c; ++t) {
-                float x[E];
-                tile_key<E>(A, g.d, j * c + t, k0, x);
+                f2x x[H];
+                tile_key2<E>(A, g.d, j * c + t, k0, x);
 #pragma unroll
                 for (int i = 0; i < kRB; ++i) {
                     if (i >= rb || r0 + i >= R) break;
-                    axpy<E>(acc[i], W[j * Ly.wstride + (r0 + i) * c + t], x);
+                    axpy2<H>(acc[i], W[j * Ly.wstride + (r0 + i) * c + t], x);
                 }
             }
             const int64_t rec0 = (grp * g.cap[1] + leaf0 + j) * (int64_t)R;
 #pragma unroll
             for (int i = 0; i < kRB; ++i) {
                 if (i >= rb || r0 + i >= R) break;
-                store_plane<T, E, MX>(g, tp, 1, rec0 + r0 + i, acc[i], k0, true);
+                float v[E];
+                unpack_all(acc[i], v);
+                store_plane<T, E, MX>(g, tp, 1, rec0 + r0 + i, v, k0, true);
             }
         }
     }
