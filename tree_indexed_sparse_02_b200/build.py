@@ -17,6 +17,12 @@ FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std
          "-I", INCLUDE]
 
 
+# Per-file flags. The tree kernels compute the same planes in several kernels
+# (bulk build, appends, the decode step's rightmost path) and must agree bit
+# for bit: no implicit a*b+c contraction there (every FMA is written out).
+FILE_FLAGS = {"zha_tree.cu": ["--fmad=false"]}
+
+
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
@@ -43,7 +49,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         fresh = (os.path.exists(obj) and not force and not extra and
                  os.path.getmtime(obj) > max(os.path.getmtime(src), newest_header))
         if not fresh:
-            cmds.append([NVCC, *FLAGS, *extra, "-c", src, "-o", obj])
+            cmds.append([NVCC, *FLAGS, *FILE_FLAGS.get(os.path.basename(src), []), *extra, "-c", src, "-o", obj])
     # the translation units are independent: compile them side by side
     with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
         for cmd in cmds:

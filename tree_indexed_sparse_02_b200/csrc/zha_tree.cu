@@ -44,7 +44,7 @@ constexpr int kItemKeys = 256;            // keys per work item of the leaf kern
 constexpr int kTileRows = 128;            // rows of one MMA tile (M)
 constexpr int kLeafWarps = 8;             // one thread per key of an item
 constexpr int kLevelWarps = 8;
-constexpr int kSub = 16;                  // lanes per plane on the CUDA-core paths
+constexpr int kSub = 8;                   // lanes per plane on the CUDA-core paths
 constexpr int kPerWarp = 32 / kSub;       // planes per warp at a time
 constexpr long long kTreeWait = 2000000000LL;   // ~1 s at the boost clock: a wait that long is an error
 
@@ -71,11 +71,6 @@ __device__ __forceinline__ float2 upk2(f2x v) {
 __device__ __forceinline__ f2x fma2(f2x a, f2x b, f2x c) {
     f2x d;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ f2x mul2(f2x a, f2x b) {
-    f2x d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
 // bf16 pair (element 0 in the low half) -> packed fp32 pair
@@ -393,48 +388,49 @@ __device__ __forceinline__ void sub_plane_np(const P &pts, const float *a0, int6
 // Plane r of a parent from its npts children's planes r: child i enters as
 // its stored summary key x_i with log-weight l_i = F_i, its log-mass at r;
 // F = log sum_i e^{l_i}, w_i = e^{l_i - F}, mu = sum_i w_i x_i (the bias,
-// F - s r.mu, is left to the caller). NP > 0: at most NP children, all
-// loaded before any arithmetic; NP = 0: any number, streamed.
+// F - s r.mu, is left to the caller). The log-masses come first (two passes
+// over npts scalars), then the keys stream in with known weights. NP > 0:
+// at most NP children (unrolled); NP = 0: any number.
 template <int NP, class P, int E>
 __device__ __forceinline__ void parent_plane(const P &pts, const float *lm0, int64_t stride, int npts,
                                              float (&out)[E], float &F_out, int sl) {
     constexpr int H = E / 2;
-    float z = 0.f, m = -INFINITY;
+    float l[NP > 0 ? NP : 1];
+    float m = -INFINITY, z = 0.f;
     f2x acc[H];
 #pragma unroll
     for (int e = 0; e < H; ++e) acc[e] = 0ull;
     if constexpr (NP > 0) {
-        f2x x[NP][H];
-        float l[NP];
 #pragma unroll
-        for (int i = 0; i < NP; ++i) {
+        for (int i = 0; i < NP; ++i)
             if (i < npts) {
-                pts.load2(i, sl, x[i]);
                 l[i] = lm0[(int64_t)i * stride];
                 m = fmaxf(m, l[i]);
             }
-        }
 #pragma unroll
-        for (int i = 0; i < NP; ++i) {
-            if (i >= npts) continue;
-            const float w = expf(l[i] - m);
-            z += w;
-            axpy2<H>(acc, w, x[i]);
-        }
+        for (int i = 0; i < NP; ++i)
+            if (i < npts) {
+                l[i] = expf(l[i] - m);
+                z += l[i];
+            }
+        const float inv = 1.f / z;
+#pragma unroll
+        for (int i = 0; i < NP; ++i)
+            if (i < npts) {
+                f2x x[H];
+                pts.load2(i, sl, x);
+                axpy2<H>(acc, l[i] * inv, x);
+            }
     } else {
         for (int i = 0; i < npts; ++i) m = fmaxf(m, lm0[(int64_t)i * stride]);
+        for (int i = 0; i < npts; ++i) z += expf(lm0[(int64_t)i * stride] - m);
+        const float inv = 1.f / z;
         for (int i = 0; i < npts; ++i) {
             f2x x[H];
             pts.load2(i, sl, x);
-            const float w = expf(lm0[(int64_t)i * stride] - m);
-            z += w;
-            axpy2<H>(acc, w, x);
+            axpy2<H>(acc, expf(lm0[(int64_t)i * stride] - m) * inv, x);
         }
     }
-    const float inv = 1.f / z;
-    const f2x ii = pk2(inv, inv);
-#pragma unroll
-    for (int e = 0; e < H; ++e) acc[e] = mul2(acc[e], ii);
     unpack_all(acc, out);
     F_out = m + logf(z);
 }
@@ -908,10 +904,10 @@ tree_leaf_kernel(const __grid_constant__ CUtensorMap kmap, Geo g, TreePtrs tp, c
         last /= g.c;
         const int64_t n_below = level_nodes(n_now, g.c, level - 1);
         const int64_t nlo = max64(first, lo), nhi = min64(last, level_nodes(n_now, g.c, level));
-        __syncthreads();
+        __syncthreads();   // the level below is written (and visible to this CTA)
         if (nlo < nhi)
             plane_jobs<T, E * 32 / kSub, MX, C>(g, tp, K, refs, grp, level, nlo, nhi, n_below, threadIdx.x >> 5,
-                                     blockDim.x >> 5, threadIdx.x & 31);
+                                                blockDim.x >> 5, threadIdx.x & 31);
     }
 }
 
@@ -1001,7 +997,8 @@ __device__ __forceinline__ void tree_path_levels(const Geo &g, const TreePtrs &t
         const int64_t hi = level_nodes(n_now, g.c, level);
         const int64_t n_below = level_nodes(n_now, g.c, level - 1);
         __syncthreads();
-        if (lo < hi) plane_jobs<T, E * 32 / kSub, MX, C>(g, tp, K, refs, grp, level, lo, hi, n_below, warp, nwarps, lane);
+        if (lo < hi)
+            plane_jobs<T, E * 32 / kSub, MX, C>(g, tp, K, refs, grp, level, lo, hi, n_below, warp, nwarps, lane);
     }
     __syncthreads();
 }
@@ -1137,8 +1134,8 @@ cudaError_t level_launches(const Geo &g, const TreePtrs &tp, const T *K, const T
         const int64_t jobs = (bound * g.R + kPerWarp - 1) / kPerWarp;
         dim3 grid((unsigned)((jobs + kLevelWarps - 1) / kLevelWarps), g.groups());
         ProfScope ps(level_name(level), st);
-        tree_level_kernel<T, E, MX, C><<<grid, kLevelWarps * 32, 0, st>>>(g, tp, K, refs, lens, level, n_new, bound,
-                                                                       status);
+        tree_level_kernel<T, E * 32 / kSub, MX, C><<<grid, kLevelWarps * 32, 0, st>>>(g, tp, K, refs, lens, level,
+                                                                                   n_new, bound, status);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -1170,9 +1167,9 @@ cudaError_t tree_update_t(const Geo &g, const TreePtrs &tp, const T *K, const T 
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        return level_launches<T, E * 32 / kSub, MX, C>(g, tp, K, refs, lens, n_new, fused_levels(g.c, g.L) + 1, status, st);
+        return level_launches<T, E, MX, C>(g, tp, K, refs, lens, n_new, fused_levels(g.c, g.L) + 1, status, st);
     } else {
-        return level_launches<T, E * 32 / kSub, MX, C>(g, tp, K, refs, lens, n_new, 1, status, st);
+        return level_launches<T, E, MX, C>(g, tp, K, refs, lens, n_new, 1, status, st);
     }
 }
 
