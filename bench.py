@@ -55,6 +55,8 @@ def parse():
                     help="skip the 1M incremental-build record and the crossover summary of the default line")
     ap.add_argument("--scorer", default="mma", choices=["tcgen05", "mma"],
                     help="node-scoring kernel: tcgen05 (tensor memory) where it applies, or mma.sync")
+    ap.add_argument("--route", default="levels", choices=["levels", "fused"],
+                    help="routing launches: per level (default), or one fused launch (ZHA_FLAG_FUSED_ROUTE)")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="replay each decode step from a captured CUDA graph (default on)")
     ap.add_argument("--sweep", action="store_true",
@@ -337,8 +339,10 @@ def zha_arm(args, w, world, rank, local):
     n_total = W_steps + 2 * K_steps + (K_steps if not args.no_e2e else 0) + 1   # + the quality step
     cap = w.context + n_total + 8
     inp = make_inputs(w, device="cuda", capacity=cap)
+    flags = (zha.ZHA_FLAG_TCGEN05 if args.scorer == "tcgen05" else 0) | \
+        (zha.ZHA_FLAG_FUSED_ROUTE if args.route == "fused" else 0)
     cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs, w.dtype,
-                     cap, flags=zha.ZHA_FLAG_TCGEN05 if args.scorer == "tcgen05" else 0, summary=w.summary)
+                     cap, flags=flags, summary=w.summary)
     buf = zha.Buffers(cfg)
     K, V, refs, lens = inp.K, inp.V, inp.refs, inp.lens
     k_new, v_new, qs = decode_stream(w, n_total, device="cuda")
@@ -434,6 +438,7 @@ def zha_arm(args, w, world, rank, local):
            "candidates_per_level": [float(h[:, l, :].sum(dim=1).mean()) for l in range(w.levels)],
            "attended_tokens_per_step": float(attn_tokens.mean()),
            "gpu_launches": int(launches), "cuda_graph": graph is not None, "scorer": args.scorer,
+           "route": args.route,
            "clocks": clocks}
 
     # per-kernel CUDA-event timing: a second pass of K steps, every launch bracketed
@@ -850,7 +855,7 @@ def _bytes(w, cand, tokens):
 
 
 def sweep_point(N: int, tree: str, refs_mode: str, steps: int, warmup: int, p_schedule: str = "fixed",
-                summary: str = "native"):
+                summary: str = "native", route: str = "levels"):
     """ZHA decode vs the dense kernel on one identical cache of N tokens (batch
     1, 32/4 heads, d 128): the deep, wide or speed-model tree with random or
     aligned references. Returns one record."""
@@ -867,7 +872,7 @@ def sweep_point(N: int, tree: str, refs_mode: str, steps: int, warmup: int, p_sc
     cap = N + n + W + 8
     inp = make_inputs(w, device="cuda", capacity=cap)
     cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs,
-                     w.dtype, cap, summary=w.summary)
+                     w.dtype, cap, summary=w.summary, flags=zha.ZHA_FLAG_FUSED_ROUTE if route == "fused" else 0)
     buf = zha.Buffers(cfg)
     zha.tree_build(cfg, buf.tree, inp.K, inp.refs, inp.lens, buf.status)
     k_new, v_new, qs = decode_stream(w, n + W, device="cuda")
@@ -877,7 +882,8 @@ def sweep_point(N: int, tree: str, refs_mode: str, steps: int, warmup: int, p_sc
     dense_ms = _timed_dense(zha, cfg, buf, qs[0], inp.K, inp.V, inp.lens, out, flush, n, W)
     us = ms / n * 1e3
     touched = _bytes(w, cand, toks)
-    rec = {"mode": "sweep", "tree": tree, "refs": refs_mode, "context": N, "p": w.p, "summary": w.summary,
+    rec = {"mode": "sweep", "tree": tree, "refs": refs_mode, "route": route, "context": N, "p": w.p,
+           "summary": w.summary,
            "p_schedule": w.p_schedule, "zha_us_per_step": us, "dense_us_per_step": dense_ms * 1e3,
            "speedup_vs_dense": dense_ms * 1e3 / us,
            "keys_attended": toks / (w.batch * w.n_kv_heads * (N + W + n)),
@@ -897,19 +903,21 @@ def sweep_mode(args):
         for refs_mode in ("random", "aligned"):
             for N in Ns:
                 print(json.dumps(sweep_point(N, tree, refs_mode, args.steps, args.warmup, args.p_schedule,
-                                             args.summary)), flush=True)
+                                             args.summary, args.route)), flush=True)
 
 
 def crossover_summary(steps: int = 5, warmup: int = 3):
     """ZHA and dense us/step at 64K, 128K and 512K tokens for the deep and wide
-    trees with both reference modes (a bounded part of the context sweep)."""
+    trees with both reference modes, the aligned (selective) one with both
+    route modes (a bounded part of the context sweep)."""
     rows = []
     for tree in ("deep", "wide"):
-        for refs_mode in ("random", "aligned"):
+        for refs_mode, route in (("random", "levels"), ("aligned", "levels"), ("aligned", "fused")):
             for N in (65536, 131072, 524288):
-                r = sweep_point(N, tree, refs_mode, steps, warmup)
-                rows.append({k: r[k] for k in ("tree", "refs", "context", "zha_us_per_step", "dense_us_per_step",
-                                               "speedup_vs_dense", "keys_attended", "touched_frac_of_hbm")})
+                r = sweep_point(N, tree, refs_mode, steps, warmup, route=route)
+                rows.append({k: r[k] for k in ("tree", "refs", "route", "context", "zha_us_per_step",
+                                               "dense_us_per_step", "speedup_vs_dense", "keys_attended",
+                                               "touched_frac_of_hbm")})
     return {"steps": steps, "warmup": warmup, "batch": 1, "l2": "flushed before every timed step", "points": rows}
 
 

@@ -82,7 +82,15 @@ enum {
      * n_refs 16, G <= 16, batch * n_kv_heads <= 16. The default is the
      * mma.sync kernel, which streams the summaries at a higher fraction of
      * HBM bandwidth on this path */
-    ZHA_FLAG_TCGEN05 = 2
+    ZHA_FLAG_TCGEN05 = 2,
+    /* route in one launch: one thread-block cluster of 8 CTAs per (sequence,
+     * KV head) walks every level (scores, cluster barrier, selection and join
+     * by the first CTA, cluster barrier). Same selections as the default
+     * per-level launches; the launch pays off when few nodes are kept per
+     * level (trained references), the default when most are. Applies to bf16
+     * trees with native summaries, n_refs 16 and at most 8 query heads per KV
+     * head, single queries; otherwise the default route runs. */
+    ZHA_FLAG_FUSED_ROUTE = 4
 };
 
 #define ZHA_MAX_LEVELS 8

@@ -1,0 +1,125 @@
+"""The fused route (ZHA_FLAG_FUSED_ROUTE: one launch, one thread-block cluster
+per (sequence, KV head) walking every level) against the fp64 oracle, and
+against the default per-level launches, whose scores and selections it must
+reproduce bit for bit: few kept nodes (aligned references), many (random
+references: more candidates per level than its shared-memory kept masks
+hold), a ragged batch, head_dim 64, a cache shorter than one chunk, and
+decode steps."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import zha_testlib as T
+from tree_indexed_sparse_02_b200.inputs import WIDE_32K, Workload, decode_stream, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+CASES = [Workload("deep bf16 B=2 c=4 L=4", 2, 16, 2, 128, 3001, 4, 4, 16, 0.95, 16, "bf16", 11),
+         Workload("deep aligned N=65536 L=6", 1, 32, 4, 128, 65536, 4, 6, 16, 0.95, 64, "bf16", 5,
+                  refs_mode="aligned"),
+         Workload("deep random N=65536 L=6", 1, 32, 4, 128, 65536, 4, 6, 16, 0.95, 64, "bf16", 6),
+         Workload("d64 aligned B=2 c=4 L=5", 2, 16, 2, 64, 20000, 4, 5, 16, 0.9, 16, "bf16", 31,
+                  refs_mode="aligned"),
+         dataclasses.replace(WIDE_32K, name="wide aligned N=32768 c=256", refs_mode="aligned")]
+IDS = [w.name for w in CASES]
+
+
+@pytest.fixture(scope="module")
+def zha():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from tree_indexed_sparse_02_b200 import zha as z
+    return z
+
+
+def _lens(w):
+    return None if w.batch == 1 else [w.context] + [w.context - 7 * b - 2 for b in range(1, w.batch)]
+
+
+def _routed(zha, w, inp, flags):
+    cap = w.context + 64
+    cfg = T.make_cfg(zha, w, cap, flags=flags)
+    buf = zha.Buffers(cfg)
+    zha.tree_build(cfg, buf.tree, inp.K, inp.refs, inp.lens, buf.status)
+    zha.route(cfg, buf.tree, inp.q, inp.lens, w.p, buf.sel, buf.workspace, buf.status)
+    out = torch.zeros_like(inp.q)
+    zha.sparse_attn(cfg, inp.q, inp.K, inp.V, inp.lens, buf.sel, out, buf.workspace, buf.status)
+    torch.cuda.synchronize()
+    buf.check_status()
+    return cfg, buf, out
+
+
+@pytest.mark.parametrize("w", CASES, ids=IDS)
+def test_fused_route_matches_oracle_and_default(zha, w):
+    inp = make_inputs(w, capacity=w.context + 64, lens=_lens(w))
+    dev = T.to_device(inp)
+    cfg, fused, out_f = _routed(zha, w, dev, zha.ZHA_FLAG_FUSED_ROUTE)
+    _, ref, out_r = _routed(zha, w, dev, 0)
+    # the oracle, group by group (level by level, selections, outputs)
+    flipped = 0
+    for b in range(w.batch):
+        for kvh in range(w.n_kv_heads):
+            flipped += len(T.check_group_vs_oracle(w, inp, fused, b, kvh, [w.p] * w.levels, out=out_f))
+    assert flipped <= max(2, w.batch * w.n_q_heads // 8), flipped
+    # the default launches: same candidates, scores, kept masks, selection and output
+    for level in range(1, w.levels + 1):
+        a, r = fused.level_state(level), ref.level_state(level)
+        assert torch.equal(a["count"], r["count"]), level
+        for b in range(w.batch):
+            for kvh in range(w.n_kv_heads):
+                n = int(r["count"][b, kvh])
+                for key in ("cand_idx", "cand_mask", "kept_mask"):
+                    assert torch.equal(a[key][b, kvh, :n], r[key][b, kvh, :n]), (level, key)
+                assert torch.equal(a["scores"][b, kvh, :, :n], r["scores"][b, kvh, :, :n]), level
+    assert torch.equal(fused.sel["count"], ref.sel["count"])
+    for b in range(w.batch):
+        for kvh in range(w.n_kv_heads):
+            n = int(ref.sel["count"][b, kvh])
+            assert torch.equal(fused.sel["leaf_idx"][b, kvh, :n], ref.sel["leaf_idx"][b, kvh, :n])
+            assert torch.equal(fused.sel["head_mask"][b, kvh, :n], ref.sel["head_mask"][b, kvh, :n])
+    assert torch.equal(fused.sel["level_kept"], ref.sel["level_kept"])
+    assert torch.equal(out_f, out_r)
+
+
+@pytest.mark.parametrize("N", [1, 3, 5, 17])
+def test_fused_route_short_caches(zha, N):
+    """Caches shorter than a few chunks: an empty or tiny tree still routes."""
+    w = Workload("short", 1, 8, 1, 128, N, 4, 3, 16, 0.9, 0, "bf16", 23)
+    inp = make_inputs(w, capacity=N + 16)
+    dev = T.to_device(inp)
+    cfg, fused, out_f = _routed(zha, w, dev, zha.ZHA_FLAG_FUSED_ROUTE)
+    _, ref, out_r = _routed(zha, w, dev, 0)
+    assert torch.equal(fused.sel["count"], ref.sel["count"])
+    assert torch.equal(out_f, out_r)
+
+
+def test_fused_decode_steps_equal_default(zha):
+    """zha_decode with the fused route: the same outputs and selections as the
+    default launches, step after step (tokens appended, chunks completing)."""
+    w = dataclasses.replace(CASES[1], name="decode aligned")
+    steps = 9
+    cap = w.context + steps + 8
+    inp = T.to_device(make_inputs(w, capacity=cap))
+    k_new, v_new, qs = decode_stream(w, steps, device="cuda")
+    runs = []
+    for flags in (zha.ZHA_FLAG_FUSED_ROUTE, 0):
+        cfg = T.make_cfg(zha, w, cap, flags=flags)
+        buf = zha.Buffers(cfg)
+        K, V, lens = inp.K.clone(), inp.V.clone(), inp.lens.clone()
+        zha.tree_build(cfg, buf.tree, K, inp.refs, lens, buf.status)
+        outs, sels = [], []
+        for i in range(steps):
+            out = torch.zeros_like(qs[i])
+            zha.decode(cfg, buf.tree, K, V, inp.refs, lens, qs[i], k_new[i], v_new[i], w.p, buf.sel, out,
+                       buf.workspace, buf.status)
+            outs.append(out)
+            sels.append(buf.sel["count"].clone())
+        torch.cuda.synchronize()
+        buf.check_status()
+        runs.append((outs, sels))
+    for (of, sf), (orr, sr) in zip(zip(*runs[0]), zip(*runs[1])):
+        assert torch.equal(of, orr)
+        assert torch.equal(sf, sr)
+    assert np.isfinite(runs[0][0][-1].float().cpu().numpy()).all()

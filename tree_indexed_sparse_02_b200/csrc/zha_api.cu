@@ -24,7 +24,7 @@ zha_status check_config(const zha_config *c) {
     if (!pow2(c->chunk) || c->chunk < 2 || c->chunk > 256) return ZHA_ERR_UNSUPPORTED;
     if (c->levels > ZHA_MAX_LEVELS || c->n_refs > 32) return ZHA_ERR_UNSUPPORTED;
     if (c->dtype != ZHA_BF16 && c->dtype != ZHA_F32) return ZHA_ERR_UNSUPPORTED;
-    if (c->flags & ~(ZHA_FLAG_TAIL_ONLY | ZHA_FLAG_TCGEN05)) return ZHA_ERR_UNSUPPORTED;
+    if (c->flags & ~(ZHA_FLAG_TAIL_ONLY | ZHA_FLAG_TCGEN05 | ZHA_FLAG_FUSED_ROUTE)) return ZHA_ERR_UNSUPPORTED;
     // int32 token and leaf indices; fixed-point mass sums need <= 2^23 candidates
     if (c->max_len > (1 << 30) || c->max_len / c->chunk > (1 << 23)) return ZHA_ERR_UNSUPPORTED;
     if (c->attn_splits < 0 || c->attn_splits > 4096) return ZHA_ERR_INVALID_ARG;

@@ -243,6 +243,7 @@ cudaError_t launch_decode_prologue(const Geo &g, void *tree, void *K, void *V, c
                                    int32_t *status, cudaStream_t st);
 Geo make_geo_for(const zha_config *c);
 bool score_tc_supported(const Geo &g);
+bool fused_route_supported(const Geo &g);
 cudaError_t launch_score_tc(const Geo &g, const void *mu_level, const float *bias, const void *q,
                             const int32_t *lens, int level, int32_t *cand, uint32_t *cmask, float *scores,
                             int32_t *count, uint32_t *maxkey, uint32_t *minkey, const int32_t *plist_up,

@@ -74,12 +74,24 @@ inline LevelWs level_ws(const Geo &g, void *ws, int l) {
 __device__ __forceinline__ uint32_t all_heads(int G) { return G >= 32 ? 0xffffffffu : ((1u << G) - 1u); }
 
 // Candidate i of a group at a level: its node and the heads it is a candidate for.
+// Loads of workspace data: through the read-only path where the kernel only
+// reads it; plain (coherent) loads where other CTAs of the same launch write
+// it between cluster barriers.
+template <bool NC, typename T>
+__device__ __forceinline__ T ld_ws(const T *p) {
+    if constexpr (NC)
+        return __ldg(p);
+    else
+        return *p;
+}
+
 struct CandSource {
     int lc;                   // log2(c)
     int top;                  // top level: candidate i is node i, for every head
     int n_here;               // nodes at this level
     const int32_t *plist;     // nodes kept one level up
     const uint32_t *pmask;
+    template <bool NC = true>
     __device__ __forceinline__ void at(int i, int &node, uint32_t &mask, uint32_t all) const {
         if (top) {
             node = i;
@@ -87,8 +99,8 @@ struct CandSource {
             return;
         }
         const int j = i >> lc;
-        node = (__ldg(&plist[j]) << lc) | (i & ((1 << lc) - 1));
-        mask = node < n_here ? __ldg(&pmask[j]) : 0u;
+        node = (ld_ws<NC>(&plist[j]) << lc) | (i & ((1 << lc) - 1));
+        mask = node < n_here ? ld_ws<NC>(&pmask[j]) : 0u;
     }
 };
 
@@ -1349,18 +1361,19 @@ __device__ __forceinline__ int warp_hist_cross(const WarpHist &wh, int lane, uns
 }
 
 // Exact top-p of one query row by one warp: members are candidates i < n with
-// (cmask[i] & bit); their kept bits are OR-ed into sh.kmask. Returns (in every
-// lane) the number kept.
-__device__ int small_row_topp(SmallShared &sh, int w, const float *sc, const uint32_t *cmask, int n, uint32_t bit,
-                              float p, uint32_t kmax, uint32_t kmin) {
+// (cmask[i] & bit); their kept bits are OR-ed into kmask[i] (shared or global
+// memory). Returns (in every lane) the number kept.
+template <bool NC = true>
+__device__ int small_row_topp(SmallShared &sh, uint32_t *kmask, int w, const float *sc, const uint32_t *cmask, int n,
+                              uint32_t bit, float p, uint32_t kmax, uint32_t kmin) {
     const int lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
     if (kmax == 0u) return 0;  // no member
     int kept = 0;
     if (p >= 1.f) {
         for (int i = lane; i < n; i += 32)
-            if (__ldg(cmask + i) & bit) {
-                atomicOr(&sh.kmask[i], bit);
+            if (ld_ws<NC>(cmask + i) & bit) {
+                atomicOr(&kmask[i], bit);
                 ++kept;
             }
         return warp_sum_int(kept);
@@ -1382,8 +1395,8 @@ __device__ int small_row_topp(SmallShared &sh, int w, const float *sc, const uin
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             const int i = i0 + u * 32 + lane;
-            c[u] = i < n ? __ldg(cmask + i) : 0u;
-            e[u] = i < n ? __ldg(sc + i) : 0.f;
+            c[u] = i < n ? ld_ws<NC>(cmask + i) : 0u;
+            e[u] = i < n ? ld_ws<NC>(sc + i) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kU; ++u)
@@ -1406,15 +1419,15 @@ __device__ int small_row_topp(SmallShared &sh, int w, const float *sc, const uin
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             const int i = i0 + u * 32 + lane;
-            c[u] = i < n ? __ldg(cmask + i) : 0u;
-            e[u] = i < n ? __ldg(sc + i) : 0.f;
+            c[u] = i < n ? ld_ws<NC>(cmask + i) : 0u;
+            e[u] = i < n ? ld_ws<NC>(sc + i) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             const int i = i0 + u * 32 + lane;
             const int bk = (c[u] & bit) ? bucket(e[u]) : kSmallBuckets + 1;
             if (bk < bstar) {
-                atomicOr(&sh.kmask[i], bit);
+                atomicOr(&kmask[i], bit);
                 ++kept;
             }
             const unsigned tb = __ballot_sync(0xffffffffu, bk == bstar);
@@ -1448,7 +1461,7 @@ __device__ int small_row_topp(SmallShared &sh, int w, const float *sc, const uin
             const unsigned long long ms = r < ntie ? fixed_mass(key_to_float(sh.lkey[w][j]), m) : 0ull;
             const unsigned long long incl = warp_incl_scan64(ms, lane);
             if (r < ntie && cum + (incl - ms) < target) {
-                atomicOr(&sh.kmask[sh.lidx[w][j]], bit);
+                atomicOr(&kmask[sh.lidx[w][j]], bit);
                 ++kept;
             }
             cum += __shfl_sync(0xffffffffu, incl, 31);
@@ -1466,8 +1479,8 @@ __device__ int small_row_topp(SmallShared &sh, int w, const float *sc, const uin
             for (int j = lane; j < kSmallBuckets; j += 32) lo[j] = hi[j] = 0u;
             __syncwarp();
             for (int i = lane; i < n; i += 32) {
-                if (!(__ldg(cmask + i) & bit)) continue;
-                const float e = __ldg(sc + i);
+                if (!(ld_ws<NC>(cmask + i) & bit)) continue;
+                const float e = ld_ws<NC>(sc + i);
                 if (bucket(e) != bstar) continue;
                 const uint32_t u = kmax - ordered_key(e);
                 if (hb < 32 && (u >> hb) != (prefix >> hb)) continue;
@@ -1488,19 +1501,19 @@ __device__ int small_row_topp(SmallShared &sh, int w, const float *sc, const uin
         unsigned long long cum = ab;
         for (int i0 = 0; i0 < n; i0 += 32) {
             const int i = i0 + lane;
-            const bool mem = i < n && (__ldg(cmask + i) & bit);
-            const float e = mem ? __ldg(sc + i) : 0.f;
+            const bool mem = i < n && (ld_ws<NC>(cmask + i) & bit);
+            const float e = mem ? ld_ws<NC>(sc + i) : 0.f;
             const bool inb = mem && bucket(e) == bstar;
             const uint32_t u = inb ? kmax - ordered_key(e) : 0u;
             if (inb && u < tau) {
-                atomicOr(&sh.kmask[i], bit);
+                atomicOr(&kmask[i], bit);
                 ++kept;
             }
             const bool tie = inb && u == tau;
             const unsigned long long ms = (tie && cum < target) ? (unsigned long long)fixed_mass(e, m) : 0ull;
             const unsigned long long incl = warp_incl_scan64(ms, lane);
             if (tie && cum + (incl - ms) < target) {
-                atomicOr(&sh.kmask[i], bit);
+                atomicOr(&kmask[i], bit);
                 ++kept;
             }
             cum += __shfl_sync(0xffffffffu, incl, 31);
@@ -1523,7 +1536,8 @@ select_small_kernel(Geo g, LevelWs lw, int level, float p, int32_t *level_kept, 
     for (int h = w; h < g.G; h += kSmallWarps) {
         const uint32_t kmax = lw.maxkey[(int64_t)grp * g.G + h];
         const uint32_t kmin = lw.minkey[(int64_t)grp * g.G + h];
-        const int nk = small_row_topp(sh, w, lw.scores + (grp * g.G + h) * capv, cmask, n, 1u << h, p, kmax, kmin);
+        const int nk = small_row_topp(sh, sh.kmask, w, lw.scores + (grp * g.G + h) * capv, cmask, n, 1u << h, p,
+                                      kmax, kmin);
         if (level_kept && lane == 0) level_kept[((int64_t)grp * g.G + h) * g.L + (level - 1)] = nk;
     }
     __syncthreads();
@@ -1555,6 +1569,189 @@ select_small_kernel(Geo g, LevelWs lw, int level, float p, int32_t *level_kept, 
             lw.pcount[grp] = (int32_t)total;
         else
             sel.count[grp] = (int32_t)total;
+    }
+    pdl_trigger();
+}
+
+// ------------------------------------------------------ fused route: one launch
+//
+// The whole route in one launch, for trees where few nodes are kept per level
+// (trained references): one thread-block cluster of kFusedCTAs CTAs per
+// (sequence, KV head) group walks the levels top-down. Per level, the
+// cluster's CTAs score the group's candidates (each warp a candidate at a
+// time, on the mma.sync scheme of score_mma_kernel, so the scores are the
+// same bits), a cluster barrier, the first CTA selects every query row (a
+// warp per row, the exact selection of select_small_kernel) and joins the
+// rows into the next level's candidates, a cluster barrier. Candidate lists,
+// scores and kept masks use the same workspace views as the per-level
+// launches (kept masks in shared memory up to kFusedMax candidates, in the
+// workspace beyond). Any number of candidates is handled; the launch pays
+// off when the numbers are small. Cluster barriers are hardware barriers:
+// every CTA takes the same number of them, so nothing waits unboundedly.
+
+constexpr int kFusedCTAs = 8;
+constexpr int kFusedMax = 4096;
+
+struct FusedArgs {
+    LevelWs lw[kMaxLevels + 1];
+    float p[kMaxLevels + 1];
+    const __nv_bfloat16 *mu[kMaxLevels + 1];
+    const float *bias[kMaxLevels + 1];
+};
+
+__device__ __forceinline__ void cluster_barrier() {
+    __threadfence();   // global writes before the barrier are seen by the whole cluster after it
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSmallThreads)
+route_fused_kernel(Geo g, FusedArgs a, const __nv_bfloat16 *q, const int32_t *lens, zha_selection sel) {
+    __shared__ SmallShared sh;
+    __shared__ uint32_t kms[kFusedMax];
+    constexpr int KP = D / 32;
+    const int grp = blockIdx.y;
+    const int b = grp / g.Hkv, kvh = grp % g.Hkv;
+    const int rank = (int)cluster_ctarank();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gq = lane >> 2, t = lane & 3;
+    // the group's query rows (G <= 8: one n-tile), as B fragments
+    uint32_t bq[KP][4];
+#pragma unroll
+    for (int kp = 0; kp < KP; ++kp) {
+        uint4 w = make_uint4(0, 0, 0, 0);
+        if (gq < g.G) w = ldg16(q + g.qrow(b, kvh, gq) * D + kp * 32 + t * 8);
+        bq[kp][0] = w.x; bq[kp][1] = w.y; bq[kp][2] = w.z; bq[kp][3] = w.w;
+    }
+    pdl_wait();
+    const int64_t N = group_len(g, lens, grp);
+    const uint32_t all = all_heads(g.G);
+    const float s = g.s;
+    for (int level = g.L; level >= 1; --level) {
+        const LevelWs &lw = a.lw[level];
+        const LevelWs &up = a.lw[level < g.L ? level + 1 : level];
+        const CandSource src = cand_source(g, up, level, grp, N);
+        const int n = (int)cand_count(g, up, level, grp, src.n_here);
+        const int64_t cap = g.cap[level], capv = g.capv[level];
+        if (rank == 0 && tid == 0) lw.count[grp] = n;
+        // 1. scores of every candidate for every query row
+        float runmax[2] = {-INFINITY, -INFINITY}, runmin[2] = {INFINITY, INFINITY};
+        for (int i = rank * kSmallWarps + warp; i < n; i += kFusedCTAs * kSmallWarps) {
+            int node;
+            uint32_t hm;
+            src.at<false>(i, node, hm, all);
+            if (lane == 0) {
+                lw.cand[grp * capv + i] = node;
+                lw.cmask[grp * capv + i] = hm;
+            }
+            if (hm == 0u) {
+                if (lane < g.G) lw.scores[(grp * g.G + lane) * capv + i] = -INFINITY;
+                continue;
+            }
+            const __nv_bfloat16 *base = a.mu[level] + (grp * cap + node) * (int64_t)g.R * D;
+            uint4 ra[KP], rb[KP];
+#pragma unroll
+            for (int kp = 0; kp < KP; ++kp) {
+                ra[kp] = ldg16(base + (int64_t)gq * D + kp * 32 + t * 8);
+                rb[kp] = ldg16(base + (int64_t)(gq + 8) * D + kp * 32 + t * 8);
+            }
+            const float *bb = a.bias[level] + (grp * cap + node) * (int64_t)g.R;
+            const float b0 = bb[gq], b1 = bb[gq + 8];
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kp = 0; kp < KP; ++kp) {
+                const uint4 &xa = ra[kp], &xb = rb[kp];
+                const uint32_t a0[4] = {xa.x, xb.x, xa.y, xb.y};
+                const uint32_t a1[4] = {xa.z, xb.z, xa.w, xb.w};
+                mma_bf16_16816(acc, a0, bq[kp][0], bq[kp][1]);
+                mma_bf16_16816(acc, a1, bq[kp][2], bq[kp][3]);
+            }
+            float e[2];
+            e[0] = fmaxf(-INFINITY, fmaxf(fmaf(s, acc[0], b0), fmaf(s, acc[2], b1)));
+            e[1] = fmaxf(-INFINITY, fmaxf(fmaf(s, acc[1], b0), fmaf(s, acc[3], b1)));
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                float v = e[j];
+                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                e[j] = v;
+            }
+            if (gq == 0) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int h = 2 * t + j;
+                    if (h < g.G) {
+                        lw.scores[(grp * g.G + h) * capv + i] = e[j];
+                        if ((hm >> h) & 1u) {
+                            runmax[j] = fmaxf(runmax[j], e[j]);
+                            runmin[j] = fminf(runmin[j], e[j]);
+                        }
+                    }
+                }
+            }
+        }
+        if (gq == 0) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int h = 2 * t + j;
+                if (h < g.G && runmax[j] > -INFINITY) {
+                    atomicMax(&lw.maxkey[(int64_t)grp * g.G + h], ordered_key(runmax[j]));
+                    atomicMin(&lw.minkey[(int64_t)grp * g.G + h], ordered_key(runmin[j]));
+                }
+            }
+        }
+        cluster_barrier();
+        // 2. the first CTA: every row's selection, then the join
+        if (rank == 0) {
+            uint32_t *km = n <= kFusedMax ? kms : lw.kept + grp * capv;
+            for (int i = tid; i < n; i += kSmallThreads) km[i] = 0u;
+            __syncthreads();
+            const uint32_t *cmask = lw.cmask + grp * capv;
+            for (int h = warp; h < g.G; h += kSmallWarps) {
+                const uint32_t kmax = lw.maxkey[(int64_t)grp * g.G + h];
+                const uint32_t kmin = lw.minkey[(int64_t)grp * g.G + h];
+                const int nk = small_row_topp<false>(sh, km, warp, lw.scores + (grp * g.G + h) * capv, cmask, n,
+                                                     1u << h, a.p[level], kmax, kmin);
+                if (sel.level_kept && lane == 0) sel.level_kept[((int64_t)grp * g.G + h) * g.L + (level - 1)] = nk;
+            }
+            __syncthreads();
+            const int per = (n + kSmallThreads - 1) / kSmallThreads;
+            const int i0 = tid * per;
+            int cnt = 0;
+            for (int k = 0; k < per; ++k) {
+                const int i = i0 + k;
+                cnt += (i < n && km[i] != 0u);
+            }
+            unsigned long long total;
+            int64_t o = (int64_t)block_exclusive_scan<unsigned long long>((unsigned long long)cnt, sh.red, &total);
+            int32_t *out_idx = level > 1 ? lw.plist + grp * cap : sel.leaf_idx + grp * g.cap[1];
+            uint32_t *out_mask = level > 1 ? lw.pmask + grp * cap : sel.head_mask + grp * g.cap[1];
+            for (int k = 0; k < per; ++k) {
+                const int i = i0 + k;
+                if (i >= n) break;
+                const uint32_t m = km[i];
+                if (km == kms) lw.kept[grp * capv + i] = m;
+                if (m) {
+                    out_idx[o] = lw.cand[grp * capv + i];
+                    out_mask[o] = m;
+                    ++o;
+                }
+            }
+            if (tid == 0) {
+                if (level > 1)
+                    lw.pcount[grp] = (int32_t)total;
+                else
+                    sel.count[grp] = (int32_t)total;
+            }
+        }
+        cluster_barrier();
     }
     pdl_trigger();
 }
@@ -2029,6 +2226,13 @@ int64_t split_slots() {
 
 }  // namespace
 
+// The fused route covers bf16 trees with native summaries, 16 reference
+// planes per node and at most 8 query rows per group (single queries).
+bool fused_route_supported(const Geo &g) {
+    return g.dtype == ZHA_BF16 && !g.mx() && g.R == 16 && g.G <= 8 && g.T == 1 && g.lag == 0 &&
+           (g.d == 64 || g.d == 128);
+}
+
 #define ZHA_TRY(call)                         \
     do {                                      \
         const cudaError_t le_ = (call);       \
@@ -2056,6 +2260,36 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
         if (e != cudaSuccess) return e;
     }
     const char *tb = static_cast<const char *>(tree);
+    if ((g.flags & ZHA_FLAG_FUSED_ROUTE) && fused_route_supported(g)) {
+        FusedArgs a{};
+        for (int l = 1; l <= g.L; ++l) {
+            a.lw[l] = level_ws(g, ws, l);
+            a.p[l] = p_levels[l - 1];
+            a.mu[l] = reinterpret_cast<const __nv_bfloat16 *>(tb + g.mu_off[l]);
+            a.bias[l] = reinterpret_cast<const float *>(tb + g.bias_off[l]);
+        }
+        cudaLaunchConfig_t c{};
+        c.gridDim = dim3(kFusedCTAs, groups);
+        c.blockDim = dim3(kSmallThreads);
+        c.dynamicSmemBytes = 0;
+        c.stream = st;
+        cudaLaunchAttribute at[2];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = kFusedCTAs;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[1].val.programmaticStreamSerializationAllowed = 1;
+        c.attrs = at;
+        c.numAttrs = 2;
+        ProfScope ps("route_fused", st);
+        const auto *qq = static_cast<const __nv_bfloat16 *>(q);
+        if (g.d == 128)
+            e = cudaLaunchKernelEx(&c, route_fused_kernel<128>, g, a, qq, lens, sel);
+        else
+            e = cudaLaunchKernelEx(&c, route_fused_kernel<64>, g, a, qq, lens, sel);
+        return e;
+    }
     for (int level = g.L; level >= 1; --level) {
         LevelWs lw = level_ws(g, ws, level);
         LevelWs up = level < g.L ? level_ws(g, ws, level + 1) : lw;

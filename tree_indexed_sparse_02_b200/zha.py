@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libzha.so")
 ZHA_BF16, ZHA_F32 = 0, 1
 ZHA_FLAG_TAIL_ONLY = 1
 ZHA_FLAG_TCGEN05 = 2
+ZHA_FLAG_FUSED_ROUTE = 4
 ZHA_P_FIXED, ZHA_P_DEPTH_ROOT = 0, 1
 ZHA_SUMMARY_NATIVE, ZHA_SUMMARY_MXFP8 = 0, 1
 ZHA_MAX_LEVELS = 8
