@@ -2,9 +2,9 @@
 per (sequence, KV head) walking every level) against the fp64 oracle, and
 against the default per-level launches, whose scores and selections it must
 reproduce bit for bit: few kept nodes (aligned references), many (random
-references: more candidates per level than its shared-memory kept masks
-hold), a ragged batch, head_dim 64, a cache shorter than one chunk, and
-decode steps."""
+references: more candidates per level than the cluster's shared memory
+holds), a ragged batch, head_dim 64, many groups (8-CTA clusters), fewer
+query rows than CTAs, a cache shorter than one chunk, and decode steps."""
 import dataclasses
 
 import numpy as np
@@ -22,7 +22,12 @@ CASES = [Workload("deep bf16 B=2 c=4 L=4", 2, 16, 2, 128, 3001, 4, 4, 16, 0.95, 
          Workload("deep random N=65536 L=6", 1, 32, 4, 128, 65536, 4, 6, 16, 0.95, 64, "bf16", 6),
          Workload("d64 aligned B=2 c=4 L=5", 2, 16, 2, 64, 20000, 4, 5, 16, 0.9, 16, "bf16", 31,
                   refs_mode="aligned"),
-         dataclasses.replace(WIDE_32K, name="wide aligned N=32768 c=256", refs_mode="aligned")]
+         dataclasses.replace(WIDE_32K, name="wide aligned N=32768 c=256", refs_mode="aligned"),
+         # many groups (clusters of 8 CTAs: the 16-CTA clusters of 20 groups do not all fit at once)
+         Workload("20 groups B=5 aligned c=4 L=5", 5, 32, 4, 128, 6000, 4, 5, 16, 0.9, 16, "bf16", 41,
+                  refs_mode="aligned"),
+         # four query rows per group (CTAs that own no row)
+         Workload("G=4 d64 B=2 c=4 L=4", 2, 16, 4, 64, 9000, 4, 4, 16, 0.9, 16, "bf16", 43)]
 IDS = [w.name for w in CASES]
 
 

@@ -268,9 +268,13 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
             for (int nt = 0; nt < NT; ++nt) e[nt][0] = e[nt][1] = -INFINITY;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                float acc[NT][4];
+                // two accumulation chains (first and second k16 half of each
+                // 32-wide k step), added at the end: half the dependent depth
+                float acc[NT][4], acc2[NT][4];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) acc[nt][v] = acc2[nt][v] = 0.f;
 #pragma unroll
                 for (int kp = 0; kp < KP; ++kp) {
                     const uint4 &xa = ra[u][mt][kp], &xb = rb[u][mt][kp];
@@ -281,13 +285,17 @@ score_mma_kernel(Geo g, const __nv_bfloat16 *mu, const float *bias, const __nv_b
                         if constexpr (QS) {
                             const uint4 f = qsm[(nt * KP + kp) * 32 + lane];
                             mma_bf16_16816(acc[nt], a0, f.x, f.y);
-                            mma_bf16_16816(acc[nt], a1, f.z, f.w);
+                            mma_bf16_16816(acc2[nt], a1, f.z, f.w);
                         } else {
                             mma_bf16_16816(acc[nt], a0, bq[nt][kp][0], bq[nt][kp][1]);
-                            mma_bf16_16816(acc[nt], a1, bq[nt][kp][2], bq[nt][kp][3]);
+                            mma_bf16_16816(acc2[nt], a1, bq[nt][kp][2], bq[nt][kp][3]);
                         }
                     }
                 }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) acc[nt][v] += acc2[nt][v];
                 const int r0 = mt * 16 + gq, r1 = r0 + 8;
                 const float b0 = r0 < g.R ? bb[r0] : -INFINITY;
                 const float b1 = r1 < g.R ? bb[r1] : -INFINITY;
@@ -1364,8 +1372,9 @@ __device__ __forceinline__ int warp_hist_cross(const WarpHist &wh, int lane, uns
 // (cmask[i] & bit); their kept bits are OR-ed into kmask[i] (shared or global
 // memory). Returns (in every lane) the number kept.
 template <bool NC = true>
-__device__ int small_row_topp(SmallShared &sh, uint32_t *kmask, int w, const float *sc, const uint32_t *cmask, int n,
-                              uint32_t bit, float p, uint32_t kmax, uint32_t kmin) {
+__device__ __forceinline__ int small_row_topp(SmallShared &sh, uint32_t *kmask, int w, const float *sc,
+                                              const uint32_t *cmask, int n, uint32_t bit, float p, uint32_t kmax,
+                                              uint32_t kmin) {
     const int lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
     if (kmax == 0u) return 0;  // no member
@@ -1576,21 +1585,28 @@ select_small_kernel(Geo g, LevelWs lw, int level, float p, int32_t *level_kept, 
 // ------------------------------------------------------ fused route: one launch
 //
 // The whole route in one launch, for trees where few nodes are kept per level
-// (trained references): one thread-block cluster of kFusedCTAs CTAs per
-// (sequence, KV head) group walks the levels top-down. Per level, the
-// cluster's CTAs score the group's candidates (each warp a candidate at a
-// time, on the mma.sync scheme of score_mma_kernel, so the scores are the
-// same bits), a cluster barrier, the first CTA selects every query row (a
-// warp per row, the exact selection of select_small_kernel) and joins the
-// rows into the next level's candidates, a cluster barrier. Candidate lists,
-// scores and kept masks use the same workspace views as the per-level
-// launches (kept masks in shared memory up to kFusedMax candidates, in the
-// workspace beyond). Any number of candidates is handled; the launch pays
-// off when the numbers are small. Cluster barriers are hardware barriers:
-// every CTA takes the same number of them, so nothing waits unboundedly.
+// (trained references): one thread-block cluster per
+// (sequence, KV head) group walks the levels top-down, CTA r owning query
+// row r (16 CTAs per cluster where all the groups' clusters fit on the GPU at
+// once, else 8). Per level: (1) the cluster's CTAs score the group's candidates (each
+// warp two candidates at a time, on the mma.sync scheme of score_mma_kernel,
+// so the scores are the same bits) and deliver row h's scores and extremes to
+// CTA h through distributed shared memory; a cluster barrier; (2) CTA r
+// selects row r with all its threads (the exact selection of the per-level
+// kernels) and ORs its kept bits into every CTA's kept masks; a cluster
+// barrier; (3) every CTA joins the rows into the next level's candidates by
+// itself, so the next level starts without another barrier. The level's
+// candidates and scores are copied out to the workspace views that the
+// per-level launches fill by the CTAs that own no row while the rows select
+// (16-CTA clusters), else after the join. A level with more than kFusedSm candidates goes through the
+// workspace instead (correct at any size, but one warp per row then selects
+// over all of them: the per-level launches are the faster route there).
+// Cluster barriers are hardware barriers that every CTA takes the same
+// number of times, so nothing waits unboundedly.
 
-constexpr int kFusedCTAs = 8;
-constexpr int kFusedMax = 4096;
+constexpr int kFusedSm = 1024;     // candidates per level that a level keeps in shared memory
+constexpr int kFusedPer = kFusedSm / kSmallThreads;
+static_assert(kSmallThreads == kSmallBuckets, "one histogram bucket per thread");
 
 struct FusedArgs {
     LevelWs lw[kMaxLevels + 1];
@@ -1599,9 +1615,31 @@ struct FusedArgs {
     const float *bias[kMaxLevels + 1];
 };
 
-__device__ __forceinline__ void cluster_barrier() {
-    __threadfence();   // global writes before the barrier are seen by the whole cluster after it
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+// Per-CTA shared state. CTA r < G of a cluster owns query row r of its group:
+// the other CTAs deliver that row's scores and extremes to it through
+// distributed shared memory, and each row's CTA ORs its kept bits into every
+// CTA's km, so that each CTA joins the level by itself.
+struct FusedShared {
+    float sc[2][kFusedSm];          // this CTA's row: scores of the level's candidates (by level parity)
+    uint32_t km[kFusedSm];          // kept head masks of the level's candidates
+    uint32_t rk[kFusedSm];          // this CTA's row: candidate kept (1) or not (0)
+    uint32_t mb[kFusedSm];          // this CTA's row: candidate is a member (for the warp selection)
+    int32_t pl[2][kFusedSm];        // nodes kept one level up and their head masks, when they fit
+    uint32_t pm[2][kFusedSm];       // (by level parity: a join writes one half while the other is read)
+    uint32_t hlo[kSmallBuckets];    // the row's mass histogram (64-bit buckets from native 32-bit
+    uint32_t hhi[kSmallBuckets];    // shared atomics: low words and carry words)
+    unsigned long long above, target;
+    int32_t tidx[kSmallList];       // crossing-bucket members: index, ordered key, rank order
+    uint32_t tkey[kSmallList];
+    int32_t tord[kSmallList];
+    int32_t wsum[kSmallWarps];      // per-warp kept counts of the join
+    uint32_t maxk, mink;            // ordered keys of this row's largest and smallest member score
+    int32_t bstar, ntie, nkept;
+    SmallShared sh;                 // the warp selection: rows with many equal-bucket members
+};
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;\n" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -1610,11 +1648,211 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
     return r;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kSmallThreads)
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+template <typename T>
+__device__ __forceinline__ uint32_t cluster_addr(T *p, uint32_t rank) {
+    uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p)), r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+
+// reductions into another CTA's shared memory that return nothing (no round trip)
+__device__ __forceinline__ void red_max_cluster(uint32_t addr, uint32_t v) {
+    asm volatile("red.relaxed.cluster.shared::cluster.max.u32 [%0], %1;\n" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_min_cluster(uint32_t addr, uint32_t v) {
+    asm volatile("red.relaxed.cluster.shared::cluster.min.u32 [%0], %1;\n" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_or_cluster(uint32_t addr, uint32_t v) {
+    asm volatile("red.relaxed.cluster.shared::cluster.or.b32 [%0], %1;\n" ::"r"(addr), "r"(v) : "memory");
+}
+
+// generic address of the same shared variable in CTA `rank` of the cluster
+template <typename T>
+__device__ __forceinline__ T *cluster_peer(T *p, uint32_t rank) {
+    uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p)), r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(a), "r"(rank));
+    uint64_t gen;
+    asm volatile("cvta.shared::cluster.u64 %0, %1;\n" : "=l"(gen) : "l"((uint64_t)r));
+    return reinterpret_cast<T *>(gen);
+}
+
+// Exact top-p of this CTA's row over the level's n <= kFusedSm candidates, in
+// shared memory, by the whole CTA: the same definition as small_row_topp (and
+// topp_core) -- members by (score desc, index asc), each kept while the mass
+// before it is below ceil(p * total), masses in 2^-31 fixed point relative to
+// the row's maximum -- found with one mass histogram over the same buckets
+// (scanned by one warp), and the crossing bucket's members ranked by one
+// warp. A crossing bucket with more than kSmallList members goes to
+// small_row_topp. Sets fs.rk[i] for the kept candidates and returns (in every
+// thread) how many were kept. The histogram is all zero on entry and on return.
+template <class Member>
+__device__ int cta_row_topp(FusedShared &fs, const float *sc, int n, float p, Member member) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t kmax = fs.maxk, kmin = fs.mink;
+    if (kmax == 0u) {   // no member
+#pragma unroll
+        for (int k = 0; k < kFusedPer; ++k)
+            if (tid + k * kSmallThreads < n) fs.rk[tid + k * kSmallThreads] = 0u;
+        __syncthreads();
+        return 0;
+    }
+    float e[kFusedPer];
+    bool mem[kFusedPer];
+#pragma unroll
+    for (int k = 0; k < kFusedPer; ++k) {
+        const int i = tid + k * kSmallThreads;
+        mem[k] = i < n && member(i);
+        e[k] = mem[k] ? sc[i] : 0.f;
+        if (i < n) fs.rk[i] = 0u;
+    }
+    int kept = 0;
+    if (p >= 1.f) {
+#pragma unroll
+        for (int k = 0; k < kFusedPer; ++k)
+            if (mem[k]) {
+                fs.rk[tid + k * kSmallThreads] = 1u;
+                ++kept;
+            }
+        return (int)block_sum<unsigned long long>((unsigned long long)kept, fs.sh.red);
+    }
+    const float m = key_to_float(kmax);
+    float W = (float)kSmallBuckets / fminf(m - key_to_float(kmin), kMassRange);
+    if (kmax == kmin || !(W < 1e30f)) W = 0.f;  // one score value (or a sub-denormal span): one bucket
+    auto bucket = [&](float x) -> int {
+        const float y = (m - x) * W;
+        return y < (float)(kSmallBuckets - 1) ? (int)y : kSmallBuckets - 1;
+    };
+#pragma unroll
+    for (int k = 0; k < kFusedPer; ++k)
+        if (mem[k]) {
+            const uint32_t w = fixed_mass(e[k], m);
+            if (w) hist_add(fs.hlo, fs.hhi, bucket(e[k]), w);
+        }
+    __syncthreads();
+    if (warp == 0) {
+        // lane l scans buckets [8 l, 8 l + 8) (and zeroes them for the next use)
+        constexpr int kPer = kSmallBuckets / 32;
+        unsigned long long hb[kPer], mine = 0ull;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int bk = lane * kPer + j;
+            hb[j] = ((unsigned long long)fs.hhi[bk] << 32) | fs.hlo[bk];
+            fs.hlo[bk] = fs.hhi[bk] = 0u;
+            mine += hb[j];
+        }
+        const unsigned long long incl = warp_incl_scan64(mine, lane);
+        const unsigned long long total = __shfl_sync(0xffffffffu, incl, 31);
+        const unsigned long long target = (unsigned long long)ceil((double)p * (double)total);
+        unsigned long long run = incl - mine, ab = 0ull;
+        int found = -1;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            if (found < 0 && hb[j] && run < target && run + hb[j] >= target) {
+                found = lane * kPer + j;
+                ab = run;
+            }
+            run += hb[j];
+        }
+        const unsigned ball = __ballot_sync(0xffffffffu, found >= 0);
+        if (lane == 0) {
+            fs.bstar = kSmallBuckets;   // unreachable (target <= total): keep every member
+            fs.ntie = 0;
+            fs.nkept = 0;
+            fs.target = target;
+        }
+        if (ball && lane == __ffs(ball) - 1) {
+            fs.bstar = found;
+            fs.above = ab;
+        }
+    }
+    __syncthreads();
+    const int bstar = fs.bstar;
+#pragma unroll
+    for (int k = 0; k < kFusedPer; ++k) {
+        if (!mem[k]) continue;
+        const int i = tid + k * kSmallThreads;
+        const int b = bucket(e[k]);
+        if (b < bstar) {
+            fs.rk[i] = 1u;
+            ++kept;
+        } else if (b == bstar) {
+            const int slot = atomicAdd(&fs.ntie, 1);
+            if (slot < kSmallList) {
+                fs.tidx[slot] = i;
+                fs.tkey[slot] = ordered_key(e[k]);
+            }
+        }
+    }
+    __syncthreads();
+    const int ntie = fs.ntie;
+    if (ntie == 1) {
+        // a lone member of the crossing bucket: the mass before it (that of
+        // the buckets before) is below the target, so it is kept
+        if (tid == 0) {
+            fs.rk[fs.tidx[0]] = 1u;
+            ++kept;
+        }
+    } else if (ntie <= kSmallList) {
+        if (warp == 0) {
+            const unsigned long long target = fs.target;
+            // rank the crossing bucket's members by (key desc, index asc)
+            for (int j = lane; j < ntie; j += 32) {
+                const uint32_t kj = fs.tkey[j];
+                const int ij = fs.tidx[j];
+                int r = 0;
+                for (int v = 0; v < ntie; ++v) {
+                    const uint32_t kv = fs.tkey[v];
+                    r += (kv > kj) || (kv == kj && fs.tidx[v] < ij);
+                }
+                fs.tord[r] = j;
+            }
+            __syncwarp();
+            unsigned long long cum = fs.above;
+            for (int r0 = 0; r0 < ntie && cum < target; r0 += 32) {
+                const int r = r0 + lane;
+                const int j = r < ntie ? fs.tord[r] : 0;
+                const unsigned long long ms = r < ntie ? fixed_mass(key_to_float(fs.tkey[j]), m) : 0ull;
+                const unsigned long long incl = warp_incl_scan64(ms, lane);
+                if (r < ntie && cum + (incl - ms) < target) {
+                    fs.rk[fs.tidx[j]] = 1u;
+                    ++kept;
+                }
+                cum += __shfl_sync(0xffffffffu, incl, 31);
+            }
+        }
+    }
+    if (ntie <= kSmallList) {
+        const int wk = __reduce_add_sync(0xffffffffu, kept);
+        if (lane == 0 && wk) atomicAdd(&fs.nkept, wk);
+        __syncthreads();
+        return fs.nkept;
+    }
+    // many members in the crossing bucket: warp 0 runs the warp selection over
+    // the whole row (it marks a superset of the candidates marked above:
+    // exactly the kept ones)
+#pragma unroll
+    for (int k = 0; k < kFusedPer; ++k) {
+        const int i = tid + k * kSmallThreads;
+        if (i < n) fs.mb[i] = mem[k] ? 1u : 0u;
+    }
+    __syncthreads();
+    if (warp == 0) small_row_topp<false>(fs.sh, fs.rk, 0, sc, fs.mb, n, 1u, p, kmax, kmin);
+    __syncthreads();
+    kept = 0;
+#pragma unroll
+    for (int k = 0; k < kFusedPer; ++k) {
+        const int i = tid + k * kSmallThreads;
+        kept += (i < n && fs.rk[i] != 0u);
+    }
+    return (int)block_sum<unsigned long long>((unsigned long long)kept, fs.sh.red);
+}
+
+template <int D, int CL>
+__global__ void __launch_bounds__(kSmallThreads, 2)
 route_fused_kernel(Geo g, FusedArgs a, const __nv_bfloat16 *q, const int32_t *lens, zha_selection sel) {
-    __shared__ SmallShared sh;
-    __shared__ uint32_t kms[kFusedMax];
+    extern __shared__ __align__(16) unsigned char fused_raw[];
+    FusedShared &fs = *reinterpret_cast<FusedShared *>(fused_raw);
     constexpr int KP = D / 32;
     const int grp = blockIdx.y;
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
@@ -1629,69 +1867,169 @@ route_fused_kernel(Geo g, FusedArgs a, const __nv_bfloat16 *q, const int32_t *le
         if (gq < g.G) w = ldg16(q + g.qrow(b, kvh, gq) * D + kp * 32 + t * 8);
         bq[kp][0] = w.x; bq[kp][1] = w.y; bq[kp][2] = w.z; bq[kp][3] = w.w;
     }
+    for (int i = tid; i < kFusedSm; i += kSmallThreads) fs.km[i] = 0u;
+    fs.hlo[tid] = fs.hhi[tid] = 0u;
+    if (tid == 0) {
+        fs.maxk = 0u;
+        fs.mink = 0xffffffffu;
+    }
     pdl_wait();
     const int64_t N = group_len(g, lens, grp);
     const uint32_t all = all_heads(g.G);
     const float s = g.s;
+    const int lc = __ffs(g.c) - 1;
+    // nodes of each level (c is a power of two: shifts, not divisions)
+    auto nodes_at = [&](int level) -> int {
+        int64_t m = N >> lc;
+        for (int l = 2; l <= level; ++l) m = (m + g.c - 1) >> lc;
+        return (int)m;
+    };
+    // scores and extremes of row h go to CTA h (lanes with gq == 0 hold rows 2t, 2t + 1)
+    float *sc_row[2][2];
+    uint32_t mx_row[2], mn_row[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const uint32_t h = (uint32_t)min(2 * t + j, CL - 1);
+        sc_row[0][j] = cluster_peer(&fs.sc[0][0], h);
+        sc_row[1][j] = cluster_peer(&fs.sc[1][0], h);
+        mx_row[j] = cluster_addr(&fs.maxk, h);
+        mn_row[j] = cluster_addr(&fs.mink, h);
+    }
+    cluster_sync();   // every CTA has started (its shared memory exists) and reset its state
+    bool pl_local = false;  // the nodes kept one level up are in fs.pl[par] (else in the workspace)
+    int par = 0, n_up = 0;
+    int n_here = nodes_at(g.L);
     for (int level = g.L; level >= 1; --level) {
         const LevelWs &lw = a.lw[level];
         const LevelWs &up = a.lw[level < g.L ? level + 1 : level];
-        const CandSource src = cand_source(g, up, level, grp, N);
-        const int n = (int)cand_count(g, up, level, grp, src.n_here);
+        const bool top = level == g.L;
+        const int n = top ? n_here : n_up * g.c;
+        const int n_below = level > 1 ? nodes_at(level - 1) : 0;
+        const bool sm = n <= kFusedSm;
         const int64_t cap = g.cap[level], capv = g.capv[level];
-        if (rank == 0 && tid == 0) lw.count[grp] = n;
-        // 1. scores of every candidate for every query row
-        float runmax[2] = {-INFINITY, -INFINITY}, runmin[2] = {INFINITY, INFINITY};
-        for (int i = rank * kSmallWarps + warp; i < n; i += kFusedCTAs * kSmallWarps) {
-            int node;
-            uint32_t hm;
-            src.at<false>(i, node, hm, all);
-            if (lane == 0) {
-                lw.cand[grp * capv + i] = node;
-                lw.cmask[grp * capv + i] = hm;
+        const int64_t cap_up = top ? 0 : g.cap[level + 1];
+        // candidate i: its node and the heads that route to it
+        auto cand_at = [&](int i, int &node, uint32_t &hm) {
+            if (top) {
+                node = i;
+                hm = all;
+                return;
             }
-            if (hm == 0u) {
-                if (lane < g.G) lw.scores[(grp * g.G + lane) * capv + i] = -INFINITY;
-                continue;
-            }
-            const __nv_bfloat16 *base = a.mu[level] + (grp * cap + node) * (int64_t)g.R * D;
-            uint4 ra[KP], rb[KP];
-#pragma unroll
-            for (int kp = 0; kp < KP; ++kp) {
-                ra[kp] = ldg16(base + (int64_t)gq * D + kp * 32 + t * 8);
-                rb[kp] = ldg16(base + (int64_t)(gq + 8) * D + kp * 32 + t * 8);
-            }
-            const float *bb = a.bias[level] + (grp * cap + node) * (int64_t)g.R;
-            const float b0 = bb[gq], b1 = bb[gq + 8];
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kp = 0; kp < KP; ++kp) {
-                const uint4 &xa = ra[kp], &xb = rb[kp];
-                const uint32_t a0[4] = {xa.x, xb.x, xa.y, xb.y};
-                const uint32_t a1[4] = {xa.z, xb.z, xa.w, xb.w};
-                mma_bf16_16816(acc, a0, bq[kp][0], bq[kp][1]);
-                mma_bf16_16816(acc, a1, bq[kp][2], bq[kp][3]);
-            }
-            float e[2];
-            e[0] = fmaxf(-INFINITY, fmaxf(fmaf(s, acc[0], b0), fmaf(s, acc[2], b1)));
-            e[1] = fmaxf(-INFINITY, fmaxf(fmaf(s, acc[1], b0), fmaf(s, acc[3], b1)));
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                float v = e[j];
-                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-                e[j] = v;
-            }
-            if (gq == 0) {
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int h = 2 * t + j;
+            const int j = i >> lc;
+            const int pn = pl_local ? fs.pl[par][j] : up.plist[grp * cap_up + j];
+            node = (pn << lc) | (i & (g.c - 1));
+            hm = node < n_here ? (pl_local ? fs.pm[par][j] : up.pmask[grp * cap_up + j]) : 0u;
+        };
+        // the level's candidates and scores, out to the workspace views (a
+        // level held in shared memory). With CTAs that own no row, those copy
+        // while the rows select (before the level's last cluster barrier: the
+        // rows' scores are read from their CTAs' shared memory). Otherwise
+        // every CTA copies after the join, its own row's scores and a share of
+        // the candidates: no CTA reads another's shared memory after the last
+        // barrier, when that CTA may have finished.
+        auto copy_out = [&]() {
+            if (CL > g.G) {
+                const int nc = CL - g.G, rc = rank - g.G;
+                for (int x = rc * kSmallThreads + tid; x < n * (g.G + 1); x += nc * kSmallThreads) {
+                    const int h = x / n, i = x - h * n;
                     if (h < g.G) {
-                        lw.scores[(grp * g.G + h) * capv + i] = e[j];
-                        if ((hm >> h) & 1u) {
-                            runmax[j] = fmaxf(runmax[j], e[j]);
-                            runmin[j] = fminf(runmin[j], e[j]);
+                        lw.scores[(grp * g.G + h) * capv + i] = cluster_peer(&fs.sc[par][0], (uint32_t)h)[i];
+                    } else {
+                        int node;
+                        uint32_t hm;
+                        cand_at(i, node, hm);
+                        lw.cand[grp * capv + i] = node;
+                        lw.cmask[grp * capv + i] = hm;
+                    }
+                }
+            } else {
+                for (int i = tid; i < n; i += kSmallThreads) lw.scores[(grp * g.G + rank) * capv + i] = fs.sc[par][i];
+                for (int i = rank * kSmallThreads + tid; i < n; i += CL * kSmallThreads) {
+                    int node;
+                    uint32_t hm;
+                    cand_at(i, node, hm);
+                    lw.cand[grp * capv + i] = node;
+                    lw.cmask[grp * capv + i] = hm;
+                }
+            }
+        };
+        if (!sm && rank == 0)
+            for (int i = tid; i < n; i += kSmallThreads) lw.kept[grp * capv + i] = 0u;
+        // 1. scores of every candidate for every query row, each warp two
+        //    candidates at a time: to the row's CTA, or (a level with more
+        //    candidates than fit) to the workspace
+        constexpr int U = 2;
+        float runmax[2] = {-INFINITY, -INFINITY}, runmin[2] = {INFINITY, INFINITY};
+        for (int i0 = (rank * kSmallWarps + warp) * U; i0 < n; i0 += CL * kSmallWarps * U) {
+            int node[U];
+            uint32_t hm[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                node[u] = 0;
+                hm[u] = 0u;
+                if (i0 + u < n) {
+                    cand_at(i0 + u, node[u], hm[u]);
+                    if (!sm && lane == 0) {
+                        lw.cand[grp * capv + i0 + u] = node[u];
+                        lw.cmask[grp * capv + i0 + u] = hm[u];
+                    }
+                }
+            }
+            uint4 ra[U][KP], rb[U][KP];
+            float b0[U], b1[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const __nv_bfloat16 *base = a.mu[level] + (grp * cap + node[u]) * (int64_t)g.R * D;
+                const float *bb = a.bias[level] + (grp * cap + node[u]) * (int64_t)g.R;
+#pragma unroll
+                for (int kp = 0; kp < KP; ++kp) {
+                    ra[u][kp] = hm[u] ? ldg16(base + (int64_t)gq * D + kp * 32 + t * 8) : make_uint4(0, 0, 0, 0);
+                    rb[u][kp] = hm[u] ? ldg16(base + (int64_t)(gq + 8) * D + kp * 32 + t * 8) : make_uint4(0, 0, 0, 0);
+                }
+                b0[u] = hm[u] ? bb[gq] : 0.f;
+                b1[u] = hm[u] ? bb[gq + 8] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + u;
+                if (i >= n) break;
+                float e[2] = {-INFINITY, -INFINITY};
+                if (hm[u]) {
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int kp = 0; kp < KP; ++kp) {
+                        const uint4 &xa = ra[u][kp], &xb = rb[u][kp];
+                        const uint32_t a0[4] = {xa.x, xb.x, xa.y, xb.y};
+                        const uint32_t a1[4] = {xa.z, xb.z, xa.w, xb.w};
+                        mma_bf16_16816(acc, a0, bq[kp][0], bq[kp][1]);
+                        mma_bf16_16816(acc2, a1, bq[kp][2], bq[kp][3]);
+                    }
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) acc[v] += acc2[v];
+                    e[0] = fmaxf(-INFINITY, fmaxf(fmaf(s, acc[0], b0[u]), fmaf(s, acc[2], b1[u])));
+                    e[1] = fmaxf(-INFINITY, fmaxf(fmaf(s, acc[1], b0[u]), fmaf(s, acc[3], b1[u])));
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        float v = e[j];
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                        e[j] = v;
+                    }
+                }
+                if (gq == 0) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int h = 2 * t + j;
+                        if (h < g.G) {
+                            if (sm)
+                                (par ? sc_row[1][j] : sc_row[0][j])[i] = e[j];
+                            else
+                                lw.scores[(grp * g.G + h) * capv + i] = e[j];
+                            if ((hm[u] >> h) & 1u) {
+                                runmax[j] = fmaxf(runmax[j], e[j]);
+                                runmin[j] = fminf(runmin[j], e[j]);
+                            }
                         }
                     }
                 }
@@ -1702,56 +2040,119 @@ route_fused_kernel(Geo g, FusedArgs a, const __nv_bfloat16 *q, const int32_t *le
             for (int j = 0; j < 2; ++j) {
                 const int h = 2 * t + j;
                 if (h < g.G && runmax[j] > -INFINITY) {
-                    atomicMax(&lw.maxkey[(int64_t)grp * g.G + h], ordered_key(runmax[j]));
-                    atomicMin(&lw.minkey[(int64_t)grp * g.G + h], ordered_key(runmin[j]));
+                    red_max_cluster(mx_row[j], ordered_key(runmax[j]));
+                    red_min_cluster(mn_row[j], ordered_key(runmin[j]));
                 }
             }
         }
-        cluster_barrier();
-        // 2. the first CTA: every row's selection, then the join
-        if (rank == 0) {
-            uint32_t *km = n <= kFusedMax ? kms : lw.kept + grp * capv;
-            for (int i = tid; i < n; i += kSmallThreads) km[i] = 0u;
-            __syncthreads();
-            const uint32_t *cmask = lw.cmask + grp * capv;
-            for (int h = warp; h < g.G; h += kSmallWarps) {
-                const uint32_t kmax = lw.maxkey[(int64_t)grp * g.G + h];
-                const uint32_t kmin = lw.minkey[(int64_t)grp * g.G + h];
-                const int nk = small_row_topp<false>(sh, km, warp, lw.scores + (grp * g.G + h) * capv, cmask, n,
-                                                     1u << h, a.p[level], kmax, kmin);
-                if (sel.level_kept && lane == 0) sel.level_kept[((int64_t)grp * g.G + h) * g.L + (level - 1)] = nk;
+        if (!sm) __threadfence();   // workspace scores and kept masks reach the other CTAs through L2
+        cluster_sync();
+        // 2. CTA r selects row r, and ORs its kept bits into every CTA's km
+        //    (CTAs without a row copy the level out meanwhile)
+        if (sm && CL > g.G && rank >= g.G) copy_out();
+        if (rank < g.G) {
+            const uint32_t bit = 1u << rank;
+            int nk;
+            if (sm) {
+                nk = cta_row_topp(fs, fs.sc[par], n, a.p[level], [&](int i) {
+                    int node;
+                    uint32_t hm;
+                    cand_at(i, node, hm);
+                    return (hm & bit) != 0u;
+                });
+                for (int i = tid; i < n; i += kSmallThreads)
+                    if (fs.rk[i])
+#pragma unroll
+                        for (int r = 0; r < CL; ++r) red_or_cluster(cluster_addr(&fs.km[i], (uint32_t)r), bit);
+            } else {
+                nk = 0;
+                if (warp == 0)
+                    nk = small_row_topp<false>(fs.sh, lw.kept + grp * capv, 0, lw.scores + (grp * g.G + rank) * capv,
+                                               lw.cmask + grp * capv, n, bit, a.p[level], fs.maxk, fs.mink);
+                __syncthreads();
             }
-            __syncthreads();
-            const int per = (n + kSmallThreads - 1) / kSmallThreads;
-            const int i0 = tid * per;
-            int cnt = 0;
-            for (int k = 0; k < per; ++k) {
-                const int i = i0 + k;
-                cnt += (i < n && km[i] != 0u);
-            }
-            unsigned long long total;
-            int64_t o = (int64_t)block_exclusive_scan<unsigned long long>((unsigned long long)cnt, sh.red, &total);
-            int32_t *out_idx = level > 1 ? lw.plist + grp * cap : sel.leaf_idx + grp * g.cap[1];
-            uint32_t *out_mask = level > 1 ? lw.pmask + grp * cap : sel.head_mask + grp * g.cap[1];
-            for (int k = 0; k < per; ++k) {
-                const int i = i0 + k;
-                if (i >= n) break;
-                const uint32_t m = km[i];
-                if (km == kms) lw.kept[grp * capv + i] = m;
-                if (m) {
-                    out_idx[o] = lw.cand[grp * capv + i];
-                    out_mask[o] = m;
-                    ++o;
-                }
-            }
+            if (sel.level_kept && tid == 0) sel.level_kept[((int64_t)grp * g.G + rank) * g.L + (level - 1)] = nk;
             if (tid == 0) {
-                if (level > 1)
-                    lw.pcount[grp] = (int32_t)total;
-                else
-                    sel.count[grp] = (int32_t)total;
+                fs.maxk = 0u;
+                fs.mink = 0xffffffffu;
             }
         }
-        cluster_barrier();
+        if (!sm) __threadfence();
+        cluster_sync();
+        // 3. every CTA joins the rows into the next level's candidates (the
+        //    first CTA also writes them to the workspace and the selection):
+        //    thread-contiguous runs, compacted in order
+        const int per = (n + kSmallThreads - 1) / kSmallThreads;
+        const int i0 = tid * per;
+        const uint32_t *kmv = sm ? fs.km : lw.kept + grp * capv;
+        int cnt = 0;
+        for (int k = 0; k < per; ++k) {
+            const int i = i0 + k;
+            cnt += (i < n && kmv[i] != 0u);
+        }
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) fs.wsum[warp] = incl;
+        __syncthreads();
+        int o = incl - cnt, total = 0;
+#pragma unroll
+        for (int w = 0; w < kSmallWarps; ++w) {
+            const int v = fs.wsum[w];
+            o += w < warp ? v : 0;
+            total += v;
+        }
+        const bool fits = total <= kFusedSm;
+        int32_t *out_idx = level > 1 ? lw.plist + grp * cap : sel.leaf_idx + grp * g.cap[1];
+        uint32_t *out_mask = level > 1 ? lw.pmask + grp * cap : sel.head_mask + grp * g.cap[1];
+        for (int k = 0; k < per; ++k) {
+            const int i = i0 + k;
+            if (i >= n) break;
+            const uint32_t m = kmv[i];
+            if (sm && rank == 0) lw.kept[grp * capv + i] = m;
+            if (m) {
+                int node;
+                if (sm) {
+                    uint32_t hm;
+                    cand_at(i, node, hm);
+                } else {
+                    node = lw.cand[grp * capv + i];
+                }
+                if (fits) {
+                    fs.pl[par ^ 1][o] = node;
+                    fs.pm[par ^ 1][o] = m;
+                }
+                if (rank == 0) {
+                    out_idx[o] = node;
+                    out_mask[o] = m;
+                }
+                ++o;
+            }
+        }
+        if (rank == 0 && tid == 0) {
+            lw.count[grp] = n;
+            if (level > 1)
+                lw.pcount[grp] = total;
+            else
+                sel.count[grp] = total;
+        }
+        __syncthreads();
+        if (sm) {
+            for (int i = tid; i < n; i += kSmallThreads) fs.km[i] = 0u;
+            if (CL == g.G) copy_out();
+        }
+        if (!fits) {
+            // the next level reads the kept nodes from the workspace
+            __threadfence();
+            cluster_sync();
+        }
+        pl_local = fits;
+        n_up = total;
+        n_here = n_below;
+        par ^= 1;
     }
     pdl_trigger();
 }
@@ -2268,14 +2669,44 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
             a.mu[l] = reinterpret_cast<const __nv_bfloat16 *>(tb + g.mu_off[l]);
             a.bias[l] = reinterpret_cast<const float *>(tb + g.bias_off[l]);
         }
+        // clusters of 16 where every group's cluster is resident at once, else 8
+        static const int max16 = [] {
+            const int bytes = (int)sizeof(FusedShared);
+            for (auto k : {route_fused_kernel<128, 8>, route_fused_kernel<64, 8>, route_fused_kernel<128, 16>,
+                           route_fused_kernel<64, 16>})
+                if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+                    return -1;
+            for (auto k : {route_fused_kernel<128, 16>, route_fused_kernel<64, 16>})
+                if (cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+                    return 0;
+            cudaLaunchConfig_t c{};
+            c.gridDim = dim3(16, 1);
+            c.blockDim = dim3(kSmallThreads);
+            c.dynamicSmemBytes = bytes;
+            cudaLaunchAttribute at;
+            at.id = cudaLaunchAttributeClusterDimension;
+            at.val.clusterDim.x = 16;
+            at.val.clusterDim.y = 1;
+            at.val.clusterDim.z = 1;
+            c.attrs = &at;
+            c.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, route_fused_kernel<128, 16>, &c) != cudaSuccess) {
+                (void)cudaGetLastError();
+                return 0;
+            }
+            return n;
+        }();
+        if (max16 < 0) return cudaErrorInvalidConfiguration;
+        const int cl = max16 >= groups ? 16 : 8;
         cudaLaunchConfig_t c{};
-        c.gridDim = dim3(kFusedCTAs, groups);
+        c.gridDim = dim3(cl, groups);
         c.blockDim = dim3(kSmallThreads);
-        c.dynamicSmemBytes = 0;
+        c.dynamicSmemBytes = sizeof(FusedShared);
         c.stream = st;
         cudaLaunchAttribute at[2];
         at[0].id = cudaLaunchAttributeClusterDimension;
-        at[0].val.clusterDim.x = kFusedCTAs;
+        at[0].val.clusterDim.x = cl;
         at[0].val.clusterDim.y = 1;
         at[0].val.clusterDim.z = 1;
         at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -2285,9 +2716,11 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
         ProfScope ps("route_fused", st);
         const auto *qq = static_cast<const __nv_bfloat16 *>(q);
         if (g.d == 128)
-            e = cudaLaunchKernelEx(&c, route_fused_kernel<128>, g, a, qq, lens, sel);
+            e = cl == 16 ? cudaLaunchKernelEx(&c, route_fused_kernel<128, 16>, g, a, qq, lens, sel)
+                         : cudaLaunchKernelEx(&c, route_fused_kernel<128, 8>, g, a, qq, lens, sel);
         else
-            e = cudaLaunchKernelEx(&c, route_fused_kernel<64>, g, a, qq, lens, sel);
+            e = cl == 16 ? cudaLaunchKernelEx(&c, route_fused_kernel<64, 16>, g, a, qq, lens, sel)
+                         : cudaLaunchKernelEx(&c, route_fused_kernel<64, 8>, g, a, qq, lens, sel);
         return e;
     }
     for (int level = g.L; level >= 1; --level) {
