@@ -368,6 +368,29 @@ enum { ZHA_P_FIXED = 0, ZHA_P_DEPTH_ROOT = 1 };
  */
 ZHA_API zha_status zha_p_schedule(float p, int32_t levels, int32_t schedule, float *p_levels);
 
+/* waits of zha_wait_expiry_check */
+enum { ZHA_WAIT_ROW_BARRIER = 0, ZHA_WAIT_MBARRIER = 1 };
+
+/*
+ * zha_wait_expiry_check -- failure detection (no counterpart on the pages).
+ * Every wait inside the library's kernels is bounded: the counter barrier of
+ * the selection spread over several CTAs per query row, and the mbarrier
+ * waits of the tensor-core kernels, give up after about a second, set
+ * ZHA_ERR_TIMEOUT in the call's device status and return (the call's results
+ * are then invalid; the context stays usable). This entry runs one of those
+ * waits on a condition that nothing satisfies, with a caller-given limit, so
+ * that the expiry path can be exercised without a fault:
+ *   ZHA_WAIT_ROW_BARRIER  the counter barrier, entered by one of two CTAs
+ *                         (the other returns without arriving);
+ *   ZHA_WAIT_MBARRIER     an mbarrier wait on a barrier that no copy or
+ *                         commit completes.
+ * limit_cycles: SM clock cycles before the wait gives up, 1 .. 2^31.
+ * dev_status: device int32, required; ZHA_ERR_TIMEOUT is written there when
+ * the wait runs out. Asynchronous on `stream`. ZHA_ERR_INVALID_ARG for an
+ * unknown kind, a limit outside the range or a null dev_status.
+ */
+ZHA_API zha_status zha_wait_expiry_check(int32_t kind, int64_t limit_cycles, int32_t *dev_status, void *stream);
+
 /*
  * Instrumentation (no counterpart on the pages; for measurement only).
  * zha_launch_count: kernels this library has launched since it was loaded.

@@ -93,6 +93,11 @@ def test_invalid_arguments_are_rejected_before_launch(zha):
     assert L.zha_dense_decode(ctypes.byref(cfg), ctypes.c_void_p(18), ctypes.c_void_p(16), ctypes.c_void_p(16),
                               ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), None, None) == 1
     assert L.zha_status_string(3).decode().startswith("capacity")
+    # the bounded-wait expiry check: unknown kind, limit out of range, no status
+    assert L.zha_wait_expiry_check(7, 1000, ctypes.c_void_p(16), None) == 1
+    assert L.zha_wait_expiry_check(zha.ZHA_WAIT_MBARRIER, 0, ctypes.c_void_p(16), None) == 1
+    assert L.zha_wait_expiry_check(zha.ZHA_WAIT_MBARRIER, (1 << 31) + 1, ctypes.c_void_p(16), None) == 1
+    assert L.zha_wait_expiry_check(zha.ZHA_WAIT_ROW_BARRIER, 1000, None, None) == 1
 
 
 def test_p_schedule_host_rule(zha, orc):

@@ -361,6 +361,12 @@ zha_status zha_topp_select(const float *scores, const int32_t *counts, int32_t n
                                                static_cast<cudaStream_t>(stream)));
 }
 
+zha_status zha_wait_expiry_check(int32_t kind, int64_t limit_cycles, int32_t *dev_status, void *stream) {
+    if (kind != ZHA_WAIT_ROW_BARRIER && kind != ZHA_WAIT_MBARRIER) return ZHA_ERR_INVALID_ARG;
+    if (limit_cycles < 1 || limit_cycles > (int64_t(1) << 31) || !dev_status) return ZHA_ERR_INVALID_ARG;
+    return cuda_status(zha::launch_wait_expiry(kind, limit_cycles, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
 zha_status zha_p_schedule(float p, int32_t levels, int32_t schedule, float *p_levels) {
     if (!p_levels || !(p > 0.f) || levels < 1 || levels > ZHA_MAX_LEVELS) return ZHA_ERR_INVALID_ARG;
     if (schedule != ZHA_P_FIXED && schedule != ZHA_P_DEPTH_ROOT) return ZHA_ERR_INVALID_ARG;

@@ -252,4 +252,5 @@ cudaError_t launch_score_tc(const Geo &g, const void *mu_level, const float *bia
 cudaError_t launch_topp_select(const float *scores, const int32_t *counts, int n_sets,
                                int64_t stride, float p, uint8_t *kept, int32_t *status,
                                cudaStream_t st);
+cudaError_t launch_wait_expiry(int kind, long long limit, int32_t *status, cudaStream_t st);
 }  // namespace zha

@@ -32,6 +32,7 @@
 //             by a launch of its own.
 #include "zha_common.cuh"
 #include "zha_route_state.cuh"
+#include "zha_tc.cuh"
 
 namespace zha {
 
@@ -2175,7 +2176,8 @@ struct SplitWs {
 // Arrive at a counter shared by the CTAs of one row and wait, bounded, until
 // it reaches target. On timeout the status is set and false returned (the
 // results of the call are then invalid; nothing waits forever).
-__device__ bool row_barrier(uint32_t *ctr, uint32_t target, int32_t *status, int *ok_sh) {
+__device__ bool row_barrier(uint32_t *ctr, uint32_t target, int32_t *status, int *ok_sh,
+                            long long limit = kSpinCycles) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -2183,7 +2185,7 @@ __device__ bool row_barrier(uint32_t *ctr, uint32_t target, int32_t *status, int
         const long long t0 = clock64();
         int ok = 1;
         while (*reinterpret_cast<volatile uint32_t *>(ctr) < target) {
-            if (clock64() - t0 > kSpinCycles) {
+            if (clock64() - t0 > limit) {
                 set_status(status, ZHA_ERR_TIMEOUT);
                 ok = 0;
                 break;
@@ -2870,6 +2872,39 @@ cudaError_t launch_route(const Geo &g, const void *tree, const void *q, const in
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+
+// ------------------------------------------------------- bounded-wait expiry
+//
+// The library's bounded device waits, run on conditions that nothing
+// satisfies, with a caller-given limit: the counter barrier of the multi-CTA
+// selection entered by one of two CTAs (the other returns without arriving,
+// as a lost arrival would), and an mbarrier wait on a barrier that no copy or
+// commit completes. Each must give up after its limit, set ZHA_ERR_TIMEOUT and
+// return, leaving the context usable.
+
+__device__ uint32_t g_expiry_ctr;
+
+__global__ void wait_expiry_kernel(int kind, long long limit, int32_t *status) {
+    __shared__ int ok_sh;
+    __shared__ __align__(8) uint64_t bar;
+    if (kind == ZHA_WAIT_ROW_BARRIER) {
+        if (blockIdx.x == 1) return;   // the CTA that never arrives
+        if (threadIdx.x == 0) g_expiry_ctr = 0u;
+        row_barrier(&g_expiry_ctr, 2u, status, &ok_sh, limit);
+    } else {
+        if (blockIdx.x != 0) return;
+        if (threadIdx.x == 0) mbar_init(smem_u32(&bar), 1u);
+        __syncthreads();
+        if (threadIdx.x == 0) mbar_wait_bounded(smem_u32(&bar), 0u, limit, nullptr, status);
+        __syncthreads();
+    }
+}
+
+cudaError_t launch_wait_expiry(int kind, long long limit, int32_t *status, cudaStream_t st) {
+    ProfScope ps("wait_expiry", st);
+    wait_expiry_kernel<<<2, 64, 0, st>>>(kind, limit, status);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_topp_select(const float *scores, const int32_t *counts, int n_sets,

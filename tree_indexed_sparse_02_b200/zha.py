@@ -20,6 +20,7 @@ ZHA_FLAG_TAIL_ONLY = 1
 ZHA_FLAG_TCGEN05 = 2
 ZHA_FLAG_FUSED_ROUTE = 4
 ZHA_P_FIXED, ZHA_P_DEPTH_ROOT = 0, 1
+ZHA_WAIT_ROW_BARRIER, ZHA_WAIT_MBARRIER = 0, 1
 ZHA_SUMMARY_NATIVE, ZHA_SUMMARY_MXFP8 = 0, 1
 ZHA_MAX_LEVELS = 8
 STATUS_NAMES = {0: "ZHA_OK", 1: "ZHA_ERR_INVALID_ARG", 2: "ZHA_ERR_UNSUPPORTED",
@@ -85,6 +86,7 @@ def _load():
         "zha_dense_decode": ([CP, P, P, P, P, P, P, P, P], i32),
         "zha_topp_select": ([P, P, i32, i64, f32, P, P, P], i32),
         "zha_p_schedule": ([f32, i32, i32, ctypes.POINTER(f32)], i32),
+        "zha_wait_expiry_check": ([i32, i64, P, P], i32),
         "zha_launch_count": ([], ctypes.c_uint64),
         "zha_profile_enable": ([i32], i32),
         "zha_profile_read": ([ctypes.c_char_p, i32, ctypes.POINTER(ctypes.c_double),
@@ -223,6 +225,14 @@ def topp_select(scores, counts, p, kept, dev_status=None, stream=None):
     n_sets, stride = scores.shape
     check(_lib.zha_topp_select(_p(scores), _p(counts), int(n_sets), int(stride), float(p), _p(kept),
                                _p(dev_status), _stream(stream)), "zha_topp_select")
+
+
+def wait_expiry_check(kind: int, limit_cycles: int, dev_status, stream=None):
+    """Run one of the library's bounded device waits on a condition nothing
+    satisfies (ZHA_WAIT_ROW_BARRIER or ZHA_WAIT_MBARRIER), giving up after
+    limit_cycles SM cycles with ZHA_ERR_TIMEOUT in dev_status."""
+    check(_lib.zha_wait_expiry_check(int(kind), int(limit_cycles), _p(dev_status), _stream(stream)),
+          "zha_wait_expiry_check")
 
 
 def launch_count() -> int:
