@@ -321,15 +321,21 @@ ZHA_API zha_status zha_dense_decode(const zha_config *cfg, const void *q, const 
  * latency-critical loop that must not pay for cudaMalloc, which can
  * synchronise the device. This entry point takes the same inputs and output
  * as zha_dense_decode and no workspace: its split-K scratch is a fixed 4 MiB
- * array compiled into the library, which every device that loads the library
- * keeps reserved until the process exits. Configurations whose split-K
+ * array compiled into the library. It takes device memory when the library's
+ * module is loaded on a device -- under CUDA's default lazy loading, at the
+ * first call into the library on that device, which may be this entry's
+ * first call -- and keeps it until the process exits or the context is
+ * reset. A caller that hands the rest of device memory to its own arena makes
+ * one call (any entry point) first. Configurations whose split-K
  * partials (batch * n_kv_heads * splits * G * (head_dim + 2) floats, each
  * part rounded up to 256 bytes) exceed 4 MiB return ZHA_ERR_CAPACITY.
  * All calls share the array, so calls whose kernels overlap on the GPU (for
  * example on two streams at once) race and must be serialised by the caller.
- * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture. It allocates nothing, in the library or in any library it calls.
+ * Every call made outside a stream capture looks up the array's device
+ * address (with that device current; after a context reset the array may
+ * have moved); a call being captured uses the address of the last call
+ * outside capture, so make one call before the first capture and again after
+ * a reset. It allocates nothing, in the library or in any library it calls.
  */
 ZHA_API zha_status zha_dense_decode_noalloc(const zha_config *cfg, const void *q, const void *K,
                                             const void *V, const int32_t *lens, void *out,

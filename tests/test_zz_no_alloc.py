@@ -2,12 +2,16 @@
 device memory (a host framework that owns every allocation, or a loop that
 must not pay for cudaMalloc). It keeps its split-K scratch in a fixed array
 inside the library. Checked through the C ABI against zha_dense_decode, on
-two calls in a row (the second call reuses the scratch the first one left)."""
+two calls in a row (the second call reuses the scratch the first one left),
+and against the oracle's exact attention after a larger call, with shorter
+caches and other split counts (splits with no tokens)."""
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+import zha_oracle as orc
 import zha_testlib as T
 from tree_indexed_sparse_02_b200.inputs import TINY_F32, Workload, make_inputs
 
@@ -62,3 +66,41 @@ def test_noalloc_rejects_configs_beyond_its_scratch(zha):
     lens = torch.zeros(4, dtype=torch.int32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     assert _noalloc(zha, cfg, z, z, z, lens, z, status) == 3   # ZHA_ERR_CAPACITY, nothing launched
+
+
+def test_noalloc_after_a_larger_call_matches_the_oracle(zha):
+    """A call over long caches fills many partials; the next calls, over
+    shorter ragged caches and with other split counts, leave some splits
+    without tokens (they write an empty partial). Every output is checked
+    against the oracle's exact softmax attention."""
+    w = Workload("noalloc ragged B=3", 3, 16, 2, 128, 6000, 4, 3, 16, 0.9, 8, "bf16", 37)
+    cap = w.context + 16
+    inp = make_inputs(w, capacity=cap)
+    dev = T.to_device(inp)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    big = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs, w.dtype, cap,
+                     attn_splits=32)
+    out = torch.zeros_like(dev.q)
+    assert _noalloc(zha, big, dev.q, dev.K, dev.V, dev.lens, out, status) == 0
+    s = T.scale_of(w)
+    G = w.group
+    for splits, lens in ((32, [700, 1, 0]), (7, [5999, 33, 2]), (64, [64, 3, 4096])):
+        cfg = zha.config(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.levels, w.n_refs, w.dtype,
+                         cap, attn_splits=splits)
+        dlens = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        out = torch.full_like(dev.q, float("nan"))
+        assert _noalloc(zha, cfg, dev.q, dev.K, dev.V, dlens, out, status) == 0
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        for b in range(w.batch):
+            N = lens[b]
+            for kvh in range(w.n_kv_heads):
+                got = T.np64(out[b, kvh * G:(kvh + 1) * G])
+                if N == 0:
+                    assert np.all(got == 0.0), (splits, b)   # no token: a zero output
+                    continue
+                K = T.np64(inp.K[b, kvh, :N])
+                V = T.np64(inp.V[b, kvh, :N])
+                q = T.np64(inp.q[b, kvh * G:(kvh + 1) * G])
+                ref = np.stack([orc.attend(q[h], K, V, N, s) for h in range(G)])
+                assert T.rel_err(got, ref) <= T.TOL[w.dtype], (splits, b, kvh)

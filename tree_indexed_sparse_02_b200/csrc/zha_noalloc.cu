@@ -7,10 +7,11 @@
 
 namespace {
 
-// 4 MiB of split-K scratch, reserved on every device that loads the library
-// until the process exits. Calls share it and it keeps the last call's
-// partials; every partial a call reads it first writes, so nothing needs
-// clearing between calls.
+// 4 MiB of split-K scratch, placed in a device's memory when the library's
+// module is loaded there (on first use under CUDA's lazy loading) and kept
+// until the process exits or the context is reset. Calls share it and it
+// keeps the last call's partials; every partial a call reads it first
+// writes, so nothing needs clearing between calls.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -22,14 +23,25 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // The device address of the scratch array on the current device. The name of
 // a __device__ variable is only a host-side handle, so the address is asked
-// for once per device (with that device current) and cached.
-zha_status scratch_address(void **out) {
+// for with the device current. It is asked for again on every call made
+// outside a stream capture (a reset context reloads the module, and the array
+// may move); a call being captured, where a lookup that loads the module is
+// not allowed, uses the address of the last call outside capture.
+zha_status scratch_address(cudaStream_t stream, void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZHA_ERR_CUDA;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+        (void)cudaGetLastError();
+        cs = cudaStreamCaptureStatusActive;   // unknown: do not look up
+    }
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    if (cs == cudaStreamCaptureStatusNone || !g_scratch_addr[dev]) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ZHA_ERR_CUDA;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            (void)cudaGetLastError();
+            return ZHA_ERR_CUDA;
+        }
         g_scratch_addr[dev] = p;
     }
     *out = g_scratch_addr[dev];
@@ -57,7 +69,7 @@ extern "C" zha_status zha_dense_decode_noalloc(const zha_config *cfg, const void
     g.ws_part_ml = 0;
     g.ws_part_o = ml_bytes;
     void *scratch = nullptr;
-    zha_status s = scratch_address(&scratch);
+    zha_status s = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
     if (s != ZHA_OK) return s;
     cudaError_t e = zha::launch_attention(g, q, K, V, lens, nullptr, out, scratch, dev_status,
                                           static_cast<cudaStream_t>(stream));
