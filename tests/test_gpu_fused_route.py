@@ -4,7 +4,8 @@ against the default per-level launches, whose scores and selections it must
 reproduce bit for bit: few kept nodes (aligned references), many (random
 references: more candidates per level than the cluster's shared memory
 holds), a ragged batch, head_dim 64, many groups (8-CTA clusters), fewer
-query rows than CTAs, a cache shorter than one chunk, and decode steps."""
+query rows than CTAs, a cache shorter than one chunk, and decode steps
+(against the default path and against the oracle repeating each step)."""
 import dataclasses
 
 import numpy as np
@@ -128,3 +129,59 @@ def test_fused_decode_steps_equal_default(zha):
         assert torch.equal(of, orr)
         assert torch.equal(sf, sr)
     assert np.isfinite(runs[0][0][-1].float().cpu().numpy()).all()
+
+
+DECODE_CASES = [CASES[0], CASES[4], CASES[5], CASES[6],
+                Workload("short N=3 c=4 L=3", 1, 8, 1, 128, 3, 4, 3, 16, 0.9, 0, "bf16", 29)]
+
+
+@pytest.mark.parametrize("w", DECODE_CASES, ids=[w.name for w in DECODE_CASES])
+def test_fused_decode_steps_match_oracle(zha, w):
+    """zha_decode with the fused route against the oracle repeating each step
+    (append, route, exact attention): ragged batch, the wide tree, 8-CTA
+    clusters, four query rows per group, and a cache that starts shorter than
+    one chunk (sink, kept leaves and current chunk overlapping)."""
+    import zha_oracle as orc
+    steps = 6
+    cap = w.context + steps + 8
+    inp = make_inputs(w, capacity=cap, lens=_lens(w))
+    dev = T.to_device(inp)
+    cfg = T.make_cfg(zha, w, cap, flags=zha.ZHA_FLAG_FUSED_ROUTE)
+    buf = zha.Buffers(cfg)
+    zha.tree_build(cfg, buf.tree, dev.K, dev.refs, dev.lens, buf.status)
+    G = w.group
+    s = T.scale_of(w)
+    g = torch.Generator().manual_seed(7)
+    dt = w.torch_dtype()
+    K_host, V_host = inp.K.clone(), inp.V.clone()
+    lens0 = [int(x) for x in inp.lens]
+    trees = {(b, kvh): T.oracle_tree(w, inp, b, kvh, lens0[b], s, cap)
+             for b in range(w.batch) for kvh in range(w.n_kv_heads)}
+    flipped_total = 0
+    for step in range(steps):
+        k_new = torch.randn((w.batch, w.n_kv_heads, w.head_dim), generator=g).to(dt)
+        v_new = torch.randn((w.batch, w.n_kv_heads, w.head_dim), generator=g).to(dt)
+        q = torch.randn((w.batch, w.n_q_heads, w.head_dim), generator=g).to(dt)
+        out = torch.zeros_like(dev.q)
+        zha.decode(cfg, buf.tree, dev.K, dev.V, dev.refs, dev.lens, q.cuda(), k_new.cuda(), v_new.cuda(),
+                   w.p, buf.sel, out, buf.workspace, buf.status)
+        torch.cuda.synchronize()
+        buf.check_status()
+        states = {l: buf.level_state(l) for l in range(1, w.levels + 1)}
+        for b in range(w.batch):
+            N = lens0[b] + step + 1
+            assert int(dev.lens[b]) == N
+            K_host[b, :, N - 1] = k_new[b]
+            V_host[b, :, N - 1] = v_new[b]
+            for kvh in range(w.n_kv_heads):
+                t = trees[(b, kvh)]
+                orc.tree_update(t, T.np64(K_host[b, kvh, :N]), T.np64(inp.refs[kvh]), N)
+                qg = T.np64(q[b, kvh * G:(kvh + 1) * G])
+                o, r, masks = orc.decode_group(t, qg, T.np64(K_host[b, kvh, :N]), T.np64(V_host[b, kvh, :N]), w.p)
+                flipped, worst = T.compare_routing(r, states, b, kvh, G, N, w, [w.p] * w.levels)
+                flipped_total += len(flipped)
+                got = T.np64(out[b, kvh * G:(kvh + 1) * G])
+                for h in range(G):
+                    if h not in flipped:
+                        assert T.rel_err(got[h], o[h]) <= T.TOL[w.dtype], (step, b, kvh, h)
+    assert flipped_total <= max(2, steps * w.batch * w.n_q_heads // 8)

@@ -135,7 +135,9 @@ def compare_routing(route_o, states, b, kvh, G, N, w: Workload, p_levels):
     sum allow (4 x score error + 1e-5 + fixed_point_band), widened by the
     mass of candidates whose scores are within twice the score error of the
     node's (near ties the two sides may order differently); each one is
-    recorded in FLIPS.
+    recorded in FLIPS. A head is compared down to its first flip: below it
+    the two sides route over different candidate sets (scores of the common
+    candidates are still compared).
     Returns (flipped_heads, max score err)."""
     L = w.levels
     flipped = set()
@@ -157,6 +159,10 @@ def compare_routing(route_o, states, b, kvh, G, N, w: Workload, p_levels):
             sg = score_g[common]
             err = float(np.max(np.abs(sg - so)))
             worst = max(worst, err / max(1.0, float(np.max(np.abs(so)))))
+            if diverged:
+                # after a flip above, the two sides score different candidate
+                # sets at this level: their running masses are not comparable
+                continue
             flips = np.nonzero((kept_g != kept_o) & common)[0]
             if flips.size:
                 p = float(p_levels[level - 1])
