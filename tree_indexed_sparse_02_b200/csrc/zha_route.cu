@@ -1586,24 +1586,27 @@ select_small_kernel(Geo g, LevelWs lw, int level, float p, int32_t *level_kept, 
 // ------------------------------------------------------ fused route: one launch
 //
 // The whole route in one launch, for trees where few nodes are kept per level
-// (trained references): one thread-block cluster per
-// (sequence, KV head) group walks the levels top-down, CTA r owning query
-// row r (16 CTAs per cluster where all the groups' clusters fit on the GPU at
-// once, else 8). Per level: (1) the cluster's CTAs score the group's candidates (each
-// warp two candidates at a time, on the mma.sync scheme of score_mma_kernel,
-// so the scores are the same bits) and deliver row h's scores and extremes to
-// CTA h through distributed shared memory; a cluster barrier; (2) CTA r
-// selects row r with all its threads (the exact selection of the per-level
-// kernels) and ORs its kept bits into every CTA's kept masks; a cluster
-// barrier; (3) every CTA joins the rows into the next level's candidates by
-// itself, so the next level starts without another barrier. The level's
-// candidates and scores are copied out to the workspace views that the
-// per-level launches fill by the CTAs that own no row while the rows select
-// (16-CTA clusters), else after the join. A level with more than kFusedSm candidates goes through the
-// workspace instead (correct at any size, but one warp per row then selects
-// over all of them: the per-level launches are the faster route there).
-// Cluster barriers are hardware barriers that every CTA takes the same
-// number of times, so nothing waits unboundedly.
+// (trained references): one thread-block cluster per (sequence, KV head)
+// group walks the levels top-down, CTA r owning query row r (16 CTAs per
+// cluster where all the groups' clusters fit on the GPU at once, else 8).
+// Per level:
+//   1. the cluster's CTAs score the group's candidates (each warp two
+//      candidates at a time, on the mma.sync scheme of score_mma_kernel, so
+//      the scores are the same bits) and deliver row h's scores and extremes
+//      to CTA h through distributed shared memory; a cluster barrier;
+//   2. CTA r selects row r with all its threads (the exact selection of the
+//      per-level kernels) and ORs its kept bits into every CTA's kept masks;
+//      a cluster barrier;
+//   3. every CTA joins the rows into the next level's candidates by itself,
+//      so the next level starts without another barrier.
+// The level's candidates and scores are copied out to the workspace views
+// that the per-level launches fill -- by the CTAs that own no row while the
+// rows select (16-CTA clusters), else after the join. A level with more than
+// kFusedSm candidates goes through the workspace instead (correct at any
+// size, but one warp per row then selects over all of them: the per-level
+// launches are the faster route there). Cluster barriers are hardware
+// barriers that every CTA takes the same number of times, so nothing waits
+// unboundedly.
 
 constexpr int kFusedSm = 1024;     // candidates per level that a level keeps in shared memory
 constexpr int kFusedPer = kFusedSm / kSmallThreads;
