@@ -812,12 +812,12 @@ __device__ __forceinline__ bool update_range(const Geo &g, const int32_t *lens, 
     return (n_now / g.c) > (n_old / g.c);
 }
 
-// Highest level whose nodes span at most one work item of keys (computed
-// inside the leaf kernel's CTA).
-__host__ __device__ inline int fused_levels(int c, int L) {
+// Highest level whose nodes span at most one work item of item_keys keys
+// (computed inside the leaf kernel's CTA).
+__host__ __device__ inline int fused_levels(int c, int L, int item_keys = kItemKeys) {
     int k = 1;
     int64_t span = (int64_t)c * c;
-    while (k < L && span <= kItemKeys) {
+    while (k < L && span <= item_keys) {
         ++k;
         span *= c;
     }
@@ -825,14 +825,15 @@ __host__ __device__ inline int fused_levels(int c, int L) {
 }
 
 // Bulk leaves of a bf16 cache (tree build and large appends): one CTA per
-// work item of 256 keys (grid.x: items from the one holding the first
+// work item of `tiles` 128-key tiles (two; one when a small update's grid
+// would leave most SMs idle) (grid.x: items from the one holding the first
 // changed leaf; grid.y: groups). Keys come by TMA (3-D tensor map over
 // [group][max_len][d], rows past max_len zero-filled), then the leaf work,
 // then the item's parents up to fused_levels.
 template <typename T, int E, bool MX, int C, bool LARGE>
 __global__ void __launch_bounds__(kLeafWarps * 32, 2)
 tree_leaf_kernel(const __grid_constant__ CUtensorMap kmap, Geo g, TreePtrs tp, const T *K, const T *refs,
-                 const int32_t *lens, int n_new, int32_t *status) {
+                 const int32_t *lens, int n_new, int tiles, int32_t *status) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int grp = blockIdx.y;
@@ -840,18 +841,19 @@ tree_leaf_kernel(const __grid_constant__ CUtensorMap kmap, Geo g, TreePtrs tp, c
     int64_t n_old, n_now;
     if (!update_range(g, lens, b, n_new, n_old, n_now, status)) return;
     const int64_t lo1 = n_old / g.c, hi1 = n_now / g.c;          // changed leaves
-    const int64_t key0 = ((lo1 * g.c) / kItemKeys + blockIdx.x) * kItemKeys;
+    const int item_keys = tiles * kTileRows;
+    const int64_t key0 = ((lo1 * g.c) / item_keys + blockIdx.x) * item_keys;
     if (key0 >= hi1 * g.c) return;
-    const int per_item = kItemKeys / g.c > 0 ? kItemKeys / g.c : 1;
+    const int per_item = item_keys / g.c > 0 ? item_keys / g.c : 1;
     const int64_t leaf0 = key0 / g.c;
     const int store_lo = (int)max64(lo1 - leaf0, 0);
     const int store_hi = (int)min64(hi1 - leaf0, per_item);
-    const LeafLayout Ly = leaf_layout(g.d, g.R, g.c, 2);
+    const LeafLayout Ly = leaf_layout(g.d, g.R, g.c, tiles);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Ly.bar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const uint32_t full = smem_u32(bars), mma_bar = smem_u32(bars + 1);
-    const uint32_t cols = tmem_cols_for(Ly.npad, 2);
+    const uint32_t cols = tmem_cols_for(Ly.npad, tiles);
     if (threadIdx.x == 0) {
         mbar_init(full, 1);
         mbar_init(mma_bar, 1);
@@ -861,9 +863,9 @@ tree_leaf_kernel(const __grid_constant__ CUtensorMap kmap, Geo g, TreePtrs tp, c
     __syncthreads();
     if ((threadIdx.x >> 5) == 0) tc_alloc(tmem_slot, cols);
     if (threadIdx.x == 0) {
-        // two tiles of 128 rows, d/64 boxes of 64 columns each
-        mbar_expect_tx(full, (uint32_t)(2 * kTileRows * g.d * 2));
-        for (int t = 0; t < 2; ++t)
+        // tiles of 128 rows, d/64 boxes of 64 columns each
+        mbar_expect_tx(full, (uint32_t)(tiles * kTileRows * g.d * 2));
+        for (int t = 0; t < tiles; ++t)
             for (int kb = 0; kb < g.d / 64; ++kb)
                 tma_load_3d(smem_u32(smem + Ly.a + t * kTileRows * g.d * 2 + kb * kTileRows * 128), &kmap,
                             kb * 64, (int)(key0 + t * kTileRows), grp, full);
@@ -877,10 +879,10 @@ tree_leaf_kernel(const __grid_constant__ CUtensorMap kmap, Geo g, TreePtrs tp, c
     if (threadIdx.x == 0) {
         if (mbar_wait_bounded(full, 0, kTreeWait, abort, status)) {
             tc_fence_after();
-            leaf_mma(smem_u32(smem + Ly.a), smem_u32(smem + Ly.b), tmem, 2, g.d, Ly.npad, mma_bar);
+            leaf_mma(smem_u32(smem + Ly.a), smem_u32(smem + Ly.b), tmem, tiles, g.d, Ly.npad, mma_bar);
         }
     }
-    const int rows = (int)min64(hi1 * g.c - key0, 2 * kTileRows);
+    const int rows = (int)min64(hi1 * g.c - key0, (int64_t)tiles * kTileRows);
     const bool ok = leaf_item<T, E, MX, C, LARGE>(g, tp, Ly, smem, tmem, mma_bar, abort, grp, leaf0, store_lo,
                                                   store_hi, rows, status);
     tc_fence_before();
@@ -896,7 +898,7 @@ tree_leaf_kernel(const __grid_constant__ CUtensorMap kmap, Geo g, TreePtrs tp, c
     if (!ok) return;
     // the item's parents, level by level (children written by this CTA are
     // visible to it after the barrier)
-    const int kf = fused_levels(g.c, g.L);
+    const int kf = fused_levels(g.c, g.L, item_keys);
     int64_t lo = lo1, first = leaf0, last = leaf0 + per_item;      // item's nodes at the level below
     for (int level = 2; level <= kf; ++level) {
         lo /= g.c;
@@ -1156,18 +1158,33 @@ cudaError_t tree_update_t(const Geo &g, const TreePtrs &tp, const T *K, const T 
     if constexpr (sizeof(T) == 2) {
         CUtensorMap map;
         if (!make_key_map(g, K, &map)) return cudaErrorNotSupported;
-        const int64_t keys = n_new < 0 ? g.cap[1] * g.c : (int64_t)n_new + kItemKeys;
-        const int64_t items = (keys + kItemKeys - 1) / kItemKeys + 1;
+        // items of two tiles; of one where two-tile items would not cover the
+        // SMs (an append to a few sequences): twice the CTAs, each half as long
+        static const int sms = [] {
+            int dev = 0, n = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return 0;
+            return n;
+        }();
+        int item_keys = kItemKeys;
+        auto items_for = [&](int ik) {
+            const int64_t keys = n_new < 0 ? g.cap[1] * g.c : (int64_t)n_new + ik;
+            return (keys + ik - 1) / ik + 1;
+        };
+        if (g.c <= kTileRows && items_for(kItemKeys) * g.groups() <= sms) item_keys = kTileRows;
+        const int64_t items = items_for(item_keys);
         const size_t smem = item_smem(g);
         set_smem_attr<tree_leaf_kernel<T, E, MX, C, LARGE>>(smem);
         {
             ProfScope ps("tree_leaf", st);
             tree_leaf_kernel<T, E, MX, C, LARGE><<<dim3((unsigned)items, g.groups()), kLeafWarps * 32, smem, st>>>(
-                map, g, tp, K, refs, lens, n_new, status);
+                map, g, tp, K, refs, lens, n_new, item_keys / kTileRows, status);
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        return level_launches<T, E, MX, C>(g, tp, K, refs, lens, n_new, fused_levels(g.c, g.L) + 1, status, st);
+        return level_launches<T, E, MX, C>(g, tp, K, refs, lens, n_new, fused_levels(g.c, g.L, item_keys) + 1,
+                                           status, st);
     } else {
         return level_launches<T, E, MX, C>(g, tp, K, refs, lens, n_new, 1, status, st);
     }
