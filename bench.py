@@ -651,30 +651,37 @@ def routing_quality(w, inp, buf, K, refs, lens, q_step, p_levels, with_oracle: b
     return res
 
 
+# The translation unit that holds each profiled kernel (with every header).
+KERNEL_SOURCE = {"score": "zha_route.cu", "select": "zha_route.cu", "join": "zha_route.cu",
+                 "route": "zha_route.cu", "attn": "zha_attn.cu", "tree": "zha_tree.cu"}
+
+
 def traffic_for(kernel: str, alg_bytes_per_launch: float):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source; None otherwise."""
+    the current source of the kernel's translation unit; None otherwise."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         ent = d["kernels"][kernel]
-        if ent.get("source_sha", d.get("source_sha")) != source_sha():
+        unit = KERNEL_SOURCE[kernel.split("[")[0].split("_")[0]]
+        if ent.get("source_sha") != source_sha(unit):
             return None
         return ent["dram_bytes_per_alg_byte"] * alg_bytes_per_launch
     except Exception:
         return None
 
 
-def source_sha():
-    """Hash of the kernel sources with comments and blank space removed (a
-    comment edit does not invalidate counters taken on the same code)."""
+def source_sha(unit: str | None = None):
+    """Hash of a kernel translation unit and every header (all units when
+    None), comments and blank space removed (a comment edit does not
+    invalidate counters taken on the same code)."""
     import hashlib
     import re
     hsh = hashlib.sha256()
     csrc = os.path.join(ROOT, "tree_indexed_sparse_02_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
+        if name.endswith(".cuh") or (name.endswith(".cu") and (unit is None or name == unit)):
             src = open(os.path.join(csrc, name)).read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
             src = re.sub(r"//[^\n]*", "", src)

@@ -53,15 +53,25 @@ def test_source_sha_ignores_comments_only(tmp_path, monkeypatch):
 
 
 def test_traffic_needs_matching_sources(tmp_path, monkeypatch):
+    """A kernel's traffic ratio holds while its own translation unit and the
+    headers are unchanged: another unit's edit leaves it, its own or a
+    header's voids it."""
     csrc = tmp_path / "tree_indexed_sparse_02_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "k.cu").write_text("int f() { return 1; }\n")
+    (csrc / "zha_route.cu").write_text("int f() { return 1; }\n")
+    (csrc / "zha_attn.cu").write_text("int g() { return 1; }\n")
+    (csrc / "zha_common.cuh").write_text("int h();\n")
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    entry = {"dram_bytes_per_alg_byte": 1.25, "dram_bytes": 1.25e9, "alg_bytes": 1e9}
-    (tmp_path / "profiles" / "traffic.json").write_text(
-        json.dumps({"source_sha": bench.source_sha(), "kernels": {"score[l1]": entry}}))
+    entry = {"dram_bytes_per_alg_byte": 1.25, "dram_bytes": 1.25e9, "alg_bytes": 1e9,
+             "source_sha": bench.source_sha("zha_route.cu")}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"kernels": {"score[l1]": entry}}))
     assert bench.traffic_for("score[l1]", 2e9) == pytest.approx(2.5e9)
     assert bench.traffic_for("attn_sparse", 2e9) is None
-    (csrc / "k.cu").write_text("int f() { return 3; }\n")
+    (csrc / "zha_attn.cu").write_text("int g() { return 2; }\n")
+    assert bench.traffic_for("score[l1]", 2e9) == pytest.approx(2.5e9)
+    (csrc / "zha_common.cuh").write_text("int h(int);\n")
+    assert bench.traffic_for("score[l1]", 2e9) is None
+    (csrc / "zha_common.cuh").write_text("int h();\n")
+    (csrc / "zha_route.cu").write_text("int f() { return 3; }\n")
     assert bench.traffic_for("score[l1]", 2e9) is None
