@@ -185,3 +185,43 @@ def test_fused_decode_steps_match_oracle(zha, w):
                     if h not in flipped:
                         assert T.rel_err(got[h], o[h]) <= T.TOL[w.dtype], (step, b, kvh, h)
     assert flipped_total <= max(2, steps * w.batch * w.n_q_heads // 8)
+
+
+@pytest.mark.parametrize("p", [1.0, 0.5])
+def test_fused_route_p_edges(zha, p):
+    """p = 1 keeps every member (the selection's shortcut); p = 0.5 keeps few:
+    both equal the per-level launches bit for bit."""
+    w = dataclasses.replace(CASES[0], name=f"p={p}", p=p)
+    inp = make_inputs(w, capacity=w.context + 64, lens=_lens(w))
+    dev = T.to_device(inp)
+    _, fused, out_f = _routed(zha, w, dev, zha.ZHA_FLAG_FUSED_ROUTE)
+    _, ref, out_r = _routed(zha, w, dev, 0)
+    assert torch.equal(fused.sel["count"], ref.sel["count"])
+    assert torch.equal(fused.sel["level_kept"], ref.sel["level_kept"])
+    assert torch.equal(out_f, out_r)
+
+
+@pytest.mark.parametrize("noise", [0.0, 1e-3])
+def test_fused_route_equal_scores(zha, noise):
+    """Keys that are all equal (every node of a level scores the same: one
+    bucket holding every candidate, more than the ranked list takes, so the
+    warp selection decides, ties by node index) and keys a hair apart (a
+    crowded crossing bucket): the fused route equals the per-level launches
+    bit for bit, level by level."""
+    w = Workload(f"equal keys noise={noise}", 1, 16, 2, 128, 65536, 4, 4, 16, 0.9, 0, "bf16", 47)
+    inp = make_inputs(w, capacity=w.context + 64)
+    g = torch.Generator().manual_seed(3)
+    base = torch.randn(w.head_dim, generator=g)
+    K = base.expand_as(inp.K).clone() + noise * torch.randn(inp.K.shape, generator=g)
+    inp = dataclasses.replace(inp, K=K.to(inp.K.dtype))
+    dev = T.to_device(inp)
+    _, fused, out_f = _routed(zha, w, dev, zha.ZHA_FLAG_FUSED_ROUTE)
+    _, ref, out_r = _routed(zha, w, dev, 0)
+    for level in range(1, w.levels + 1):
+        a, r = fused.level_state(level), ref.level_state(level)
+        assert torch.equal(a["count"], r["count"]), level
+        for kvh in range(w.n_kv_heads):
+            n = int(r["count"][0, kvh])
+            assert torch.equal(a["kept_mask"][0, kvh, :n], r["kept_mask"][0, kvh, :n]), level
+    assert torch.equal(fused.sel["count"], ref.sel["count"])
+    assert torch.equal(out_f, out_r)
