@@ -965,13 +965,13 @@ __device__ __forceinline__ void tree_path_levels(const Geo &g, const TreePtrs &t
                 *abort = 0;
                 asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
             }
-            // keys of the chunk into rows 0 .. c-1 (rows past c are zero)
+            // keys of the chunk into rows 0 .. c-1 (the MMA's other rows are
+            // never read: each row of S depends on its own key row only)
             const int chunks = g.d / 8;
             const T *src = K + ((int64_t)grp * g.max_len + leaf * g.c) * g.d;
-            for (int i = threadIdx.x; i < tiles * kTileRows * chunks; i += blockDim.x) {
+            for (int i = threadIdx.x; i < g.c * chunks; i += blockDim.x) {
                 const int row = i / chunks, j = i % chunks;
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (row < g.c) v = *reinterpret_cast<const uint4 *>(src + (int64_t)row * g.d + j * 8);
+                const uint4 v = *reinterpret_cast<const uint4 *>(src + (int64_t)row * g.d + j * 8);
                 *reinterpret_cast<uint4 *>(smem + Ly.a + (row >> 7) * kTileRows * g.d * 2 +
                                            swz_offset(row & 127, j, kTileRows)) = v;
             }
@@ -984,7 +984,9 @@ __device__ __forceinline__ void tree_path_levels(const Geo &g, const TreePtrs &t
             tc_fence_after();
             const uint32_t tmem = *tmem_slot;
             if (threadIdx.x == 0) leaf_mma(smem_u32(smem + Ly.a), smem_u32(smem + Ly.b), tmem, tiles, g.d, Ly.npad, mma_bar);
-            ok = leaf_item<T, E, MX, C, LARGE>(g, tp, Ly, smem, tmem, mma_bar, abort, grp, leaf, 0, 1, g.c, status);
+            // one leaf: its planes spread over the warps (C = 0: the same
+            // arithmetic as the bulk kernel's register path, plane by plane)
+            ok = leaf_item<T, E, MX, 0, LARGE>(g, tp, Ly, smem, tmem, mma_bar, abort, grp, leaf, 0, 1, g.c, status);
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
