@@ -83,13 +83,19 @@ enum {
      * mma.sync kernel, which streams the summaries at a higher fraction of
      * HBM bandwidth on this path */
     ZHA_FLAG_TCGEN05 = 2,
-    /* route in one launch: one thread-block cluster of 8 CTAs per (sequence,
-     * KV head) walks every level (scores, cluster barrier, selection and join
-     * by the first CTA, cluster barrier). Same selections as the default
-     * per-level launches; the launch pays off when few nodes are kept per
-     * level (trained references), the default when most are. Applies to bf16
-     * trees with native summaries, n_refs 16 and at most 8 query heads per KV
-     * head, single queries; otherwise the default route runs. */
+    /* route in one launch: one thread-block cluster (16 CTAs where every
+     * group's cluster fits on the GPU at once, else 8) per (sequence, KV
+     * head) walks every level -- scoring into the query rows' CTAs through
+     * distributed shared memory, a cluster barrier, each row's exact
+     * selection by its own CTA, a cluster barrier, the join in every CTA.
+     * Same selections, scores and outputs as the default per-level launches,
+     * bit for bit. It pays off when few nodes are kept per level (trained
+     * references: up to ~1,000 candidates per level and group); a level with
+     * more candidates is handled correctly but slowly (one warp per query
+     * row selects over the workspace), and there the default is far faster.
+     * Applies to bf16 trees with native summaries, n_refs 16 and at most 8
+     * query heads per KV head, single queries; otherwise the default route
+     * runs. */
     ZHA_FLAG_FUSED_ROUTE = 4
 };
 
