@@ -550,7 +550,8 @@ def zha_arm(args, w, world, rank, local):
         times, cores, sample = oracle_batch_steps(w, inp, qs, k_new, v_new, W_steps, steps=2)
         res["cpu_baseline"] = {"value": w.batch * len(times) / sum(times), "unit": "tokens/s", "cores": cores,
                                "kind": "oracle", "sample": sample}
-    # the 1M deep tree built by appends (p = 0.9, 0.95, 0.99) and a bounded
+    # the 1M deep tree built by appends (p = 0.9, 0.95, 0.99), the headline
+    # configuration with aligned references on both routes, and a bounded
     # crossover summary against the dense kernel, on this GPU only
     if rank == 0 and world == 1 and not args.no_extras:
         import dataclasses
@@ -560,6 +561,7 @@ def zha_arm(args, w, world, rank, local):
         rec = incremental_record(w1m, steps=5, warmup=3)
         res["config_1m_incremental"] = {k: rec[k] for k in ("config", "append", "per_p", "dense",
                                                             "speedup_vs_dense_p095")}
+        res["selective_256k"] = selective_summary()
         res["crossover"] = crossover_summary()
     if world > 1:
         torch.distributed.barrier()
@@ -862,10 +864,10 @@ def _bytes(w, cand, tokens):
 
 
 def sweep_point(N: int, tree: str, refs_mode: str, steps: int, warmup: int, p_schedule: str = "fixed",
-                summary: str = "native", route: str = "levels"):
+                summary: str = "native", route: str = "levels", workload=None):
     """ZHA decode vs the dense kernel on one identical cache of N tokens (batch
     1, 32/4 heads, d 128): the deep, wide or speed-model tree with random or
-    aligned references. Returns one record."""
+    aligned references (or the given workload). Returns one record."""
     import dataclasses
 
     import torch
@@ -874,7 +876,8 @@ def sweep_point(N: int, tree: str, refs_mode: str, steps: int, warmup: int, p_sc
     from tree_indexed_sparse_02_b200.inputs import decode_stream, make_inputs, sweep_workload
     peak, _ = read_peaks()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    w = dataclasses.replace(sweep_workload(N, tree), refs_mode=refs_mode, p_schedule=p_schedule, summary=summary)
+    w = dataclasses.replace(workload if workload is not None else sweep_workload(N, tree), refs_mode=refs_mode,
+                            p_schedule=p_schedule, summary=summary)
     n, W = steps, warmup
     cap = N + n + W + 8
     inp = make_inputs(w, device="cuda", capacity=cap)
@@ -889,8 +892,8 @@ def sweep_point(N: int, tree: str, refs_mode: str, steps: int, warmup: int, p_sc
     dense_ms = _timed_dense(zha, cfg, buf, qs[0], inp.K, inp.V, inp.lens, out, flush, n, W)
     us = ms / n * 1e3
     touched = _bytes(w, cand, toks)
-    rec = {"mode": "sweep", "tree": tree, "refs": refs_mode, "route": route, "context": N, "p": w.p,
-           "summary": w.summary,
+    rec = {"mode": "sweep", "tree": tree, "refs": refs_mode, "route": route, "context": N, "batch": w.batch,
+           "p": w.p, "summary": w.summary,
            "p_schedule": w.p_schedule, "zha_us_per_step": us, "dense_us_per_step": dense_ms * 1e3,
            "speedup_vs_dense": dense_ms * 1e3 / us,
            "keys_attended": toks / (w.batch * w.n_kv_heads * (N + W + n)),
@@ -911,6 +914,22 @@ def sweep_mode(args):
             for N in Ns:
                 print(json.dumps(sweep_point(N, tree, refs_mode, args.steps, args.warmup, args.p_schedule,
                                              args.summary, args.route)), flush=True)
+
+
+def selective_summary(steps: int = 10, warmup: int = 3):
+    """The headline configuration (256K deep tree, B=4) with aligned
+    references -- the selective regime trained references give -- on the
+    per-level and on the fused route, each against the dense kernel on the
+    same cache."""
+    from tree_indexed_sparse_02_b200.inputs import DEEP_256K
+    rows = []
+    for route in ("levels", "fused"):
+        r = sweep_point(DEEP_256K.context, "deep", "aligned", steps, warmup, route=route, workload=DEEP_256K)
+        rows.append({k: r[k] for k in ("route", "zha_us_per_step", "dense_us_per_step", "speedup_vs_dense",
+                                       "keys_attended", "touched_frac_of_hbm")})
+        rows[-1]["tokens_per_s"] = DEEP_256K.batch / (r["zha_us_per_step"] / 1e6)
+    return {"workload": DEEP_256K.name, "refs": "aligned", "steps": steps, "warmup": warmup,
+            "l2": "flushed before every timed step", "points": rows}
 
 
 def crossover_summary(steps: int = 5, warmup: int = 3):
