@@ -282,12 +282,19 @@ class DecodeGraph:
                    buf.workspace, buf.status)
         self.kernels_per_step = launch_count() - before
 
-    def step(self, q, k_new, v_new):
-        self.q.copy_(q, non_blocking=True)
-        self.k_new.copy_(k_new, non_blocking=True)
-        self.v_new.copy_(v_new, non_blocking=True)
+    def stage(self, q, k_new, v_new):
+        """Put a step's inputs into the graph's own buffers (one multi-tensor
+        copy); a caller that produces them there directly skips this."""
+        torch._foreach_copy_([self.q, self.k_new, self.v_new], [q, k_new, v_new], non_blocking=True)
+
+    def replay(self):
+        """One decode step on the inputs in the graph's buffers."""
         self.graph.replay()
         return self.out
+
+    def step(self, q, k_new, v_new):
+        self.stage(q, k_new, v_new)
+        return self.replay()
 
 
 class Buffers:
