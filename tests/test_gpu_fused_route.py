@@ -225,3 +225,22 @@ def test_fused_route_equal_scores(zha, noise):
             assert torch.equal(a["kept_mask"][0, kvh, :n], r["kept_mask"][0, kvh, :n]), level
     assert torch.equal(fused.sel["count"], ref.sel["count"])
     assert torch.equal(out_f, out_r)
+
+
+def test_fused_flag_with_other_options(zha):
+    """The fused flag next to the tcgen05 scorer flag (the fused route runs)
+    and with MX-FP8 summaries (outside the fused route's scope: the per-level
+    route runs): each equals the per-level route of the same configuration
+    bit for bit."""
+    w = CASES[0]
+    inp = make_inputs(w, capacity=w.context + 64, lens=_lens(w))
+    dev = T.to_device(inp)
+    _, a, out_a = _routed(zha, w, dev, zha.ZHA_FLAG_FUSED_ROUTE | zha.ZHA_FLAG_TCGEN05)
+    _, r, out_r = _routed(zha, w, dev, 0)
+    assert torch.equal(a.sel["count"], r.sel["count"])
+    assert torch.equal(out_a, out_r)
+    wm = dataclasses.replace(w, name="mx", summary="mxfp8")
+    _, a, out_a = _routed(zha, wm, dev, zha.ZHA_FLAG_FUSED_ROUTE)
+    _, r, out_r = _routed(zha, wm, dev, 0)
+    assert torch.equal(a.sel["count"], r.sel["count"])
+    assert torch.equal(out_a, out_r)
