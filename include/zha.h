@@ -93,9 +93,10 @@ enum {
      * references: up to ~1,000 candidates per level and group); a level with
      * more candidates is handled correctly but slowly (one warp per query
      * row selects over the workspace), and there the default is far faster.
-     * Applies to bf16 trees with native summaries, n_refs 16 and at most 8
-     * query heads per KV head, single queries; otherwise the default route
-     * runs. */
+     * Applies to bf16 trees with native summaries, n_refs 16, at most 8
+     * query heads per KV head and at most 1,024 top-level nodes at max_len
+     * (the top level is scored whole), single queries; otherwise the default
+     * route runs. */
     ZHA_FLAG_FUSED_ROUTE = 4
 };
 

@@ -54,6 +54,11 @@ Geo make_geo(const zha_config *c, int T = 1) {
     g.R = c->n_refs;
     g.dtype = c->dtype;
     g.flags = c->flags;
+    // The fused route scores the top level whole in a cluster's shared memory
+    // (up to 1,024 candidates a level); a tree whose top level can outgrow
+    // that takes the per-level route, which is the faster one there.
+    constexpr int64_t kFusedTopNodes = 1024;
+    if (zha::level_nodes(c->max_len, c->chunk, c->levels) > kFusedTopNodes) g.flags &= ~ZHA_FLAG_FUSED_ROUTE;
     g.summary = c->summary;
     g.max_len = c->max_len;
     g.s = c->scale > 0.f ? c->scale : 1.f / sqrtf((float)c->head_dim);
