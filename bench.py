@@ -447,7 +447,7 @@ def zha_arm(args, w, world, rank, local):
            "candidates_per_level": [float(h[:, l, :].sum(dim=1).mean()) for l in range(w.levels)],
            "attended_tokens_per_step": float(attn_tokens.mean()),
            "gpu_launches": int(launches), "cuda_graph": graph is not None, "scorer": args.scorer,
-           "route": args.route,
+           "route": args.route, "route_run": "fused" if zha.route_fused(cfg) else "levels",
            "clocks": clocks}
 
     # per-kernel CUDA-event timing: a second pass of K steps, every launch bracketed
@@ -901,7 +901,8 @@ def sweep_point(N: int, tree: str, refs_mode: str, steps: int, warmup: int, p_sc
     dense_ms = _timed_dense(zha, cfg, buf, qs[0], inp.K, inp.V, inp.lens, out, flush, n, W)
     us = ms / n * 1e3
     touched = _bytes(w, cand, toks)
-    rec = {"mode": "sweep", "tree": tree, "refs": refs_mode, "route": route, "context": N, "batch": w.batch,
+    rec = {"mode": "sweep", "tree": tree, "refs": refs_mode, "route": route,
+           "route_run": "fused" if zha.route_fused(cfg) else "levels", "context": N, "batch": w.batch,
            "p": w.p, "summary": w.summary,
            "p_schedule": w.p_schedule, "zha_us_per_step": us, "dense_us_per_step": dense_ms * 1e3,
            "speedup_vs_dense": dense_ms * 1e3 / us,
@@ -934,7 +935,7 @@ def selective_summary(steps: int = 10, warmup: int = 3):
     rows = []
     for route in ("levels", "fused"):
         r = sweep_point(DEEP_256K.context, "deep", "aligned", steps, warmup, route=route, workload=DEEP_256K)
-        rows.append({k: r[k] for k in ("route", "zha_us_per_step", "dense_us_per_step", "speedup_vs_dense",
+        rows.append({k: r[k] for k in ("route", "route_run", "zha_us_per_step", "dense_us_per_step", "speedup_vs_dense",
                                        "keys_attended", "touched_frac_of_hbm")})
         rows[-1]["tokens_per_s"] = DEEP_256K.batch / (r["zha_us_per_step"] / 1e6)
     return {"workload": DEEP_256K.name, "refs": "aligned", "steps": steps, "warmup": warmup,
@@ -950,7 +951,7 @@ def crossover_summary(steps: int = 5, warmup: int = 3):
         for refs_mode, route in (("random", "levels"), ("aligned", "levels"), ("aligned", "fused")):
             for N in (65536, 131072, 524288):
                 r = sweep_point(N, tree, refs_mode, steps, warmup, route=route)
-                rows.append({k: r[k] for k in ("tree", "refs", "route", "context", "zha_us_per_step",
+                rows.append({k: r[k] for k in ("tree", "refs", "route", "route_run", "context", "zha_us_per_step",
                                                "dense_us_per_step", "speedup_vs_dense", "keys_attended",
                                                "touched_frac_of_hbm")})
     return {"steps": steps, "warmup": warmup, "batch": 1, "l2": "flushed before every timed step", "points": rows}

@@ -180,6 +180,15 @@ ZHA_API zha_status zha_check_config(const zha_config *cfg);
  * (only complete chunks enter the tree), n_l = ceil(n_{l-1} / c). */
 ZHA_API int64_t zha_level_nodes(const zha_config *cfg, int64_t n_tokens, int32_t level);
 
+/* Which routing a call with this configuration runs (host only, no GPU
+ * work): *fused = 1 if zha_route, zha_decode (T = 1) and zha_decode_block
+ * with T query positions score all levels in the one fused launch, 0 if they
+ * launch per level. The fused launch needs ZHA_FLAG_FUSED_ROUTE and the
+ * configuration that flag's description lists; any other configuration,
+ * flag set or not, routes per level. ZHA_ERR_INVALID_ARG for a bad config,
+ * T < 1 or a null `fused`. */
+ZHA_API zha_status zha_route_fused(const zha_config *cfg, int32_t T, int32_t *fused);
+
 /* Bytes of the tree buffer for cfg->max_len tokens per sequence, and the
  * byte offsets of level l's arrays inside it:
  *   mu   [batch][n_kv_heads][cap_l][n_refs][head_dim]  dtype (summary keys),

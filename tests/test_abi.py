@@ -136,3 +136,39 @@ def test_mx_summary_config_and_layout(zha):
     assert zha.tree_bytes(mx) == pytest.approx(n1 * (2176 + 64), rel=0.01)
     assert zha.tree_bytes(nat) == pytest.approx(n1 * (4160 + 64), rel=0.01)
     assert zha.lib().zha_tree_level_scales(ctypes.byref(nat), 1, ctypes.byref(off)) == 1
+
+
+def test_route_fused_query(zha):
+    """The fused launch runs only with its flag on a bf16 tree with native
+    summaries, 16 planes, at most 8 query rows per group, single queries and
+    a top level of at most 1,024 nodes at max_len; everything else routes per
+    level."""
+    F = zha.ZHA_FLAG_FUSED_ROUTE
+    base = dict(batch=1, n_q_heads=32, n_kv_heads=4, head_dim=128, chunk=4, levels=6, n_refs=16, dtype="bf16",
+                max_len=(1 << 18) + 64, flags=F)
+
+    def fused(T=1, **kw):
+        args = dict(base)
+        args.update(kw)
+        return zha.route_fused(zha.config(**args), T)
+
+    assert fused()                                   # 256K deep: 64 top-level nodes
+    assert fused(head_dim=64)
+    assert fused(n_q_heads=16)                       # 4 rows per group
+    assert not fused(flags=0)
+    assert not fused(dtype="f32")
+    assert not fused(summary="mxfp8")
+    assert not fused(n_refs=8)
+    assert not fused(n_q_heads=64)                   # 16 rows per group
+    assert not fused(T=2)
+    # top level at max_len: 1,024 nodes fused, one more per level below is not
+    assert fused(max_len=4 * 1024 * 4 ** 5)
+    assert not fused(max_len=4 * 1024 * 4 ** 5 + 4 ** 6 * 4)
+    assert not fused(max_len=4 * 1024 * 4 ** 5 + 4 ** 6)
+    # a one-level tree of 256-token chunks outgrows 1,024 nodes past 256K tokens
+    assert fused(chunk=256, levels=1, max_len=1 << 18)
+    assert not fused(chunk=256, levels=1, max_len=(1 << 18) + 256)
+    cfg = zha.config(**base)
+    with pytest.raises(zha.ZhaError):
+        zha.route_fused(cfg, 0)
+    assert zha.lib().zha_route_fused(ctypes.byref(cfg), 1, None) == 1

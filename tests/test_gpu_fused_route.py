@@ -244,3 +244,29 @@ def test_fused_flag_with_other_options(zha):
     _, r, out_r = _routed(zha, wm, dev, 0)
     assert torch.equal(a.sel["count"], r.sel["count"])
     assert torch.equal(out_a, out_r)
+
+
+@pytest.mark.parametrize("flags,dtype,max_len,fused", [(4, "bf16", 16384, True), (0, "bf16", 16384, False),
+                                                       (4, "f32", 16384, False), (4, "bf16", 16400, False)])
+def test_route_fused_query_names_the_launch(zha, flags, dtype, max_len, fused):
+    """zha_route_fused says which routing zha_route runs: the fused kernel
+    appears in the launch record exactly when it answers 1 (a two-level tree
+    of 4-token chunks has 1,024 top-level nodes at 16,384 tokens and 1,025 at
+    16,400, where it routes per level)."""
+    w = Workload("query", 1, 32, 4, 128, 3000, 4, 2, 16, 0.95, 16, dtype, 13, refs_mode="aligned")
+    inp = T.to_device(make_inputs(w, capacity=max_len))
+    cfg = T.make_cfg(zha, w, max_len, flags=flags)
+    assert zha.route_fused(cfg) == fused
+    buf = zha.Buffers(cfg)
+    zha.tree_build(cfg, buf.tree, inp.K, inp.refs, inp.lens, buf.status)
+    torch.cuda.synchronize()
+    zha.profile_read()
+    zha.profile_enable(True)
+    try:
+        zha.route(cfg, buf.tree, inp.q, inp.lens, w.p, buf.sel, buf.workspace, buf.status)
+        torch.cuda.synchronize()
+        names = zha.profile_read()
+    finally:
+        zha.profile_enable(False)
+    buf.check_status()
+    assert ("route_fused" in names) == fused, sorted(names)

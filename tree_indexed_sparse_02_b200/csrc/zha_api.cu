@@ -178,6 +178,15 @@ int64_t zha_level_nodes(const zha_config *cfg, int64_t n_tokens, int32_t level) 
     return zha::level_nodes(n_tokens, cfg->chunk, level);
 }
 
+zha_status zha_route_fused(const zha_config *cfg, int32_t T, int32_t *fused) {
+    zha_status s = check_config(cfg);
+    if (s != ZHA_OK) return s;
+    if (T < 1 || !fused) return ZHA_ERR_INVALID_ARG;
+    const Geo g = make_geo(cfg, T);
+    *fused = (g.flags & ZHA_FLAG_FUSED_ROUTE) && zha::fused_route_supported(g) ? 1 : 0;
+    return ZHA_OK;
+}
+
 size_t zha_tree_bytes(const zha_config *cfg) {
     if (check_config(cfg) != ZHA_OK) return 0;
     return make_geo(cfg).tree_bytes;

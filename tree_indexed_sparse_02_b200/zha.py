@@ -70,6 +70,7 @@ def _load():
         "zha_status_string": ([i32], ctypes.c_char_p),
         "zha_check_config": ([CP], i32),
         "zha_level_nodes": ([CP, i64, i32], i64),
+        "zha_route_fused": ([CP, i32, ctypes.POINTER(i32)], i32),
         "zha_tree_bytes": ([CP], sz),
         "zha_tree_level_offsets": ([CP, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)], i32),
         "zha_tree_level_scales": ([CP, i32, ctypes.POINTER(sz)], i32),
@@ -133,6 +134,13 @@ def _stream(stream):
 
 def level_nodes(cfg: Config, n_tokens: int, level: int) -> int:
     return int(_lib.zha_level_nodes(ctypes.byref(cfg), int(n_tokens), int(level)))
+
+
+def route_fused(cfg: Config, T: int = 1) -> bool:
+    """True if routing with cfg (T query positions) runs the fused launch."""
+    out = ctypes.c_int32(0)
+    check(_lib.zha_route_fused(ctypes.byref(cfg), int(T), ctypes.byref(out)), "zha_route_fused")
+    return bool(out.value)
 
 
 def tree_bytes(cfg: Config) -> int:
