@@ -185,7 +185,7 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t 
 }
 
 template <int D>
-constexpr int attn_smem_bytes() {
+__host__ __device__ constexpr int attn_smem_bytes() {
     return kStages * 2 * kTile * D * 2;
 }
 
@@ -193,8 +193,11 @@ constexpr int attn_smem_bytes() {
 // group's token list (K and V rows, gathered by position) into a 3-stage
 // shared-memory ring with cp.async; rows are stored with their 16-byte
 // chunks XOR-swizzled by (row & 7) so that ldmatrix reads of 8 rows at one
-// column are bank-conflict free. Each warp then computes its 16 tokens.
-template <int D>
+// column are bank-conflict free. Each warp then computes its 16 tokens for
+// MT tiles of 16 query rows (MT = 2 for groups of more than 16 rows: a
+// block of several query positions), so each K/V fragment read from shared
+// memory serves all of them and the group's K/V cross DRAM once.
+template <int D, int MT>
 __global__ void __launch_bounds__(kAttnWarps * 32)
 attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __nv_bfloat16 *V,
                 const int32_t *lens, zha_selection sel, int dense, float *part_ml, float *part_o,
@@ -207,30 +210,33 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
 
-    // the 16-row tiles of a (group, split) are adjacent in launch order, so
-    // with more than 16 rows their CTAs stream the same K/V at about the same
-    // time and the second read comes from L2
+    constexpr int RB = 16 * MT;            // query rows per CTA
     const int grp = blockIdx.z, split = blockIdx.y, S = gridDim.y;
-    const int rbase = blockIdx.x * 16;     // this CTA's 16 query rows of the group
+    const int rbase = blockIdx.x * RB;     // this CTA's query rows of the group
     const int b = grp / g.Hkv, kvh = grp % g.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gq = lane >> 2, t = lane & 3;
     const __nv_bfloat16 *Kg = K + (int64_t)grp * g.max_len * D;
     const __nv_bfloat16 *Vg = V + (int64_t)grp * g.max_len * D;
 
-    // Q as the A operand: rows gq and gq+8 are query rows of this group (rows >= G are zero)
-    uint32_t qf[D / 16][4];
-    const int h0 = rbase + gq, h1 = rbase + gq + 8;
-    {
+    // Q as the A operand: in m-tile mt, rows gq and gq+8 are query rows
+    // rbase + 16 mt + gq (+8) of this group (rows >= G are zero)
+    uint32_t qf[MT][D / 16][4];
+    uint32_t mrow[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int h0 = rbase + 16 * mt + gq, h1 = h0 + 8;
         const uint32_t *q0 = reinterpret_cast<const uint32_t *>(q + g.qrow(b, kvh, h0 < g.G ? h0 : 0) * D);
         const uint32_t *q1 = reinterpret_cast<const uint32_t *>(q + g.qrow(b, kvh, h1 < g.G ? h1 : 0) * D);
 #pragma unroll
         for (int st = 0; st < D / 16; ++st) {
-            qf[st][0] = h0 < g.G ? q0[st * 8 + t] : 0u;
-            qf[st][1] = h1 < g.G ? q1[st * 8 + t] : 0u;
-            qf[st][2] = h0 < g.G ? q0[st * 8 + 4 + t] : 0u;
-            qf[st][3] = h1 < g.G ? q1[st * 8 + 4 + t] : 0u;
+            qf[mt][st][0] = h0 < g.G ? q0[st * 8 + t] : 0u;
+            qf[mt][st][1] = h1 < g.G ? q1[st * 8 + t] : 0u;
+            qf[mt][st][2] = h0 < g.G ? q0[st * 8 + 4 + t] : 0u;
+            qf[mt][st][3] = h1 < g.G ? q1[st * 8 + 4 + t] : 0u;
         }
+        mrow[mt][0] = h0 < g.G ? (1u << h0) : 0u;
+        mrow[mt][1] = h1 < g.G ? (1u << h1) : 0u;
     }
     // the queries are the call's input; the cache, lengths and selection come from earlier kernels
     pdl_wait();
@@ -302,12 +308,15 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
     };
 
     const float sl2 = g.s * kLog2e;
-    float m_run[2] = {-INFINITY, -INFINITY};
-    float l_run[2] = {0.f, 0.f};
-    float o[NJ][4];
+    float m_run[MT][2], l_run[MT][2];
+    float o[MT][NJ][4];
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-    const uint32_t mrow[2] = {h0 < g.G ? (1u << h0) : 0u, h1 < g.G ? (1u << h1) : 0u};
+    for (int mt = 0; mt < MT; ++mt) {
+        m_run[mt][0] = m_run[mt][1] = -INFINITY;
+        l_run[mt][0] = l_run[mt][1] = 0.f;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) o[mt][j][0] = o[mt][j][1] = o[mt][j][2] = o[mt][j][3] = 0.f;
+    }
 
     // Commit groups: the prologue's lookups of tiles t_lo .. t_lo + kAhead - 1
     // (waited for at once), then one group per tile of the first kStages - 1
@@ -349,106 +358,137 @@ attn_mma_kernel(Geo g, const __nv_bfloat16 *q, const __nv_bfloat16 *K, const __n
         uint32_t mv[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) mv[u] = smask[it % kSlots][row0 + (u >> 1) * 8 + 2 * t + (u & 1)];
-        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+        float s0[MT][4], s1[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) s0[mt][u] = s1[mt][u] = 0.f;
 #pragma unroll
         for (int kp = 0; kp < D / 32; ++kp) {
             uint32_t b0, b1, b2, b3;
             const int ch = 4 * kp + (lane >> 3);
             int row = row0 + (lane & 7);
             ldsm_x4(kb + row * ROWB + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
-            mma16816(s0, qf[2 * kp][0], qf[2 * kp][1], qf[2 * kp][2], qf[2 * kp][3], b0, b1);
-            mma16816(s0, qf[2 * kp + 1][0], qf[2 * kp + 1][1], qf[2 * kp + 1][2], qf[2 * kp + 1][3], b2, b3);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const uint32_t(&qa)[4] = qf[mt][2 * kp];
+                const uint32_t(&qb)[4] = qf[mt][2 * kp + 1];
+                mma16816(s0[mt], qa[0], qa[1], qa[2], qa[3], b0, b1);
+                mma16816(s0[mt], qb[0], qb[1], qb[2], qb[3], b2, b3);
+            }
             row += 8;
             ldsm_x4(kb + row * ROWB + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
-            mma16816(s1, qf[2 * kp][0], qf[2 * kp][1], qf[2 * kp][2], qf[2 * kp][3], b0, b1);
-            mma16816(s1, qf[2 * kp + 1][0], qf[2 * kp + 1][1], qf[2 * kp + 1][2], qf[2 * kp + 1][3], b2, b3);
-        }
-        float x[2][4];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            x[r][0] = (mv[0] & mrow[r]) ? s0[2 * r + 0] * sl2 : -INFINITY;
-            x[r][1] = (mv[1] & mrow[r]) ? s0[2 * r + 1] * sl2 : -INFINITY;
-            x[r][2] = (mv[2] & mrow[r]) ? s1[2 * r + 0] * sl2 : -INFINITY;
-            x[r][3] = (mv[3] & mrow[r]) ? s1[2 * r + 1] * sl2 : -INFINITY;
-        }
-        float p[2][4];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            float mx = fmaxf(fmaxf(x[r][0], x[r][1]), fmaxf(x[r][2], x[r][3]));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(m_run[r], mx);
-            const float corr = (m_run[r] == -INFINITY) ? 0.f : exp2f(m_run[r] - m_new);
-            float ls = 0.f;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                p[r][u] = (x[r][u] == -INFINITY) ? 0.f : exp2f(x[r][u] - m_new);
-                ls += p[r][u];
-            }
-            l_run[r] = l_run[r] * corr + ls;
-            m_run[r] = m_new;
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-                o[j][2 * r] *= corr;
-                o[j][2 * r + 1] *= corr;
+            for (int mt = 0; mt < MT; ++mt) {
+                const uint32_t(&qa)[4] = qf[mt][2 * kp];
+                const uint32_t(&qb)[4] = qf[mt][2 * kp + 1];
+                mma16816(s1[mt], qa[0], qa[1], qa[2], qa[3], b0, b1);
+                mma16816(s1[mt], qb[0], qb[1], qb[2], qb[3], b2, b3);
             }
         }
-        const uint32_t pa0 = pack_bf16(p[0][0], p[0][1]);
-        const uint32_t pa1 = pack_bf16(p[1][0], p[1][1]);
-        const uint32_t pa2 = pack_bf16(p[0][2], p[0][3]);
-        const uint32_t pa3 = pack_bf16(p[1][2], p[1][3]);
+        uint32_t pa[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            float x[2][4];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                x[r][0] = (mv[0] & mrow[mt][r]) ? s0[mt][2 * r + 0] * sl2 : -INFINITY;
+                x[r][1] = (mv[1] & mrow[mt][r]) ? s0[mt][2 * r + 1] * sl2 : -INFINITY;
+                x[r][2] = (mv[2] & mrow[mt][r]) ? s1[mt][2 * r + 0] * sl2 : -INFINITY;
+                x[r][3] = (mv[3] & mrow[mt][r]) ? s1[mt][2 * r + 1] * sl2 : -INFINITY;
+            }
+            float p[2][4];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                float mx = fmaxf(fmaxf(x[r][0], x[r][1]), fmaxf(x[r][2], x[r][3]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float m_new = fmaxf(m_run[mt][r], mx);
+                const float corr = (m_run[mt][r] == -INFINITY) ? 0.f : exp2f(m_run[mt][r] - m_new);
+                float ls = 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    p[r][u] = (x[r][u] == -INFINITY) ? 0.f : exp2f(x[r][u] - m_new);
+                    ls += p[r][u];
+                }
+                l_run[mt][r] = l_run[mt][r] * corr + ls;
+                m_run[mt][r] = m_new;
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    o[mt][j][2 * r] *= corr;
+                    o[mt][j][2 * r + 1] *= corr;
+                }
+            }
+            pa[mt][0] = pack_bf16(p[0][0], p[0][1]);
+            pa[mt][1] = pack_bf16(p[1][0], p[1][1]);
+            pa[mt][2] = pack_bf16(p[0][2], p[0][3]);
+            pa[mt][3] = pack_bf16(p[1][2], p[1][3]);
+        }
 #pragma unroll
         for (int jp = 0; jp < NJ / 2; ++jp) {
             uint32_t b0, b1, b2, b3;
             const int row = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
             const int ch = 2 * jp + (lane >> 4);
             ldsm_x4_t(vb + row * ROWB + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
-            mma16816(o[2 * jp], pa0, pa1, pa2, pa3, b0, b1);
-            mma16816(o[2 * jp + 1], pa0, pa1, pa2, pa3, b2, b3);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                mma16816(o[mt][2 * jp], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b0, b1);
+                mma16816(o[mt][2 * jp + 1], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b2, b3);
+            }
         }
     }
     cp_async_wait<0>();
     __syncthreads();
-    // row sums across the 4 lanes of a row, then the 4 warps' partials via shared memory
+    // row sums across the 4 lanes of a row, then the 4 warps' partials via
+    // shared memory (in the ring's space: [warps][RB] maxima and sums, then
+    // [warps][RB][D + 4] outputs)
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
-        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
-    }
-    float *sm_m = reinterpret_cast<float *>(smem);                 // [warps][16]
-    float *sm_l = sm_m + kAttnWarps * 16;                           // [warps][16]
-    float *sm_o = sm_l + kAttnWarps * 16;                           // [warps][16][D + 4]
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            l_run[mt][r] += __shfl_xor_sync(0xffffffffu, l_run[mt][r], 1);
+            l_run[mt][r] += __shfl_xor_sync(0xffffffffu, l_run[mt][r], 2);
+        }
+    float *sm_m = reinterpret_cast<float *>(smem);                 // [warps][RB]
+    float *sm_l = sm_m + kAttnWarps * RB;                           // [warps][RB]
+    float *sm_o = sm_l + kAttnWarps * RB;                           // [warps][RB][D + 4]
     constexpr int OS = D + 4;
-    if (t == 0) {
-        sm_m[warp * 16 + gq] = m_run[0];
-        sm_m[warp * 16 + gq + 8] = m_run[1];
-        sm_l[warp * 16 + gq] = l_run[0];
-        sm_l[warp * 16 + gq + 8] = l_run[1];
-    }
+    static_assert((2 * kAttnWarps * RB + kAttnWarps * RB * OS) * 4 <= attn_smem_bytes<D>(),
+                  "the epilogue fits in the ring");
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-        sm_o[(warp * 16 + gq) * OS + 8 * j + 2 * t] = o[j][0];
-        sm_o[(warp * 16 + gq) * OS + 8 * j + 2 * t + 1] = o[j][1];
-        sm_o[(warp * 16 + gq + 8) * OS + 8 * j + 2 * t] = o[j][2];
-        sm_o[(warp * 16 + gq + 8) * OS + 8 * j + 2 * t + 1] = o[j][3];
+    for (int mt = 0; mt < MT; ++mt) {
+        const int r0 = warp * RB + 16 * mt + gq;
+        if (t == 0) {
+            sm_m[r0] = m_run[mt][0];
+            sm_m[r0 + 8] = m_run[mt][1];
+            sm_l[r0] = l_run[mt][0];
+            sm_l[r0 + 8] = l_run[mt][1];
+        }
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            sm_o[r0 * OS + 8 * j + 2 * t] = o[mt][j][0];
+            sm_o[r0 * OS + 8 * j + 2 * t + 1] = o[mt][j][1];
+            sm_o[(r0 + 8) * OS + 8 * j + 2 * t] = o[mt][j][2];
+            sm_o[(r0 + 8) * OS + 8 * j + 2 * t + 1] = o[mt][j][3];
+        }
     }
     __syncthreads();
     const int64_t pbase = ((int64_t)grp * S + split) * g.G + rbase;
-    const int rows = min(16, g.G - rbase);
+    const int rows = min(RB, g.G - rbase);
     for (int i = threadIdx.x; i < rows * D; i += blockDim.x) {
         const int h = i / D, dim = i % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, sm_m[w * 16 + h]);
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, sm_m[w * RB + h]);
         float L = 0.f, acc = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < kAttnWarps; ++w) {
-                const float mw = sm_m[w * 16 + h];
+                const float mw = sm_m[w * RB + h];
                 if (mw == -INFINITY) continue;
                 const float f = exp2f(mw - M);
-                L += sm_l[w * 16 + h] * f;
-                acc += sm_o[(w * 16 + h) * OS + dim] * f;
+                L += sm_l[w * RB + h] * f;
+                acc += sm_o[(w * RB + h) * OS + dim] * f;
             }
         }
         part_o[(pbase + h) * D + dim] = acc;
@@ -645,7 +685,10 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
     const int dense = sel == nullptr;
     zha_selection sv{};
     if (sel) sv = *sel;
-    dim3 grid((g.G + 15) / 16, S, g.groups());
+    // bf16: one CTA per 32 query rows when a group has more than 16 (two
+    // m-tiles sharing each K/V fragment), else per 16; fp32: per 16 rows
+    const bool two_tiles = g.dtype == ZHA_BF16 && g.G > 16;
+    dim3 grid(two_tiles ? (g.G + 31) / 32 : (g.G + 15) / 16, S, g.groups());
     const char *attn_name = dense ? "attn_dense" : "attn_sparse";
     if (g.dtype == ZHA_BF16) {
         auto qq = static_cast<const __nv_bfloat16 *>(q);
@@ -657,18 +700,27 @@ cudaError_t launch_attention(const Geo &g, const void *q, const void *K, const v
             int dev = 0;
             cudaGetDevice(&dev);
             if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-                cudaFuncSetAttribute(attn_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                cudaFuncSetAttribute(attn_mma_kernel<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      attn_smem_bytes<128>());
-                cudaFuncSetAttribute(attn_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                cudaFuncSetAttribute(attn_mma_kernel<64, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     attn_smem_bytes<64>());
+                cudaFuncSetAttribute(attn_mma_kernel<128, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     attn_smem_bytes<128>());
+                cudaFuncSetAttribute(attn_mma_kernel<64, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      attn_smem_bytes<64>());
                 attr_set[dev] = true;
             }
             ProfScope ps(attn_name, st);
+            const dim3 blk(kAttnWarps * 32);
             const cudaError_t e = g.d == 128
-                ? launch_pdl(attn_mma_kernel<128>, grid, dim3(kAttnWarps * 32), attn_smem_bytes<128>(), st,
-                             g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status)
-                : launch_pdl(attn_mma_kernel<64>, grid, dim3(kAttnWarps * 32), attn_smem_bytes<64>(), st,
-                             g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status);
+                ? (two_tiles ? launch_pdl(attn_mma_kernel<128, 2>, grid, blk, attn_smem_bytes<128>(), st,
+                                          g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status)
+                             : launch_pdl(attn_mma_kernel<128, 1>, grid, blk, attn_smem_bytes<128>(), st,
+                                          g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status))
+                : (two_tiles ? launch_pdl(attn_mma_kernel<64, 2>, grid, blk, attn_smem_bytes<64>(), st,
+                                          g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status)
+                             : launch_pdl(attn_mma_kernel<64, 1>, grid, blk, attn_smem_bytes<64>(), st,
+                                          g, qq, kk, vv, lens, sv, dense, part_ml, part_o, status));
             if (e != cudaSuccess) return e;
         }
         ProfScope pm("attn_merge", st);
